@@ -1,0 +1,232 @@
+/*
+ * Oracle for the paged KV-cache decode path: plain, slow, fp64, CPU only.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library. It shares no code,
+ * header, table or helper with the CUDA library; the two meet only through
+ * the seeded inputs the tests hand to both.
+ *
+ * What it follows (cited as page title + section):
+ *  - "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
+ *    section 3.1 (分块注意力计算), the paged_attention code: for every page in the
+ *    sequence's page table, score the query against that page; concatenate the
+ *    page scores; softmax(scores / sqrt(dim)); then the output is the sum over
+ *    pages of (that page's slice of the weights) @ (that page).
+ *  - same page, section 2.1 (分页式存储架构): fixed-size pages in one physical
+ *    pool reached through a per-sequence page table.
+ *  - "vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理", section PagedAttention:
+ *    blocks hold the keys and values of a fixed number of tokens (usually 16)
+ *    and need not be contiguous; section KV Cache内存共享: copy-on-write copies a
+ *    shared block before a sequence appends to it.
+ *  - "VLLM ... PageAttention 分页 KV Cache ..." (m.nxbn.cn), section 一: decode
+ *    computes only the new token's K/V, appends it to the cache, then attends.
+ *
+ * Readings where the pages are silent or garbled (each one is listed in the
+ * design notes of the repository):
+ *  - K and V live in two pools [num_blocks][num_kv_heads][block_size][head_dim];
+ *    the printed code uses one tensor for both and leaves seq_id undefined.
+ *  - Only the first context_len tokens count; the printed code scores whole
+ *    pages, which would include unwritten tail slots.
+ *  - The scale is an argument (the configurations pass 1/sqrt(head_dim)).
+ *  - Grouped-query attention: query head h reads KV head h / (H / H_kv).
+ *  - context_len == 0 gives a zero output row.
+ *
+ * Element formats: fp16 is IEEE 754 binary16; bf16 is the upper half of an
+ * IEEE 754 binary32. Both are decoded here from their bit fields.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_F16 = 0, ORACLE_BF16 = 1 };
+
+/* Decode one 16-bit element to double, from the bit-field definitions. */
+double oracle_to_double(uint16_t bits, int dtype)
+{
+    int sign = (bits >> 15) & 1;
+    double mag;
+    if (dtype == ORACLE_F16) {
+        int e = (bits >> 10) & 0x1f;      /* 5-bit exponent, bias 15 */
+        int m = bits & 0x3ff;             /* 10-bit fraction */
+        if (e == 0)
+            mag = ldexp((double)m, -24);  /* subnormal: m * 2^(1-15-10) */
+        else if (e == 31)
+            mag = m ? NAN : INFINITY;
+        else
+            mag = ldexp((double)(m + 1024), e - 25);
+    } else {
+        int e = (bits >> 7) & 0xff;       /* 8-bit exponent, bias 127 */
+        int m = bits & 0x7f;              /* 7-bit fraction */
+        if (e == 0)
+            mag = ldexp((double)m, -133); /* subnormal: m * 2^(1-127-7) */
+        else if (e == 255)
+            mag = m ? NAN : INFINITY;
+        else
+            mag = ldexp((double)(m + 128), e - 134);
+    }
+    return sign ? -mag : mag;
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Paged decode attention.
+ *   out          [num_seqs][num_heads][head_dim]          fp64 result
+ *   q            [num_seqs][num_heads][head_dim]          16-bit elements
+ *   k_pool,v_pool[num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_tables [num_seqs][max_blocks_per_seq]           physical page ids
+ *   context_lens [num_seqs]
+ * num_threads > 0 sets the OpenMP thread count; the (sequence, head) pairs are
+ * independent, so threads only split that outer loop.
+ */
+void oracle_paged_attention(double *out, const uint16_t *q,
+                            const uint16_t *k_pool, const uint16_t *v_pool,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            int num_seqs, int num_heads, int num_kv_heads,
+                            int head_dim, int block_size, int max_blocks_per_seq,
+                            double scale, int dtype, int num_threads)
+{
+    const int group = num_heads / num_kv_heads;
+    const long pairs = (long)num_seqs * num_heads;
+#ifdef _OPENMP
+    if (num_threads > 0)
+        omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long sh = 0; sh < pairs; sh++) {
+        const int s = (int)(sh / num_heads);
+        const int h = (int)(sh % num_heads);
+        const int kvh = h / group;
+        const int n = context_lens[s];
+        double *o = out + (size_t)sh * head_dim;
+        for (int d = 0; d < head_dim; d++)
+            o[d] = 0.0;
+        if (n <= 0)
+            continue;
+
+        double *qd = (double *)malloc(sizeof(double) * head_dim);
+        double *scores = (double *)malloc(sizeof(double) * n);
+        for (int d = 0; d < head_dim; d++)
+            qd[d] = oracle_to_double(q[(size_t)sh * head_dim + d], dtype);
+
+        const int pages = (n + block_size - 1) / block_size;
+        const int32_t *table = block_tables + (size_t)s * max_blocks_per_seq;
+
+        /* Page by page: scores of the query against the page's valid keys,
+           appended in logical order (the concatenation). */
+        for (int i = 0; i < pages; i++) {
+            const size_t page = (size_t)table[i];
+            for (int r = 0; r < block_size; r++) {
+                const int t = i * block_size + r;
+                if (t >= n)
+                    break;
+                const uint16_t *key =
+                    k_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;
+                double dot = 0.0;
+                for (int d = 0; d < head_dim; d++)
+                    dot += qd[d] * oracle_to_double(key[d], dtype);
+                scores[t] = dot;
+            }
+        }
+
+        /* softmax(scale * scores) over the concatenated scores. */
+        double mx = -INFINITY;
+        for (int t = 0; t < n; t++)
+            if (scale * scores[t] > mx)
+                mx = scale * scores[t];
+        double total = 0.0;
+        for (int t = 0; t < n; t++) {
+            scores[t] = exp(scale * scores[t] - mx);
+            total += scores[t];
+        }
+        for (int t = 0; t < n; t++)
+            scores[t] /= total;
+
+        /* Page by page: that page's slice of the weights times its values. */
+        for (int i = 0; i < pages; i++) {
+            const size_t page = (size_t)table[i];
+            for (int r = 0; r < block_size; r++) {
+                const int t = i * block_size + r;
+                if (t >= n)
+                    break;
+                const uint16_t *val =
+                    v_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;
+                for (int d = 0; d < head_dim; d++)
+                    o[d] += scores[t] * oracle_to_double(val[d], dtype);
+            }
+        }
+        free(scores);
+        free(qd);
+    }
+}
+
+/*
+ * Write each new token's K and V rows into its pool slot. slot = block *
+ * block_size + offset; a negative slot means "no write" for that token.
+ * Pure bit copy of the 16-bit elements.
+ */
+void oracle_reshape_and_cache(const uint16_t *k, const uint16_t *v,
+                              uint16_t *k_pool, uint16_t *v_pool,
+                              const int64_t *slot_mapping, int num_tokens,
+                              int num_kv_heads, int head_dim, int block_size)
+{
+    for (int t = 0; t < num_tokens; t++) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; h++) {
+            const size_t src = ((size_t)t * num_kv_heads + h) * head_dim;
+            const size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) * head_dim;
+            for (int d = 0; d < head_dim; d++) {
+                k_pool[dst + d] = k[src + d];
+                v_pool[dst + d] = v[src + d];
+            }
+        }
+    }
+}
+
+/*
+ * Copy-on-write block copies: for each (src, dst) pair in order and each pool,
+ * the whole block dst becomes a byte copy of block src.
+ */
+void oracle_copy_blocks(uint8_t *const *pools, int num_pools,
+                        const int64_t *src_dst_pairs, int num_pairs,
+                        size_t block_bytes)
+{
+    for (int p = 0; p < num_pairs; p++) {
+        const int64_t src = src_dst_pairs[2 * p];
+        const int64_t dst = src_dst_pairs[2 * p + 1];
+        for (int i = 0; i < num_pools; i++)
+            memcpy(pools[i] + (size_t)dst * block_bytes,
+                   pools[i] + (size_t)src * block_bytes, block_bytes);
+    }
+}
+
+/*
+ * Slot of token position pos of a sequence: the page table maps logical page
+ * pos / block_size to a physical page; the slot is that page's first slot plus
+ * the offset inside the page.
+ */
+void oracle_slot_mapping(int64_t *slots, const int32_t *block_tables,
+                         int max_blocks_per_seq, const int32_t *seq_ids,
+                         const int32_t *positions, int n, int block_size)
+{
+    for (int i = 0; i < n; i++) {
+        const int32_t *table = block_tables + (size_t)seq_ids[i] * max_blocks_per_seq;
+        const int pos = positions[i];
+        slots[i] = (int64_t)table[pos / block_size] * block_size + pos % block_size;
+    }
+}

@@ -1,0 +1,274 @@
+"""Pins for the oracle: checks against things other than the oracle itself.
+
+Each ``pin_*`` takes an ``oracle.Oracle`` handle and raises AssertionError on a
+mismatch. ``test_oracle_pins.py`` runs them on the real oracle (all must pass);
+``test_oracle_mutants.py`` runs them on copies of the oracle with one planted
+mistake each (at least one pin must fail for every copy).
+
+What pins what:
+  * element decoding      all 65536 patterns vs numpy float16 / float32 types
+  * paged attention       numpy contiguous-cache brute force; torch SDPA (fp64);
+                          closed forms (1 token -> its V row; equal keys or
+                          scale 0 -> mean of V; a 2-token case with weights
+                          1/(1+e) and e/(1+e)); invariants (physical block
+                          permutation, shared == duplicated blocks, NaN in
+                          unwritten tail slots, GQA head mapping)
+  * cache write / copies  numpy fancy-index scatter and slice copies
+  * slot mapping          enumeration of the contiguous token order
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from tests.bruteforce import bits_of, contiguous_attention, decode, sdpa_attention
+
+ATOL = 1e-12
+
+
+def _rand_bits(rng, shape, dtype):
+    x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32))
+    return bits_of(x.to(torch.float16 if dtype == "f16" else torch.bfloat16))
+
+
+def _case(rng, B, H, Hkv, D, bs, ctx, dtype, extra_blocks=3):
+    """Random pools and a random (scattered) block placement."""
+    need = sum(-(-c // bs) for c in ctx)
+    NB = need + extra_blocks
+    perm = rng.permutation(NB)
+    width = max(1, max(-(-c // bs) for c in ctx))
+    tables = np.full((B, width), -1, dtype=np.int32)
+    k = 0
+    for s, c in enumerate(ctx):
+        for j in range(-(-c // bs)):
+            tables[s, j] = perm[k]
+            k += 1
+    q = _rand_bits(rng, (B, H, D), dtype)
+    kp = _rand_bits(rng, (NB, Hkv, bs, D), dtype)
+    vp = _rand_bits(rng, (NB, Hkv, bs, D), dtype)
+    return q, kp, vp, tables, np.array(ctx, dtype=np.int32)
+
+
+SHAPES = [  # B, H, Hkv, D, bs, ctx, dtype
+    (3, 2, 2, 64, 16, [1, 17, 40], "f16"),
+    (2, 8, 2, 64, 16, [33, 5], "bf16"),
+    (2, 4, 1, 128, 32, [64, 95], "bf16"),
+    (2, 8, 1, 64, 64, [130, 64], "f16"),
+    (4, 6, 3, 16, 16, [16, 31, 2, 48], "f16"),
+]
+
+
+def pin_decode_f16(orc):
+    bits = np.arange(65536, dtype=np.uint16)
+    got = orc.to_double(bits, "f16")
+    ref = decode(bits, "f16")
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+    assert np.array_equal(np.signbit(got[m]), np.signbit(ref[m]))
+
+
+def pin_decode_bf16(orc):
+    bits = np.arange(65536, dtype=np.uint16)
+    got = orc.to_double(bits, "bf16")
+    ref = decode(bits, "bf16")
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+    assert np.array_equal(np.signbit(got[m]), np.signbit(ref[m]))
+    # torch's own bfloat16 -> float64 conversion agrees as well
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(got[m], t[m])
+
+
+def pin_bruteforce(orc, seed=0):
+    rng = np.random.default_rng(seed)
+    for B, H, Hkv, D, bs, ctx, dt in SHAPES:
+        q, kp, vp, tab, cl = _case(rng, B, H, Hkv, D, bs, ctx, dt)
+        scale = 1.0 / math.sqrt(D)
+        got = orc.paged_attention(q, kp, vp, tab, cl, scale, dt)
+        ref = contiguous_attention(decode(q, dt), decode(kp, dt), decode(vp, dt), tab, cl, scale)
+        assert np.abs(got - ref).max() <= ATOL, (B, H, Hkv, D, bs, ctx, dt)
+
+
+def pin_sdpa(orc, seed=1):
+    rng = np.random.default_rng(seed)
+    for B, H, Hkv, D, bs, ctx, dt in SHAPES:
+        q, kp, vp, tab, cl = _case(rng, B, H, Hkv, D, bs, ctx, dt)
+        scale = 0.5 / math.sqrt(D)
+        got = orc.paged_attention(q, kp, vp, tab, cl, scale, dt)
+        ref = sdpa_attention(decode(q, dt), decode(kp, dt), decode(vp, dt), tab, cl, scale)
+        assert np.abs(got - ref).max() <= ATOL
+
+
+def pin_single_token(orc, seed=2):
+    """context_len 1: the softmax of one score is 1, so out is that token's V row."""
+    rng = np.random.default_rng(seed)
+    q, kp, vp, tab, cl = _case(rng, 3, 4, 2, 64, 16, [1, 1, 1], "bf16")
+    got = orc.paged_attention(q, kp, vp, tab, cl, 0.125, "bf16")
+    V = decode(vp, "bf16")
+    for s in range(3):
+        for h in range(4):
+            assert np.array_equal(got[s, h], V[tab[s, 0], h // 2, 0])
+
+
+def pin_equal_keys(orc, seed=3):
+    """Equal keys give equal scores, so every weight is 1/n: out = mean of V.
+    Scale 0 gives the same for any keys."""
+    rng = np.random.default_rng(seed)
+    q, kp, vp, tab, cl = _case(rng, 2, 2, 2, 64, 16, [37, 9], "f16")
+    V = decode(vp, "f16")
+    same = kp.copy()
+    same[:] = kp[0, 0, 0]
+    for keys, scale in ((same, 0.125), (kp, 0.0)):
+        got = orc.paged_attention(q, keys, vp, tab, cl, scale, "f16")
+        for s in range(2):
+            n = int(cl[s])
+            rows = np.stack([V[tab[s, t // 16], :, t % 16, :] for t in range(n)])
+            for h in range(2):
+                assert np.abs(got[s, h] - rows[:, h, :].mean(axis=0)).max() <= ATOL
+
+
+def pin_two_token_closed_form(orc):
+    """q = e0, k0 = 0, k1 = e0, scale 1: scores (0, 1), weights (1, e)/(1 + e)."""
+    D, bs = 16, 16
+    one = np.float16(1.0).view(np.uint16)
+    q = np.zeros((1, 1, D), dtype=np.uint16)
+    q[0, 0, 0] = one
+    kp = np.zeros((2, 1, bs, D), dtype=np.uint16)
+    kp[1, 0, 1, 0] = one                     # token 1 lives in block 1, slot 1
+    vp = np.zeros((2, 1, bs, D), dtype=np.uint16)
+    v0 = np.arange(D, dtype=np.float16)
+    v1 = (-np.arange(D, dtype=np.float16)) * np.float16(0.5)
+    vp[1, 0, 0] = v0.view(np.uint16)
+    vp[1, 0, 1] = v1.view(np.uint16)
+    tab = np.array([[1]], dtype=np.int32)
+    got = orc.paged_attention(q, kp, vp, tab, np.array([2], np.int32), 1.0, "f16")
+    e = math.e
+    want = (v0.astype(np.float64) + e * v1.astype(np.float64)) / (1.0 + e)
+    assert np.abs(got[0, 0] - want).max() <= ATOL
+
+
+def pin_block_permutation(orc, seed=4):
+    """Physical placement is irrelevant: permuting blocks (and the tables with
+    them) gives bit-identical output."""
+    rng = np.random.default_rng(seed)
+    for B, H, Hkv, D, bs, ctx, dt in SHAPES:
+        q, kp, vp, tab, cl = _case(rng, B, H, Hkv, D, bs, ctx, dt)
+        pi = rng.permutation(kp.shape[0])
+        kp2 = np.empty_like(kp)
+        vp2 = np.empty_like(vp)
+        kp2[pi] = kp
+        vp2[pi] = vp
+        tab2 = np.where(tab >= 0, pi[np.maximum(tab, 0)], -1).astype(np.int32)
+        a = orc.paged_attention(q, kp, vp, tab, cl, 0.1, dt)
+        b = orc.paged_attention(q, kp2, vp2, tab2, cl, 0.1, dt)
+        assert np.array_equal(a, b)
+
+
+def pin_shared_equals_duplicated(orc, seed=5):
+    """Two sequences reading the same physical blocks give the same result as when
+    one of them reads a byte copy of those blocks."""
+    rng = np.random.default_rng(seed)
+    q, kp, vp, tab, cl = _case(rng, 2, 4, 2, 64, 16, [45, 45], "bf16", extra_blocks=6)
+    q[1] = q[0]
+    shared = tab.copy()
+    shared[1] = shared[0]
+    dup = tab.copy()
+    for j in range(3):          # sequence 1's own blocks become copies of 0's
+        kp[dup[1, j]] = kp[dup[0, j]]
+        vp[dup[1, j]] = vp[dup[0, j]]
+    a = orc.paged_attention(q, kp, vp, shared, cl, 0.125, "bf16")
+    b = orc.paged_attention(q, kp, vp, dup, cl, 0.125, "bf16")
+    assert np.array_equal(a, b)
+    assert np.array_equal(a[0], a[1])
+
+
+def pin_tail_slots_ignored(orc, seed=6):
+    """Unwritten slots past context_len (NaN here) never reach the output."""
+    rng = np.random.default_rng(seed)
+    for B, H, Hkv, D, bs, ctx, dt in SHAPES:
+        q, kp, vp, tab, cl = _case(rng, B, H, Hkv, D, bs, ctx, dt)
+        a = orc.paged_attention(q, kp, vp, tab, cl, 0.1, dt)
+        nan = np.uint16(0x7e00 if dt == "f16" else 0x7fc0)
+        for s, n in enumerate(cl):
+            if n % bs:
+                b = tab[s, n // bs]
+                kp[b, :, n % bs:, :] = nan
+                vp[b, :, n % bs:, :] = nan
+        b = orc.paged_attention(q, kp, vp, tab, cl, 0.1, dt)
+        assert np.isfinite(b).all() and np.array_equal(a, b)
+
+
+def pin_gqa_mapping(orc):
+    """With H=6, Hkv=3 (groups of 2) and one token, head h returns KV head h//2's V."""
+    D, bs = 16, 16
+    q = np.zeros((1, 6, D), dtype=np.uint16)
+    kp = np.zeros((1, 3, bs, D), dtype=np.uint16)
+    vp = np.zeros((1, 3, bs, D), dtype=np.uint16)
+    for kvh in range(3):
+        vp[0, kvh, 0, :] = np.full(D, kvh + 1, dtype=np.float16).view(np.uint16)
+    got = orc.paged_attention(q, kp, vp, np.array([[0]], np.int32), np.array([1], np.int32),
+                              1.0, "f16")
+    for h in range(6):
+        assert np.array_equal(got[0, h], np.full(D, h // 2 + 1, dtype=np.float64))
+
+
+def pin_empty_context(orc):
+    q, kp, vp, tab, cl = _case(np.random.default_rng(7), 2, 2, 2, 16, 16, [0, 3], "f16")
+    got = orc.paged_attention(q, kp, vp, tab, cl, 0.25, "f16")
+    assert np.array_equal(got[0], np.zeros_like(got[0])) and np.abs(got[1]).sum() > 0
+
+
+def pin_reshape_and_cache(orc, seed=8):
+    rng = np.random.default_rng(seed)
+    NB, Hkv, bs, D, T = 6, 3, 16, 32, 20
+    kp = rng.integers(0, 65536, (NB, Hkv, bs, D), dtype=np.uint16)
+    vp = rng.integers(0, 65536, (NB, Hkv, bs, D), dtype=np.uint16)
+    k = rng.integers(0, 65536, (T, Hkv, D), dtype=np.uint16)
+    v = rng.integers(0, 65536, (T, Hkv, D), dtype=np.uint16)
+    slots = rng.choice(NB * bs, T, replace=False).astype(np.int64)
+    slots[3] = -1                                   # skipped token
+    ek, ev = kp.copy(), vp.copy()
+    keep = slots >= 0
+    ek[slots[keep] // bs, :, slots[keep] % bs, :] = k[keep]
+    ev[slots[keep] // bs, :, slots[keep] % bs, :] = v[keep]
+    orc.reshape_and_cache(k, v, kp, vp, slots)
+    assert np.array_equal(kp, ek) and np.array_equal(vp, ev)
+
+
+def pin_copy_blocks(orc, seed=9):
+    rng = np.random.default_rng(seed)
+    pools = [rng.integers(0, 256, (10, 3, 4, 8), dtype=np.uint8) for _ in range(3)]
+    bb = 3 * 4 * 8
+    pairs = np.array([[1, 7], [4, 2], [1, 9]], dtype=np.int64)
+    want = [p.copy() for p in pools]
+    for w in want:
+        for s, d in pairs:
+            w[d] = w[s]
+    orc.copy_blocks(pools, pairs, bb)
+    for p, w in zip(pools, want):
+        assert np.array_equal(p, w)
+
+
+def pin_slot_mapping(orc, seed=10):
+    rng = np.random.default_rng(seed)
+    bs, B, W = 16, 5, 6
+    tables = rng.permutation(B * W).reshape(B, W).astype(np.int32)
+    seq_ids, positions, want = [], [], []
+    for s in range(B):
+        order = [tables[s, j] * bs + o for j in range(W) for o in range(bs)]  # token order
+        for pos in rng.choice(W * bs, 7, replace=False):
+            seq_ids.append(s)
+            positions.append(int(pos))
+            want.append(order[pos])
+    got = orc.slot_mapping(tables, seq_ids, positions, bs)
+    assert np.array_equal(got, np.array(want, dtype=np.int64))
+
+
+ALL_PINS = [pin_decode_f16, pin_decode_bf16, pin_bruteforce, pin_sdpa, pin_single_token,
+            pin_equal_keys, pin_two_token_closed_form, pin_block_permutation,
+            pin_shared_equals_duplicated, pin_tail_slots_ignored, pin_gqa_mapping,
+            pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_slot_mapping]

@@ -1,0 +1,144 @@
+"""Host block manager and workload builders (CPU only)."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from paged_kv_cache_372_b200 import workloads
+from paged_kv_cache_372_b200.block_manager import BlockManager, OutOfBlocks
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def test_lifo_free_list_matches_pages():
+    g = golden("allocator_lifo.json")
+    bs = 16
+    bm = BlockManager(g["max_pages"], bs)
+    for (seq, pages), want in zip(g["requests"], g["expected"]):
+        if want == "error":
+            with pytest.raises(OutOfBlocks):
+                bm.allocate(seq, pages * bs)
+        else:
+            assert bm.allocate(seq, pages * bs) == want
+
+
+def test_kv_bytes_per_token_matches_pages():
+    g = golden("kv_bytes_per_token.json")
+    wl = workloads.llama7b(0, num_seqs=2)
+    per_layer = wl.num_kv_heads * wl.head_dim * 2 * 2          # K and V, fp16
+    assert wl.num_kv_heads * wl.head_dim == g["hidden"]
+    assert per_layer * g["layers"] == g["bytes_per_token"]
+    toks = int(wl.steps[0].context_lens.sum())
+    assert wl.kv_bytes() == toks * per_layer
+
+
+def test_page_is_4kb():
+    g = golden("page_bytes.json")
+    wl = workloads.llama7b(0, num_seqs=2)
+    assert (wl.block_size, wl.head_dim) == (g["block_size"], g["head_dim"])
+    chunk = wl.k_pool[0, 0].numel() * wl.k_pool.element_size()
+    assert chunk == g["page_bytes"]
+
+
+def test_cow_fork_matches_pages():
+    g = golden("cow_fork.json")
+    bs = 16
+    bm = BlockManager(16, bs)
+    bm.allocate(0, 20)                       # tail block holds 4 of 16 tokens
+    tail = bm.tables[0][-1]
+    for c in range(1, g["beams"] + 1):
+        bm.fork(0, c)
+    bm.free_seq(0)
+    copies, in_place = 0, 0
+    for c in range(1, g["beams"] + 1):
+        r = bm.append_slot(c)
+        if r.cow:
+            assert r.cow[0] == tail
+            copies += 1
+            assert r.slot == r.cow[1] * bs + 4
+        else:
+            assert r.slot == tail * bs + 4
+            in_place += 1
+    assert (copies, in_place) == (g["expected_copies"], g["expected_in_place"])
+    bm.check()
+
+
+def test_full_tail_gets_fresh_block_without_copy():
+    bm = BlockManager(8, 16)
+    bm.allocate(0, 32)
+    bm.fork(0, 1)
+    r0, r1 = bm.append_slot(0), bm.append_slot(1)
+    assert r0.cow is None and r1.cow is None and r0.slot != r1.slot
+    assert r0.slot % 16 == 0 and r1.slot % 16 == 0
+    bm.check()
+
+
+def test_slots_agree_with_oracle_rule():
+    rng = np.random.default_rng(0)
+    bm = BlockManager(64, 16, list(rng.permutation(64)))
+    seqs, pos, slots = [], [], []
+    for s, n in enumerate([1, 15, 16, 17, 40]):
+        bm.allocate(s, 0)
+        for p in range(n):
+            seqs.append(s)
+            pos.append(p)
+            slots.append(bm.append_slot(s).slot)
+    tables = bm.block_table_array(range(5), 4, pad=0)
+    want = oracle.slot_mapping(tables, seqs, pos, 16)
+    assert np.array_equal(np.array(slots), want)
+
+
+def test_free_returns_blocks_and_refcounts_hold():
+    bm = BlockManager(10, 16)
+    bm.allocate(0, 40)
+    bm.fork(0, 1)
+    bm.append_slot(1)
+    bm.free_seq(0)
+    bm.check()
+    bm.free_seq(1)
+    bm.check()
+    assert len(bm.free) == 10
+
+
+def test_tiny_workload_shape():
+    wl = workloads.tiny(0)
+    st = wl.steps[0]
+    assert list(st.context_lens) == [1, 7, 16, 33]
+    assert wl.k_pool.shape == (32, 2, 16, 64) and wl.dtype == "f16"
+    assert st.copy_pairs.shape == (2, 2) and st.slot_mapping.shape == (4,)
+    used = set(st.block_tables[st.block_tables >= 0].tolist())
+    assert set(st.copy_pairs[:, 0].tolist()) <= used
+    assert not (set(st.copy_pairs[:, 1].tolist()) & used)
+    for s, n in enumerate(st.context_lens):
+        last = st.block_tables[s, (n - 1) // 16] * 16 + (n - 1) % 16
+        assert st.slot_mapping[s] == last
+
+
+def test_beam_workload_steps_are_consistent():
+    wl = workloads.beam(0, groups=2, steps=3)
+    for st in wl.steps:
+        B = st.q.shape[0]
+        assert B == 16 and st.slot_mapping.shape == (B,)
+        dst = st.copy_pairs[:, 1]
+        assert len(set(dst.tolist())) == len(dst)
+        assert not (set(dst.tolist()) & set(st.copy_pairs[:, 0].tolist()))
+        for s in range(B):
+            n = int(st.context_lens[s])
+            assert st.slot_mapping[s] == st.block_tables[s, (n - 1) // 16] * 16 + (n - 1) % 16
+    assert sum(len(st.copy_pairs) for st in wl.steps) > 0
+
+
+def test_long_context_prefill_slots_are_free_and_distinct():
+    wl = workloads.long32k(0, num_seqs=2, ctx_len=1024, prefill_tokens=256)
+    st = wl.steps[0]
+    pre = st.slot_mapping[2:]
+    assert len(set(pre.tolist())) == 256
+    used = set(st.block_tables[st.block_tables >= 0].tolist())
+    assert not (set((pre // 64).tolist()) & used)

@@ -1,0 +1,66 @@
+"""Pin strength: copies of the oracle with one planted mistake each must fail a pin.
+
+Each mutation edits a private copy of ``oracle/pa_oracle.c`` under a temporary
+directory and builds it there; the committed oracle is never touched. Only
+mutations that keep every memory access in bounds are planted.
+"""
+import os
+
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+MUTATIONS = {
+    "gqa_mapping": ("const int kvh = h / group;", "const int kvh = h % num_kv_heads;"),
+    "f16_exponent": ("mag = ldexp((double)(m + 1024), e - 25);",
+                     "mag = ldexp((double)(m + 1024), e - 24);"),
+    "bf16_exponent": ("mag = ldexp((double)(m + 128), e - 134);",
+                      "mag = ldexp((double)(m + 128), e - 133);"),
+    "f16_subnormal": ("mag = ldexp((double)m, -24);", "mag = ldexp((double)m, -25);"),
+    "bf16_subnormal": ("mag = ldexp((double)m, -133);", "mag = ldexp((double)m, -132);"),
+    "sign_dropped": ("return sign ? -mag : mag;", "return mag;"),
+    "scale_dropped": ("scores[t] = exp(scale * scores[t] - mx);", "scores[t] = exp(scores[t] - mx);"),
+    "key_index_reversed": ("dot += qd[d] * oracle_to_double(key[d], dtype);",
+                           "dot += qd[d] * oracle_to_double(key[head_dim - 1 - d], dtype);"),
+    "values_from_key_pool": ("v_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;",
+                             "k_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;"),
+    "key_row_swapped": ("k_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;",
+                        "k_pool + ((page * num_kv_heads + kvh) * block_size + (r ^ 1)) * head_dim;"),
+    "no_normalisation": ("scores[t] /= total;", "scores[t] /= 1.0;"),
+    "table_ignored": ("const size_t page = (size_t)table[i];", "const size_t page = (size_t)i;"),
+    "query_head_0": ("qd[d] = oracle_to_double(q[(size_t)sh * head_dim + d], dtype);",
+                     "qd[d] = oracle_to_double(q[(size_t)s * num_heads * head_dim + d], dtype);"),
+    "last_token_dropped": ("const int n = context_lens[s];",
+                           "const int n = context_lens[s] - (context_lens[s] > 1);"),
+    "cache_offset": ("const int64_t offset = slot % block_size;",
+                     "const int64_t offset = (slot + 1) % block_size;"),
+    "cache_head_swapped": ("const size_t src = ((size_t)t * num_kv_heads + h) * head_dim;",
+                           "const size_t src = ((size_t)t * num_kv_heads + (num_kv_heads - 1 - h)) * head_dim;"),
+    "copy_direction": ("const int64_t src = src_dst_pairs[2 * p];\n        const int64_t dst = src_dst_pairs[2 * p + 1];",
+                       "const int64_t src = src_dst_pairs[2 * p + 1];\n        const int64_t dst = src_dst_pairs[2 * p];"),
+    "slot_offset": ("slots[i] = (int64_t)table[pos / block_size] * block_size + pos % block_size;",
+                    "slots[i] = (int64_t)table[pos / block_size] * block_size + (pos + 1) % block_size;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutant_fails_a_pin(name, tmp_path):
+    before, after = MUTATIONS[name]
+    with open(oracle.SOURCE) as f:
+        src = f.read()
+    assert before in src, f"mutation site for {name} not found"
+    mutated = src.replace(before, after)
+    path = os.path.join(tmp_path, "mutant.c")
+    with open(path, "w") as f:
+        f.write(mutated)
+    lib = oracle.build(path, os.path.join(tmp_path, "libmutant.so"), force=True)
+    orc = oracle.Oracle(lib)
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+            break
+    assert failed, f"mutant {name} passed every pin"
