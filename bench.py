@@ -1,0 +1,398 @@
+"""Benchmark of the paged decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama7b|llama3_8b|beam|long32k|tiny] [--seed S]
+
+One step is the whole hot path once over one batch: copy-on-write block
+copies (when the workload has any), the cache write of the step's new tokens,
+and paged decode attention of every sequence. The default workload is the
+LLaMA-7B-shaped decode batch (64 sequences, 32 heads, head_dim 128,
+block_size 16, fp16, contexts uniform in [128, 2048]); its KV cache (~1.1 GB
+read per step) is larger than the 126 MB L2, so no L2 flush is needed.
+
+Under torchrun every rank runs its own replica of the workload on its own GPU
+(weak scaling, no collective on the data path); rank 0 prints one JSON line
+with the max-over-ranks device time.
+
+--impl reference times the fp64 CPU oracle on the host cores over a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: seqs/s and KV GB/s as % of B200 HBM peak, 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama7b")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def describe(wl) -> dict:
+    st = wl.steps[0]
+    ctx = st.context_lens
+    return {"workload": wl.name, "num_seqs": int(len(ctx)), "num_heads": wl.num_heads,
+            "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": wl.block_size,
+            "num_blocks": wl.num_blocks, "context_mean": float(ctx.mean()),
+            "context_min": int(ctx.min()), "context_max": int(ctx.max()),
+            "new_tokens_per_step": int(len(st.slot_mapping)),
+            "copy_pairs_per_step": int(len(st.copy_pairs)),
+            "kv_bytes_per_step": int(wl.kv_bytes()), "steps_in_plan": len(wl.steps),
+            "l2": "no flush: KV read per step (%.2f GB) exceeds the 126 MB L2" % (wl.kv_bytes() / 1e9)
+            if wl.kv_bytes() > 4 * 126e6 else "L2 flushed between steps"}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_372_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the decode kernel from a committed ncu capture,
+    only while the kernel sources are unchanged since that capture."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("source_digest") == source_digest():
+            return e["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = max(mx, float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import paged_kv_cache_372_b200 as pa
+    from paged_kv_cache_372_b200 import build, workloads
+    build.build()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    wl = workloads.build(args.workload, args.seed + rank)
+    st0 = wl.steps[0]
+    B = int(len(st0.context_lens))
+    kp, vp = wl.k_pool.to(dev), wl.v_pool.to(dev)
+    P = wl.partition_size if args.partition is None else args.partition
+    max_ctx = max(int(s.context_lens.max()) for s in wl.steps)
+    ws = pa.alloc_workspace(B, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, max_ctx, P, dev)
+    nsteps = len(wl.steps)
+    dev_steps = []
+    for st in wl.steps:
+        dev_steps.append(dict(
+            q=st.q.to(dev), out=torch.empty_like(st.q, device=dev),
+            tables=torch.from_numpy(st.block_tables).to(dev), ctx=torch.from_numpy(st.context_lens).to(dev),
+            k=st.k_new.to(dev), v=st.v_new.to(dev), slots=torch.from_numpy(st.slot_mapping).to(dev),
+            pairs=torch.from_numpy(st.copy_pairs).to(dev)))
+    stream = torch.cuda.current_stream(dev)
+    max_parts = -(-max_ctx // pa.pa_decode_partition_size(B, wl.num_heads, wl.num_kv_heads, wl.head_dim,
+                                                          wl.block_size, max_ctx, P))
+    launches_per_decode = 2 + (1 if max_parts > 1 else 0)
+
+    def step(i, ev=None):
+        d = dev_steps[i % nsteps]
+        n = 0
+        if d["pairs"].shape[0]:
+            pa.pa_copy_blocks([kp, vp], d["pairs"])
+            n += 1
+        pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
+        n += 1
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_decode(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        return n + launches_per_decode
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert pa.pa_device_errors() == 0
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(dev.index) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches = 0
+    start.record(stream)
+    for i in range(args.steps):
+        launches += step(i, evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    total_ms = start.elapsed_time(stop)
+    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    total_ms = max_over_ranks(total_ms, world)
+    decode_ms_max = max_over_ranks(decode_ms, world)
+    ms_per_step = total_ms / args.steps
+    seqs = B * world
+    value = seqs / (ms_per_step / 1e3)
+
+    kv_bytes = float(np.mean([wl.kv_bytes(i % nsteps) for i in range(args.steps)]))
+    peak, peak_kind = measured_peaks()
+    achieved = kv_bytes / (decode_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": value, "unit": "seqs/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block pool)",
+        "config": describe(wl),
+        "kv_gbs": kv_bytes * world / (ms_per_step * 1e-3) / 1e9,
+        "decode_ms": decode_ms_max,
+        "decode_kv_gbs": achieved,
+        "hbm_frac_of_%s" % peak_kind: achieved / peak,
+        "hbm_frac_of_nominal_8000": achieved / 8000.0,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind,
+                     "kernel": "pa_decode call (plan + attention + merge launches)",
+                     "traffic": profiled_traffic(wl.name)},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_e2e:
+        result["e2e"] = run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world)
+    elif not args.no_e2e:
+        run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world)
+    pa.pa_device_errors()
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(wl)
+    return result
+
+
+def run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world):
+    """Same metric through the public API with host buffers: every step copies its
+    inputs from pinned host memory and reads the output back."""
+    nsteps = len(wl.steps)
+    host = []
+    for st in wl.steps:
+        host.append(dict(q=st.q.pin_memory(), k=st.k_new.pin_memory(), v=st.v_new.pin_memory(),
+                         slots=torch.from_numpy(st.slot_mapping).pin_memory(),
+                         tables=torch.from_numpy(st.block_tables).pin_memory(),
+                         ctx=torch.from_numpy(st.context_lens).pin_memory(),
+                         pairs=torch.from_numpy(st.copy_pairs).pin_memory(),
+                         out=torch.empty_like(st.q).pin_memory()))
+    B = int(len(wl.steps[0].context_lens))
+    h0 = host[0]
+    h2d = sum(h0[k].numel() * h0[k].element_size() for k in ("q", "k", "v", "slots", "tables", "ctx", "pairs"))
+    d2h = h0["out"].numel() * h0["out"].element_size()
+
+    def step(i):
+        h = host[i % nsteps]
+        d = {k: h[k].to(dev, non_blocking=True) for k in ("q", "k", "v", "slots", "tables", "ctx", "pairs")}
+        if d["pairs"].shape[0]:
+            pa.pa_copy_blocks([kp, vp], d["pairs"])
+        pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
+        out = torch.empty_like(d["q"])
+        pa.pa_decode(out, d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws)
+        h["out"].copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for i in range(args.steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b) / args.steps, world)
+    return {"value": B * world / (ms / 1e3), "unit": "seqs/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def oracle_sample(wl, n_seqs):
+    """A bounded slice of the workload's first step for the oracle: n_seqs
+    sequences with their tables, the pools as 16-bit patterns."""
+    from tests.bruteforce import bits_of
+    st = wl.steps[0]
+    return dict(q=bits_of(st.q[:n_seqs]), kp=bits_of(wl.k_pool), vp=bits_of(wl.v_pool),
+                tables=st.block_tables[:n_seqs], ctx=st.context_lens[:n_seqs],
+                k=bits_of(st.k_new), v=bits_of(st.v_new), slots=st.slot_mapping)
+
+
+def cpu_baseline(wl, budget_s=10.0, n_seqs=None):
+    import oracle
+    B = int(len(wl.steps[0].context_lens))
+    n = min(B, n_seqs or B)
+    s = oracle_sample(wl, n)
+    kp, vp = s["kp"].copy(), s["vp"].copy()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.reshape_and_cache(s["k"], s["v"], kp, vp, s["slots"])
+        oracle.paged_attention(s["q"], kp, vp, s["tables"], s["ctx"], wl.scale, wl.dtype)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= 20:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": n / dt, "unit": "seqs/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n} of {B} sequences of the first step (cache write + fp64 attention), "
+                      f"{reps} repetitions, {dt:.3f} s each"}
+
+
+def run_reference(args, world, rank):
+    """The oracle, as it stands, on the host cores: each step is a bounded sample
+    (8 sequences) of the same workload."""
+    import oracle
+    from paged_kv_cache_372_b200 import workloads
+    wl = workloads.build(args.workload, args.seed)
+    B = int(len(wl.steps[0].context_lens))
+    n = min(B, 8)
+    s = oracle_sample(wl, n)
+    kp, vp = s["kp"].copy(), s["vp"].copy()
+
+    def step():
+        oracle.reshape_and_cache(s["k"], s["v"], kp, vp, s["slots"])
+        oracle.paged_attention(s["q"], kp, vp, s["tables"], s["ctx"], wl.scale, wl.dtype)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = n / dt
+    sample = f"{n} of {B} sequences per step (cache write + fp64 attention)"
+    return {"metric": METRIC, "value": value, "unit": "seqs/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": describe(wl),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "seqs/s", "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "seqs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps(run_reference(args, world, rank)), flush=True)
+            return
+        res = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * pa.h — C ABI of the B200 (sm_100a) paged KV-cache decode library.
+ *
+ * Three operations, each enqueued asynchronously on the caller's CUDA stream:
+ *
+ *   pa_decode             paged decode attention: every sequence's one query
+ *                         token attends over its KV cache, which is stored in
+ *                         fixed-size blocks of a global pool and reached through
+ *                         a per-sequence block table.
+ *   pa_reshape_and_cache  writes new tokens' K/V rows into their pool slots.
+ *   pa_copy_blocks        copy-on-write copies of whole blocks.
+ *
+ * Memory layouts (row-major, contiguous, device memory unless stated):
+ *   q, out        [num_seqs][num_heads][head_dim]            fp16 or bf16
+ *   k_pool,v_pool [num_blocks][num_kv_heads][block_size][head_dim]
+ *                 One (block, KV head) chunk is contiguous: block_size*head_dim
+ *                 elements (4 KB at block_size 16, head_dim 128, 16-bit).
+ *   block_tables  [num_seqs][max_blocks_per_seq] int32 physical block ids;
+ *                 entries at or past ceil(context_len/block_size) are never read.
+ *   context_lens  [num_seqs] int32, number of cached tokens, new token included.
+ *   k, v          [num_tokens][num_kv_heads][head_dim]
+ *   slot_mapping  [num_tokens] int64, slot = block * block_size + offset;
+ *                 a negative slot skips that token.
+ *   src_dst_pairs [num_pairs][2] int64 block ids.
+ * Grouped-query attention: query head h reads KV head h / (num_heads / num_kv_heads).
+ *
+ * Supported shapes: head_dim in {64, 128}; block_size in {16, 32, 64};
+ * num_heads % num_kv_heads == 0 with group size in {1, 2, 4, 8}. All device
+ * pointers must be 16-byte aligned. Anything else returns PA_ERR_UNSUPPORTED
+ * (shape) or PA_ERR_INVALID (argument).
+ *
+ * Ownership: the caller owns every buffer, workspace included. The library
+ * allocates no memory, never synchronises except in pa_device_errors(), and
+ * launches only on the given stream (a cudaStream_t; NULL = legacy default).
+ *
+ * Errors: host-side validation returns a status before anything is launched.
+ * A failed launch returns PA_ERR_CUDA (pa_last_error() gives the text).
+ * Kernels never fault on bad indices: a block id, slot or copy pair out of
+ * range is skipped and sets a bit in a per-device error word, and a context
+ * length above the limit is clamped and flagged; read (and clear) the word
+ * with pa_device_errors(). Results are then undefined but memory stays safe.
+ *
+ * Calls on one stream are ordered. Concurrent pa_decode calls on different
+ * streams must use different workspaces.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID = 1,      /* bad argument: null pointer, misalignment, size */
+    PA_ERR_UNSUPPORTED = 2,  /* valid but unsupported shape */
+    PA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    PA_ERR_DEVICE_CHECK = 4  /* pa_device_errors(): a kernel flagged bad input */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the per-device error word (pa_device_errors). */
+#define PA_DEVERR_BLOCK_ID 1u   /* block table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT  2u   /* context_len < 0 or above the limit (clamped) */
+#define PA_DEVERR_SLOT     4u   /* slot_mapping entry >= num_blocks*block_size */
+#define PA_DEVERR_PAIR     8u   /* copy pair id outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT 16u   /* a bounded device-side wait ran out */
+
+/* Opaque CUDA stream handle (cudaStream_t). */
+typedef void *pa_stream_t;
+
+/* Name of a status code. */
+PA_API const char *pa_status_string(int status);
+
+/* Text of the last failure on this host thread ("" if none). */
+PA_API const char *pa_last_error(void);
+
+/*
+ * Paged decode attention.
+ *
+ * Defined by: "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
+ * section 3.1 (分块注意力计算) — walk the sequence's page table, score the query
+ * against each page, softmax(scores * scale) over the concatenation, and sum
+ * each page's weight slice times its values; with blocks and block tables as
+ * in "vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理", section PagedAttention.
+ * Only the first context_lens[s] tokens of sequence s count.
+ *
+ *   out[s][h][:] = sum_t softmax_t(scale * q[s][h] . K_t) V_t,
+ *   K_t = k_pool[block_tables[s][t / block_size]][h / group][t % block_size].
+ *
+ * Long contexts are split into partitions of partition_size tokens whose
+ * partial results (max, sum, unnormalised output) are merged by the
+ * log-sum-exp identity. partition_size = 0 picks one automatically; otherwise
+ * it must be a multiple of 16 and of block_size, with
+ * partition_size / block_size <= 32 and partition_size * group <= 2048.
+ *
+ * max_context_len bounds every context_lens entry (larger ones are clamped and
+ * flagged) and sizes the workspace. scale multiplies q.k (1/sqrt(head_dim) for
+ * standard attention). context_len 0 gives a zero output row.
+ *
+ * workspace: device memory of at least pa_decode_workspace_size(...) bytes,
+ * 256-byte aligned, owned by the caller, contents need no initialisation.
+ * out is fp16/bf16 (dtype), rounded to nearest even from fp32 accumulation.
+ */
+PA_API pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_pool,
+                    const int32_t *block_tables, const int32_t *context_lens,
+                    int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                    int block_size, int max_blocks_per_seq, int num_blocks,
+                    int max_context_len, float scale, int dtype, int partition_size,
+                    void *workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/* Workspace bytes pa_decode needs for these sizes (0 if the shape is invalid). */
+PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                int head_dim, int block_size, int max_context_len,
+                                int partition_size);
+
+/* The partition size pa_decode uses for these arguments (resolves 0 = auto);
+ * returns 0 if the arguments are invalid. */
+PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                             int block_size, int max_context_len, int partition_size);
+
+/*
+ * Cache write: for each token t with slot_mapping[t] >= 0,
+ *   k_pool[slot / block_size][h][slot % block_size][:] = k[t][h][:]  (all h),
+ * and the same for v. Bit copy.
+ *
+ * Defined by: the m.nxbn.cn VLLM explainer, section 一 — decode computes only
+ * the new token's K/V and appends it to the cache; prefill writes all prompt
+ * tokens (section 3.2).
+ *
+ * Precondition: non-negative slots are distinct (two tokens into one slot race).
+ * A slot >= num_blocks*block_size is skipped and flagged (PA_DEVERR_SLOT).
+ */
+PA_API pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void *v_pool,
+                               const int64_t *slot_mapping, int num_tokens,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int num_blocks, int dtype, pa_stream_t stream);
+
+/*
+ * Copy-on-write block copies: for each pair p and each pool i,
+ *   bytes [dst*block_bytes, (dst+1)*block_bytes) of pools[i] become a copy of
+ *   bytes [src*block_bytes, (src+1)*block_bytes).
+ *
+ * Defined by: "vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理", section
+ * KV Cache内存共享 — before a sequence appends into a block shared with others,
+ * a new block is taken, the data copied and the block table updated.
+ *
+ * pools is a HOST array of num_pools device pointers (e.g. K and V of every
+ * layer); src_dst_pairs is DEVICE memory. block_bytes is one block of one
+ * pool (num_kv_heads*block_size*head_dim*element size) and must be a multiple
+ * of 16. Precondition: destination blocks are distinct and no destination is
+ * also a source in the same call (the copies run in parallel). An id outside
+ * [0, num_blocks) skips that pair and sets PA_DEVERR_PAIR.
+ */
+PA_API pa_status pa_copy_blocks(void *const *pools, int num_pools, const int64_t *src_dst_pairs,
+                         int num_pairs, size_t block_bytes, int num_blocks,
+                         pa_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns the current device's error word in
+ * *flags (PA_DEVERR_* bits) and clears it when `clear` is non-zero. Returns
+ * PA_ERR_DEVICE_CHECK when any bit was set, PA_OK otherwise.
+ */
+PA_API pa_status pa_device_errors(unsigned int *flags, int clear, pa_stream_t stream);
+
+/* Number of SMs the library sizes its persistent grids for (current device). */
+PA_API int pa_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,75 @@
+// The two data movers of the paged cache, as 16-byte vector copies.
+//
+//  pa_reshape_kernel     writes each new token's K and V rows into the pool
+//                        slot its slot_mapping entry names (the append of the
+//                        m.nxbn.cn VLLM explainer, section 一).
+//  pa_copy_blocks_kernel copy-on-write copies of whole blocks across a list
+//                        of pools ("vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理",
+//                        section KV Cache内存共享).
+// Both are bit copies. Out-of-range indices are skipped and flagged.
+#pragma once
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+// One thread moves one 16-byte vector of K and the matching vector of V.
+// The flat vector index i over [T][Hkv][D/8] is both the source index and,
+// through the slot, the row and column of the destination.
+__global__ void __launch_bounds__(256) pa_reshape_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                                                         uint4 *__restrict__ k_pool, uint4 *__restrict__ v_pool,
+                                                         const int64_t *__restrict__ slot_mapping,
+                                                         long long total_vectors, int vec_per_row, int num_kv_heads,
+                                                         int block_size, long long num_slots) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vectors; i += stride) {
+        const long long row = i / vec_per_row;  // (token, head)
+        const int vec = (int)(i - row * vec_per_row);
+        const long long t = row / num_kv_heads;
+        const int h = (int)(row - t * num_kv_heads);
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+            raise_error(PA_DEVERR_SLOT);
+            continue;
+        }
+        const int64_t blk = slot / block_size;
+        const int64_t off = slot - blk * block_size;
+        const size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * vec_per_row + vec;
+        const uint4 kv = k[i];
+        const uint4 vv = v[i];
+        k_pool[dst] = kv;
+        v_pool[dst] = vv;
+    }
+}
+
+constexpr int COPY_MAX_POOLS = 64;
+
+struct PoolList {
+    uint4 *ptr[COPY_MAX_POOLS];
+};
+
+// blockIdx.x = pair, blockIdx.y = pool; the CTA copies one whole block.
+__global__ void __launch_bounds__(256) pa_copy_blocks_kernel(PoolList pools, const int64_t *__restrict__ pairs,
+                                                             long long vec_per_block, long long num_blocks) {
+    const int64_t src = pairs[2 * (size_t)blockIdx.x];
+    const int64_t dst = pairs[2 * (size_t)blockIdx.x + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0) raise_error(PA_DEVERR_PAIR);
+        return;
+    }
+    uint4 *base = pools.ptr[blockIdx.y];
+    const uint4 *from = base + (size_t)src * vec_per_block;
+    uint4 *to = base + (size_t)dst * vec_per_block;
+    long long i = threadIdx.x;
+    for (; i + 3 * 256 < vec_per_block; i += 4 * 256) {
+        const uint4 a = from[i], b = from[i + 256], c = from[i + 512], d = from[i + 768];
+        to[i] = a;
+        to[i + 256] = b;
+        to[i + 512] = c;
+        to[i + 768] = d;
+    }
+    for (; i < vec_per_block; i += 256) to[i] = from[i];
+}
+
+}  // namespace pa

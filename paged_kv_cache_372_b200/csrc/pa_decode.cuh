@@ -1,0 +1,598 @@
+// Paged decode attention for sm_100a: three launches per call.
+//
+//  1. pa_plan_kernel   (1 CTA) cuts every sequence into partitions of P tokens
+//     and writes the work list, longest partitions first, so that the
+//     persistent attention kernel finishes with the short ones.
+//  2. pa_decode_kernel (one persistent CTA per SM) — every warp is an
+//     independent worker. It takes (sequence, KV head, partition) units from
+//     the work list with an atomic counter and streams the unit's 16-token K
+//     and V tiles, each one contiguous chunk of the pool, through a private
+//     ring of shared-memory stages filled by 1-D bulk copies (TMA) that
+//     complete on mbarriers. The block-table entries of a unit are loaded
+//     once into lane registers and handed to the copy-issuing lane by a
+//     shuffle. Per unit: K phase (scores of the G query heads of the KV head,
+//     kept in shared memory), exact max, exponentials, V phase (weighted sum).
+//     A unit that is a whole sequence writes the normalised output; otherwise
+//     it writes (max, sum, unnormalised output) partials.
+//  3. pa_merge_kernel  merges the partials of split sequences by the
+//     log-sum-exp identity and writes their outputs.
+//
+// The arithmetic is the definition in "别再让GPU内存拖后腿了：vLLM的PagedAttention
+// 如何像操作系统一样管理KV Cache", section 3.1: scores of the query against every
+// page, softmax over the concatenation with the 1/sqrt(dim) scale, weighted sum
+// of the pages' values. Scores are kept in the log2 domain (q is pre-scaled by
+// scale*log2(e)) and accumulated in fp32.
+#pragma once
+
+#include <math.h>
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+struct DecodeParams {
+    void *out;
+    const void *q;
+    const void *k_pool;
+    const void *v_pool;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    int num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks;
+    int ctx_limit;   // context lengths are clamped to [0, ctx_limit]
+    int partition;   // P, tokens per partition
+    int max_parts;   // ceil(ctx_limit / P)
+    float qscale;    // scale * log2(e)
+    int *counter;    // work-list cursor (reset by the plan kernel)
+    int *num_entries;
+    int4 *entries;   // {seq, partition, tokens, partitions of seq}
+    float2 *ml;      // [seq][head][part] (max in log2 units, sum of weights)
+    float *part_acc; // [seq][head][part][D] unnormalised outputs
+};
+
+// Workspace layout: header (counter, entry count), work list, partials.
+struct WsLayout {
+    size_t entries, ml, acc, total;
+};
+
+inline __host__ __device__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline __host__ __device__ WsLayout ws_layout(int B, int H, int D, int max_parts) {
+    WsLayout L;
+    size_t off = 256;
+    L.entries = off;
+    off = align256(off + sizeof(int4) * (size_t)B * max_parts);
+    L.ml = off;
+    off = align256(off + sizeof(float2) * (size_t)B * H * max_parts);
+    L.acc = off;
+    off = align256(off + sizeof(float) * (size_t)B * H * max_parts * D);
+    L.total = off;
+    return L;
+}
+
+__device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, bool flag) {
+    int c = p.context_lens[s];
+    if (c < 0 || c > p.ctx_limit) {
+        if (flag) raise_error(PA_DEVERR_CONTEXT);
+        c = c < 0 ? 0 : p.ctx_limit;
+    }
+    return c;
+}
+
+// ---- 1. work list -----------------------------------------------------------
+constexpr int PLAN_THREADS = 1024;
+constexpr int PLAN_MAX_BINS = 129;  // tiles per partition <= 128
+
+__global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParams p) {
+    __shared__ int s_bin_count[PLAN_MAX_BINS];
+    __shared__ int s_bin_next[PLAN_MAX_BINS];
+    __shared__ int s_warp[32];
+    __shared__ int s_carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int P = p.partition, tiles = P / 16;
+    for (int i = tid; i < PLAN_MAX_BINS; i += PLAN_THREADS) s_bin_count[i] = 0;
+    if (tid == 0) s_carry = 0;
+    __syncthreads();
+
+    // Pass 1: full partitions in sequence order; histogram of the tails.
+    for (int base = 0; base < p.num_seqs; base += PLAN_THREADS) {
+        const int s = base + tid;
+        const int ctx = s < p.num_seqs ? clamped_context(p, s, true) : 0;
+        const int full = ctx / P, tail = ctx - full * P;
+        if (tail > 0) atomicAdd(&s_bin_count[(tail + 15) >> 4], 1);
+        int incl = full;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(FULL_MASK, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) s_warp[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int w = s_warp[lane];
+            int wi = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(FULL_MASK, wi, o);
+                if (lane >= o) wi += v;
+            }
+            s_warp[lane] = wi - w;
+        }
+        __syncthreads();
+        const int off = s_carry + s_warp[warp] + incl - full;
+        const int nparts = full + (tail > 0);
+        for (int j = 0; j < full; ++j) p.entries[off + j] = make_int4(s, j, P, nparts);
+        __syncthreads();
+        if (tid == PLAN_THREADS - 1) s_carry = off + full;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        int pos = s_carry;
+        for (int b = tiles; b >= 1; --b) {
+            s_bin_next[b] = pos;
+            pos += s_bin_count[b];
+        }
+        *p.num_entries = pos;
+        *p.counter = 0;
+    }
+    __syncthreads();
+    // Pass 2: each sequence's last, partial partition, longest first. An
+    // empty sequence gets no work; its output rows are zeroed here.
+    for (int s = tid; s < p.num_seqs; s += PLAN_THREADS) {
+        const int ctx = clamped_context(p, s, false);
+        const int full = ctx / P, tail = ctx - full * P;
+        if (tail > 0) {
+            const int pos = atomicAdd(&s_bin_next[(tail + 15) >> 4], 1);
+            p.entries[pos] = make_int4(s, full, tail, full + 1);
+        } else if (ctx == 0) {
+            const int nvec = p.num_heads * p.head_dim / 8;
+            uint4 *row = static_cast<uint4 *>(p.out) + (size_t)s * nvec;
+            for (int i = 0; i < nvec; ++i) row[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+// ---- 2. attention -------------------------------------------------------------
+// Lane geometry of the K phase. A 16-token tile row is D elements = NV vectors
+// of 16 bytes. Each lane holds VPL vectors of the row (so G*VPL*8 = 64 query
+// values in registers) for TPL tokens; DG lanes share a token and their
+// partial dot products are summed through a small shared-memory transpose.
+// After it each lane owns R = G/2 (token, head) scores (G = 1: one, shared by
+// a lane pair). DG < 8 rotates each lane's vector order by its token group so
+// that the 8 lanes of a shared-memory phase hit distinct banks.
+template <int D, int G>
+struct Geo {
+    static constexpr int NV = D / 8;
+    static constexpr int VPL = (8 / G < NV / 2) ? 8 / G : NV / 2;
+    static constexpr int DG = NV / VPL;
+    static constexpr int TG = 32 / DG;
+    static constexpr int TPL = 16 / TG;
+    static constexpr int V = TPL * G;
+    static constexpr int R = G >= 2 ? G / 2 : 1;
+    static constexpr bool ROT = DG < 8;
+    static constexpr int EPL = D / 32;  // V phase: elements of a row per lane
+    static constexpr int TILE_BYTES = 16 * D * 2;
+    static constexpr int Q_BYTES = G * D * 2;
+    static constexpr int XROW = (V % 4 == 0) ? V + 4 : V + 1;
+    static constexpr int XTG = DG * XROW + ((V % 4 == 0) ? 16 : 0);
+    static constexpr int XB_BYTES = G >= 2 ? ((TG * XTG * 4 + 15) & ~15) : 0;
+    static_assert(TG * DG == 32 && TPL * TG == 16, "lane geometry");
+    static_assert(G == 1 || V == DG * R, "reduction geometry");
+};
+
+template <int D, int G, int NS>
+__host__ __device__ constexpr int warp_smem_bytes(int partition) {
+    return NS * Geo<D, G>::TILE_BYTES + 2 * Geo<D, G>::Q_BYTES + Geo<D, G>::XB_BYTES + 16 * ((NS * 8 + 15) / 16) +
+           ((partition * G * 4 + 15) & ~15);
+}
+
+constexpr int DECODE_MAX_WARPS = 12;
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
+
+struct Unit {
+    int s, kvh, part, ntok, nparts, ntiles, tbl, slot;
+    bool valid;
+};
+
+template <int D, int G, typename T, int NS>
+__global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(const DecodeParams p) {
+    using Gm = Geo<D, G>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int P = p.partition;
+    const int Hkv = p.num_kv_heads, H = p.num_heads, bs = p.block_size;
+
+    uint8_t *ring = smem + (size_t)warp * warp_smem_bytes<D, G, NS>(P);
+    uint8_t *qbuf = ring + NS * Gm::TILE_BYTES;
+    float *xb = reinterpret_cast<float *>(qbuf + 2 * Gm::Q_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(xb) + Gm::XB_BYTES);
+    float *sc = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 16 * ((NS * 8 + 15) / 16));
+    const uint32_t ring_s = smem_u32(ring), qbuf_s = smem_u32(qbuf), bar_s = smem_u32(bars);
+
+    if (lane == 0) {
+        for (int i = 0; i < NS; ++i) mbar_init(bar_s + 8 * i, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+
+    const T *kpool = static_cast<const T *>(p.k_pool);
+    const T *vpool = static_cast<const T *>(p.v_pool);
+    const T *qg = static_cast<const T *>(p.q);
+    const int total_units = *p.num_entries * Hkv;
+    const uint64_t policy = l2_policy_evict_first();
+
+    // K-phase lane geometry.
+    const int tg = lane / Gm::DG, dg = lane % Gm::DG;
+    int voff[Gm::VPL];
+#pragma unroll
+    for (int c = 0; c < Gm::VPL; ++c)
+        voff[c] = 16 * (dg + Gm::DG * (Gm::ROT ? ((c + tg) % Gm::VPL) : c));
+    const int i_own = G >= 2 ? dg / 2 : 0;
+    const int t_own = tg + Gm::TG * i_own;
+    const int g0 = G >= 2 ? (dg & 1) * Gm::R : 0;
+    const bool owner = G >= 2 || dg == 0;
+
+    auto fetch = [&](Unit &x) {
+        int u = 0;
+        if (lane == 0) u = atomicAdd(p.counter, 1);
+        u = __shfl_sync(FULL_MASK, u, 0);
+        x.valid = u < total_units;
+        if (!x.valid) return;
+        const int e = u / Hkv;
+        x.kvh = u - e * Hkv;
+        const int4 ent = p.entries[e];
+        x.s = ent.x;
+        x.part = ent.y;
+        x.ntok = ent.z;
+        x.nparts = ent.w;
+        x.ntiles = (x.ntok + 15) >> 4;
+        const int nblk = (x.ntok + bs - 1) / bs;
+        x.tbl = lane < nblk ? p.block_tables[(size_t)x.s * p.max_blocks_per_seq + x.part * (P / bs) + lane] : 0;
+    };
+
+    // Issue item `it` of a unit: items [0, ntiles) are its K tiles, the rest
+    // its V tiles; item 0 also brings the unit's G query rows.
+    auto issue = [&](int s, int kvh, int ntiles, int tbl, int qslot, int it, uint32_t stage) {
+        const bool is_v = it >= ntiles;
+        const int tok = 16 * (is_v ? it - ntiles : it);
+        const int bi = tok / bs;
+        const int pb = __shfl_sync(FULL_MASK, tbl, bi);
+        if (lane == 0) {
+            const uint32_t bar = bar_s + 8 * stage;
+            const bool ok = (unsigned)pb < (unsigned)p.num_blocks;
+            if (!ok) raise_error(PA_DEVERR_BLOCK_ID);
+            const uint32_t bytes = (ok ? Gm::TILE_BYTES : 0) + (it == 0 ? Gm::Q_BYTES : 0);
+            fence_proxy_async_smem();
+            if (bytes) {
+                mbar_arrive_expect_tx(bar, bytes);
+                if (ok) {
+                    const T *pool = is_v ? vpool : kpool;
+                    const T *src = pool + (((size_t)pb * Hkv + kvh) * bs + (tok - bi * bs)) * D;
+                    bulk_load(ring_s + stage * Gm::TILE_BYTES, src, Gm::TILE_BYTES, bar, policy);
+                }
+                if (it == 0)
+                    bulk_load(qbuf_s + qslot * Gm::Q_BYTES, qg + ((size_t)s * H + kvh * G) * D, Gm::Q_BYTES, bar,
+                              policy);
+            } else {
+                mbar_arrive(bar);
+            }
+        }
+    };
+
+    Unit cur, nxt;
+    fetch(cur);
+    if (!cur.valid) return;
+    cur.slot = 0;
+    nxt.valid = false;
+    int next_slot = 1;
+    bool prod_on_nxt = false, exhausted = false;
+    int pitem = 0;
+    uint32_t issued = 0, consumed = 0;
+
+    // Issue the producer's next item; open the next unit when the current one
+    // is fully issued (never more than one unit ahead of the consumer).
+    auto produce = [&]() {
+        if (exhausted) return;
+        if (pitem >= 2 * (prod_on_nxt ? nxt.ntiles : cur.ntiles)) {
+            if (prod_on_nxt) return;
+            fetch(nxt);
+            if (!nxt.valid) {
+                exhausted = true;
+                return;
+            }
+            nxt.slot = next_slot;
+            next_slot ^= 1;
+            prod_on_nxt = true;
+            pitem = 0;
+        }
+        if (prod_on_nxt)
+            issue(nxt.s, nxt.kvh, nxt.ntiles, nxt.tbl, nxt.slot, pitem, issued % NS);
+        else
+            issue(cur.s, cur.kvh, cur.ntiles, cur.tbl, cur.slot, pitem, issued % NS);
+        ++pitem;
+        ++issued;
+    };
+
+    // Wait for the consumer's next item; on a timeout flag it, wait (bounded)
+    // for the copies still in flight, and report failure.
+    auto wait_item = [&]() -> bool {
+        const uint32_t stage = consumed % NS, parity = (consumed / NS) & 1;
+        bool ok = mbar_wait_bounded(bar_s + 8 * stage, parity, WAIT_LIMIT_NS);
+        ok = __all_sync(FULL_MASK, ok);
+        if (!ok) {
+            if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+            for (uint32_t c = consumed; c < issued; ++c)
+                mbar_wait_bounded(bar_s + 8 * (c % NS), (c / NS) & 1, WAIT_LIMIT_NS);
+        }
+        return ok;
+    };
+
+    for (int i = 0; i < NS; ++i) produce();
+
+    float qf[G][Gm::VPL * 8];
+    float acc[G][Gm::EPL];
+    float Mg[G], Lg[G];
+
+    for (;;) {
+        // ---------------- K phase: scores of this unit -----------------------
+        float mx[Gm::R];
+#pragma unroll
+        for (int r = 0; r < Gm::R; ++r) mx[r] = -INFINITY;
+        for (int k = 0; k < cur.ntiles; ++k) {
+            if (!wait_item()) return;
+            const uint8_t *tile = ring + (consumed % NS) * Gm::TILE_BYTES;
+            if (k == 0) {
+                const uint8_t *qs = qbuf + cur.slot * Gm::Q_BYTES;
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int c = 0; c < Gm::VPL; ++c) {
+                        float f[8];
+                        unpack8<T>(*reinterpret_cast<const uint4 *>(qs + g * D * 2 + voff[c]), f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) qf[g][c * 8 + e] = f[e] * p.qscale;
+                    }
+            }
+            const int valid = min(16, cur.ntok - 16 * k);
+            float part[Gm::TPL][G];
+#pragma unroll
+            for (int i = 0; i < Gm::TPL; ++i) {
+                const uint8_t *row = tile + (tg + Gm::TG * i) * (D * 2);
+#pragma unroll
+                for (int g = 0; g < G; ++g) part[i][g] = 0.f;
+#pragma unroll
+                for (int c = 0; c < Gm::VPL; ++c) {
+                    float f[8];
+                    unpack8<T>(*reinterpret_cast<const uint4 *>(row + voff[c]), f);
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) part[i][g] = fmaf(qf[g][c * 8 + e], f[e], part[i][g]);
+                }
+            }
+            float sred[Gm::R];
+            if constexpr (G == 1) {
+                float v = part[0][0];
+                v += __shfl_xor_sync(FULL_MASK, v, 1);
+                sred[0] = v;
+            } else {
+                float *xrow = xb + tg * Gm::XTG + dg * Gm::XROW;
+                if constexpr (Gm::V % 4 == 0) {
+#pragma unroll
+                    for (int j = 0; j < Gm::V; j += 4)
+                        *reinterpret_cast<float4 *>(xrow + j) =
+                            make_float4(part[j / G][j % G], part[(j + 1) / G][(j + 1) % G],
+                                        part[(j + 2) / G][(j + 2) % G], part[(j + 3) / G][(j + 3) % G]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < Gm::V; ++j) xrow[j] = part[j / G][j % G];
+                }
+                __syncwarp();
+#pragma unroll
+                for (int r = 0; r < Gm::R; ++r) sred[r] = 0.f;
+#pragma unroll
+                for (int d2 = 0; d2 < Gm::DG; ++d2) {
+                    const float *src = xb + tg * Gm::XTG + d2 * Gm::XROW + dg * Gm::R;
+                    if constexpr (Gm::R == 4) {
+                        const float4 v = *reinterpret_cast<const float4 *>(src);
+                        sred[0] += v.x; sred[1] += v.y; sred[2] += v.z; sred[3] += v.w;
+                    } else if constexpr (Gm::R == 2) {
+                        const float2 v = *reinterpret_cast<const float2 *>(src);
+                        sred[0] += v.x; sred[1] += v.y;
+                    } else {
+                        sred[0] += src[0];
+                    }
+                }
+            }
+            const bool tvalid = t_own < valid;
+#pragma unroll
+            for (int r = 0; r < Gm::R; ++r) {
+                const float s = tvalid ? sred[r] : -INFINITY;
+                mx[r] = fmaxf(mx[r], s);
+                if (owner) sc[(g0 + r) * P + 16 * k + t_own] = s;
+            }
+            ++consumed;
+            __syncwarp();
+            produce();
+        }
+
+        // ---------------- exact max, exponentials, sums ----------------------
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float m = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < Gm::R; ++r)
+                if (g == g0 + r) m = mx[r];
+            Mg[g] = m;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+            for (int g = 0; g < G; ++g) Mg[g] = fmaxf(Mg[g], __shfl_xor_sync(FULL_MASK, Mg[g], o));
+        float mown[Gm::R], ls[Gm::R];
+#pragma unroll
+        for (int r = 0; r < Gm::R; ++r) {
+            ls[r] = 0.f;
+            mown[r] = 0.f;
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                if (g == g0 + r) mown[r] = Mg[g];
+        }
+        if (owner) {
+            for (int k = 0; k < cur.ntiles; ++k) {
+#pragma unroll
+                for (int r = 0; r < Gm::R; ++r) {
+                    float *a = sc + (g0 + r) * P + 16 * k + t_own;
+                    const float e = exp2f(*a - mown[r]);
+                    *a = e;
+                    ls[r] += e;
+                }
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float l = 0.f;
+#pragma unroll
+            for (int r = 0; r < Gm::R; ++r)
+                if (owner && g == g0 + r) l = ls[r];
+            Lg[g] = l;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+            for (int g = 0; g < G; ++g) Lg[g] += __shfl_xor_sync(FULL_MASK, Lg[g], o);
+        __syncwarp();
+
+        // ---------------- V phase: weighted sum of values --------------------
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < Gm::EPL; ++e) acc[g][e] = 0.f;
+        for (int k = 0; k < cur.ntiles; ++k) {
+            if (!wait_item()) return;
+            const uint8_t *tile = ring + (consumed % NS) * Gm::TILE_BYTES;
+            const int valid = min(16, cur.ntok - 16 * k);
+#pragma unroll
+            for (int t4 = 0; t4 < 4; ++t4) {
+                float pq[G][4];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float4 v = *reinterpret_cast<const float4 *>(sc + g * P + 16 * k + 4 * t4);
+                    pq[g][0] = v.x; pq[g][1] = v.y; pq[g][2] = v.z; pq[g][3] = v.w;
+                }
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                    const int t = 4 * t4 + tt;
+                    if (t < valid) {
+                        const uint8_t *src = tile + t * (D * 2) + lane * (Gm::EPL * 2);
+                        float f[Gm::EPL];
+                        if constexpr (Gm::EPL == 4) {
+                            const uint2 raw = *reinterpret_cast<const uint2 *>(src);
+                            const float2 a = Elem<T>::pair(raw.x), b = Elem<T>::pair(raw.y);
+                            f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+                        } else {
+                            const float2 a = Elem<T>::pair(*reinterpret_cast<const uint32_t *>(src));
+                            f[0] = a.x; f[1] = a.y;
+                        }
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+#pragma unroll
+                            for (int e = 0; e < Gm::EPL; ++e) acc[g][e] = fmaf(pq[g][tt], f[e], acc[g][e]);
+                    }
+                }
+            }
+            ++consumed;
+            __syncwarp();
+            produce();
+        }
+
+        // ---------------- store ---------------------------------------------
+        const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;
+        if (cur.nparts == 1) {
+            T *out = static_cast<T *>(p.out);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float inv = 1.f / Lg[g];
+                T *dst = out + (head0 + g) * D + lane * Gm::EPL;
+                if constexpr (Gm::EPL == 4) {
+                    uint2 w;
+                    w.x = Elem<T>::pack(acc[g][0] * inv, acc[g][1] * inv);
+                    w.y = Elem<T>::pack(acc[g][2] * inv, acc[g][3] * inv);
+                    *reinterpret_cast<uint2 *>(dst) = w;
+                } else {
+                    *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(acc[g][0] * inv, acc[g][1] * inv);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const size_t row = (head0 + g) * p.max_parts + cur.part;
+                float *dst = p.part_acc + row * D + lane * Gm::EPL;
+                if constexpr (Gm::EPL == 4)
+                    *reinterpret_cast<float4 *>(dst) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+                else
+                    *reinterpret_cast<float2 *>(dst) = make_float2(acc[g][0], acc[g][1]);
+                if (lane == g) p.ml[row] = make_float2(Mg[g], Lg[g]);
+            }
+        }
+
+        // ---------------- next unit -------------------------------------------
+        while (!prod_on_nxt && !exhausted) produce();
+        if (!prod_on_nxt) break;
+        cur = nxt;
+        prod_on_nxt = false;
+    }
+}
+
+// ---- 3. merge of split sequences ---------------------------------------------
+constexpr int MERGE_WARPS = 8;
+
+template <int D, typename T>
+__global__ void __launch_bounds__(MERGE_WARPS * 32) pa_merge_kernel(const DecodeParams p) {
+    constexpr int EPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long wid = (long)blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);
+    if (wid >= (long)p.num_seqs * p.num_heads) return;
+    const int s = (int)(wid / p.num_heads);
+    const int ctx = clamped_context(p, s, false);
+    const int nparts = (ctx + p.partition - 1) / p.partition;
+    if (nparts <= 1) return;  // written by the attention kernel (or zeroed by the plan)
+    T *dst = static_cast<T *>(p.out) + (size_t)wid * D + lane * EPL;
+    float o[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) o[e] = 0.f;
+    if (nparts > 1) {
+        const float2 *ml = p.ml + (size_t)wid * p.max_parts;
+        const float *acc = p.part_acc + (size_t)wid * p.max_parts * D + lane * EPL;
+        float M = -INFINITY;
+        for (int j = 0; j < nparts; ++j) M = fmaxf(M, ml[j].x);
+        float L = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < nparts; ++j) {
+            const float2 v = ml[j];
+            const float w = exp2f(v.x - M);
+            L = fmaf(w, v.y, L);
+            if constexpr (EPL == 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(acc + (size_t)j * D);
+                o[0] = fmaf(w, a.x, o[0]); o[1] = fmaf(w, a.y, o[1]);
+                o[2] = fmaf(w, a.z, o[2]); o[3] = fmaf(w, a.w, o[3]);
+            } else {
+                const float2 a = *reinterpret_cast<const float2 *>(acc + (size_t)j * D);
+                o[0] = fmaf(w, a.x, o[0]); o[1] = fmaf(w, a.y, o[1]);
+            }
+        }
+        const float inv = 1.f / L;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[e] *= inv;
+    }
+    if constexpr (EPL == 4) {
+        uint2 w;
+        w.x = Elem<T>::pack(o[0], o[1]);
+        w.y = Elem<T>::pack(o[2], o[3]);
+        *reinterpret_cast<uint2 *>(dst) = w;
+    } else {
+        *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(o[0], o[1]);
+    }
+}
+
+}  // namespace pa

@@ -1,0 +1,41 @@
+"""The C-ABI library builds, loads and exports every function include/pa.h
+declares (CPU only: no compute calls)."""
+import ctypes
+
+import paged_kv_cache_372_b200 as pa
+from paged_kv_cache_372_b200 import build
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    build.build()
+    lib = pa.lib()
+    names = pa.header_functions()
+    assert {"pa_decode", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_workspace_size"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/pa.h but not exported"
+
+
+def test_host_only_entry_points():
+    lib = pa.lib()
+    assert lib.pa_status_string(0) == b"PA_OK"
+    assert lib.pa_status_string(2) == b"PA_ERR_UNSUPPORTED"
+    # partition choice and workspace size are pure host functions
+    assert pa.pa_decode_partition_size(8, 32, 8, 128, 64, 32768, 512) == 512
+    assert pa.pa_decode_partition_size(4, 2, 2, 64, 16, 33, 0) == 48        # one partition
+    assert pa.pa_decode_partition_size(4, 2, 2, 64, 16, 33, 24) == 0        # not a multiple of 16
+    assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 100, 0) == 112    # group 8: one partition
+    assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 8192, 0) == 256   # group 8: 8 KB of scores
+    assert pa.pa_decode_partition_size(4, 24, 4, 128, 16, 100, 0) == 0      # group 6 unsupported
+    n = pa.pa_decode_workspace_size(8, 32, 8, 128, 64, 32768, 512)
+    parts = 32768 // 512
+    assert n >= 8 * parts * 16 + 8 * 32 * parts * (8 + 128 * 4)
+    assert lib.pa_decode_workspace_size(4, 2, 2, 96, 16, 33, 0) == 0        # head_dim 96
+
+
+def test_reshape_rejects_bad_arguments_without_a_device():
+    lib = pa.lib()
+    assert lib.pa_reshape_and_cache(None, None, None, None, None, 1, 2, 64, 16, 32, 0, None) == pa.PA_ERR_INVALID
+    assert lib.pa_reshape_and_cache(None, None, None, None, None, 1, 2, 96, 16, 32, 0, None) == pa.PA_ERR_UNSUPPORTED
+    ptrs = (ctypes.c_void_p * 1)(None)
+    assert lib.pa_copy_blocks(ptrs, 1, None, 1, 100, 32, None) == pa.PA_ERR_INVALID
+    assert lib.pa_last_error() != b""

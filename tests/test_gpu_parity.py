@@ -1,0 +1,99 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Cache writes and block copies must be bit-exact (the whole pool is compared,
+which also catches stray writes); attention must be within max-abs 2e-3
+(fp16) / 1e-2 (bf16) of the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_372_b200 as pa
+from paged_kv_cache_372_b200 import workloads
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+def run_and_compare(wl, partition_size=None, steps=None):
+    kp, vp = H.to_gpu(wl)
+    okp, ovp = H.oracle_state(wl)
+    errs = []
+    for i in range(len(wl.steps) if steps is None else steps):
+        out = H.gpu_step(wl, i, kp, vp, partition_size)
+        ref = H.oracle_step(wl, i, okp, ovp)
+        torch.cuda.synchronize()
+        assert pa.pa_device_errors() == 0
+        assert H.pools_equal(kp, vp, okp, ovp), f"pools differ after step {i}"
+        err = H.max_err(out, ref)
+        errs.append(err)
+        assert err <= H.TOL[wl.dtype], (wl.name, i, err)
+    return errs
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny(seed):
+    run_and_compare(workloads.tiny(seed))
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_llama7b_small(seed):
+    run_and_compare(workloads.llama7b(seed, num_seqs=6))
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_llama3_8b_small(seed):
+    run_and_compare(workloads.llama3_8b(seed, num_seqs=12))
+
+
+def test_llama7b_full():
+    run_and_compare(workloads.llama7b(0))
+
+
+def test_llama3_8b_full():
+    run_and_compare(workloads.llama3_8b(0))
+
+
+def test_beam_all_steps():
+    run_and_compare(workloads.beam(0))
+
+
+def test_long32k_full():
+    run_and_compare(workloads.long32k(0))
+
+
+@pytest.mark.parametrize("partition", [16, 32, 128, 256])
+def test_split_partitions(partition):
+    wl = workloads.llama3_8b(3, num_seqs=10)
+    run_and_compare(wl, partition_size=partition)
+
+
+@pytest.mark.parametrize("shape", [(64, 1), (64, 2), (64, 4), (64, 8), (128, 1), (128, 2), (128, 4), (128, 8)])
+@pytest.mark.parametrize("block_size", [16, 32, 64])
+def test_shapes(shape, block_size):
+    """Every supported (head_dim, group, block_size), ragged contexts, both dtypes."""
+    D, G = shape
+    from paged_kv_cache_372_b200 import inputs
+    from paged_kv_cache_372_b200.block_manager import BlockManager
+    import math
+    for dtype in ("f16", "bf16"):
+        gen = inputs.generator(D * 100 + G * 10 + block_size)
+        ctx = [1, 15, 16, 17, 100, 333, 700]
+        hkv = 2
+        need = sum(-(-c // block_size) for c in ctx)
+        nb = need + 5
+        bm = BlockManager(nb, block_size, inputs.permutation(nb, gen))
+        for s, c in enumerate(ctx):
+            bm.allocate(s, c)
+        width = max(len(t) for t in bm.tables.values())
+        st = workloads.Step(
+            q=inputs.normal((len(ctx), hkv * G, D), dtype, gen),
+            block_tables=bm.block_table_array(range(len(ctx)), width),
+            context_lens=bm.context_lens(range(len(ctx))),
+            k_new=inputs.normal((0, hkv, D), dtype, gen), v_new=inputs.normal((0, hkv, D), dtype, gen),
+            slot_mapping=np.zeros(0, np.int64), copy_pairs=np.zeros((0, 2), np.int64))
+        wl = workloads.Workload("shape", dtype, hkv * G, hkv, D, block_size, nb, 0,
+                                inputs.normal((nb, hkv, block_size, D), dtype, gen),
+                                inputs.normal((nb, hkv, block_size, D), dtype, gen), [st])
+        for P in (0, block_size * max(1, 64 // block_size)):
+            run_and_compare(wl, partition_size=P)
