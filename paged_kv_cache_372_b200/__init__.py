@@ -15,7 +15,8 @@ import re
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "_lib", "libpa_b200.so")
+# PA_B200_LIB points the binding at another build of the same library.
+LIB_PATH = os.environ.get("PA_B200_LIB") or os.path.join(HERE, "_lib", "libpa_b200.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "pa.h")
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK = range(5)

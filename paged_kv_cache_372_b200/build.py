@@ -43,11 +43,15 @@ def stale() -> bool:
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not stale():
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          out: str | None = None) -> str:
+    """Compile when a source is newer than the library (or force). `extra` adds nvcc
+    flags (e.g. -DPA_DECODE_STAGES=6); `out` writes the library elsewhere."""
+    target = out or LIB
+    if not force and out is None and not stale():
         return LIB
-    os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB + f".tmp{os.getpid()}"
+    os.makedirs(os.path.dirname(target), exist_ok=True)
+    tmp = target + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE,
            os.path.join(CSRC, "pa_api.cu"), "-o", tmp]
@@ -59,8 +63,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         print(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

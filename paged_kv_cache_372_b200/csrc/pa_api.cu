@@ -61,13 +61,12 @@ pa_status device_info(DeviceInfo *out) {
 }
 
 // Largest partition the attention kernel takes: the unit's block-table slice
-// fits one register per lane (<= 32 blocks) and its scores fit 8 KB.
-int partition_cap(int block_size, int group) {
-    int cap = 32 * block_size;
-    if (2048 / group < cap) cap = 2048 / group;
-    if (cap > 512) cap = 512;
-    return cap - cap % block_size;
-}
+// fits one register per lane (<= 32 blocks).
+int partition_cap(int block_size) { return 32 * block_size; }
+
+// Partition used when the caller passes 0: a whole sequence when every
+// context fits 512 tokens, else 512-token partitions.
+constexpr int kAutoPartition = 512;
 
 bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_size) {
     if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return false;
@@ -78,43 +77,51 @@ bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_si
 }
 
 // Resolves partition_size (0 = auto). Returns 0 for an invalid request.
-int resolve_partition(int num_heads, int num_kv_heads, int block_size, int max_context_len, int requested) {
-    const int cap = partition_cap(block_size, num_heads / num_kv_heads);
+int resolve_partition(int block_size, int max_context_len, int requested) {
     if (requested > 0) {
-        if (requested % 16 || requested % block_size || requested > cap) return 0;
+        if (requested % 16 || requested % block_size || requested > partition_cap(block_size)) return 0;
         return requested;
     }
-    if (max_context_len <= cap) {
+    const int auto_p = kAutoPartition - kAutoPartition % block_size;
+    if (max_context_len <= auto_p) {
         const int need = max_context_len > 0 ? max_context_len : 1;
         return ((need + block_size - 1) / block_size) * block_size;
     }
-    return cap;
+    return auto_p;
 }
 
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 template <int D, int G, typename T>
 pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
-    constexpr int NS = 4;
+    constexpr int NS = pa::DECODE_STAGES;
     DeviceInfo info;
     pa_status st = device_info(&info);
     if (st != PA_OK) return st;
-    const int per_warp = pa::warp_smem_bytes<D, G, NS>(p.partition);
+    const int per_warp = pa::warp_smem_bytes<D, G, NS>();
     int warps = info.smem_optin / per_warp;
     if (warps > pa::DECODE_MAX_WARPS) warps = pa::DECODE_MAX_WARPS;
-    if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "partition %d needs %d bytes of shared memory per warp",
-                               p.partition, per_warp);
+    if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "%d bytes of shared memory per warp", per_warp);
     const int smem = warps * per_warp;
     auto kernel = pa::pa_decode_kernel<D, G, T, NS>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
     pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
-    kernel<<<info.sms, warps * 32, smem, stream>>>(p);
-    if (p.max_parts > 1) {
-        const long long warps_total = (long long)p.num_seqs * p.num_heads;
-        pa::pa_merge_kernel<D, T><<<ceil_div(warps_total, pa::MERGE_WARPS), pa::MERGE_WARPS * 32, 0, stream>>>(p);
-    }
+    // Programmatic dependent launch: the attention CTAs start their set-up
+    // while the plan kernel runs and wait for its results in-kernel.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(info.sms);
+    cfg.blockDim = dim3(warps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, p);
+    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
     return PA_OK;
@@ -152,7 +159,7 @@ int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int 
                              int max_context_len, int partition_size) {
     if (num_seqs < 0 || max_context_len < 0 || partition_size < 0) return 0;
     if (!shape_supported(num_heads, num_kv_heads, head_dim, block_size)) return 0;
-    return resolve_partition(num_heads, num_kv_heads, block_size, max_context_len, partition_size);
+    return resolve_partition(block_size, max_context_len, partition_size);
 }
 
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
@@ -161,7 +168,7 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
                                            max_context_len, partition_size);
     if (P == 0) return 0;
     const int max_parts = max_context_len > 0 ? ceil_div(max_context_len, P) : 1;
-    return pa::ws_layout(num_seqs, num_heads, head_dim, max_parts).total;
+    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts).total;
 }
 
 pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_pool, const int32_t *block_tables,
@@ -182,16 +189,16 @@ pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
         return fail(PA_ERR_INVALID, "misaligned pointer (16 B tensors, 4 B int arrays, 256 B workspace)");
-    const int P = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len, partition_size);
+    const int P = resolve_partition(block_size, max_context_len, partition_size);
     if (P == 0)
         return fail(PA_ERR_INVALID, "partition_size %d (multiple of 16 and of block_size, at most %d)",
-                    partition_size, partition_cap(block_size, num_heads / num_kv_heads));
+                    partition_size, partition_cap(block_size));
     const long long table_tokens = (long long)max_blocks_per_seq * block_size;
     const int ctx_limit = (int)(table_tokens < max_context_len ? table_tokens : max_context_len);
     const int max_parts = max_context_len > 0 ? ceil_div(max_context_len, P) : 1;
     if ((long long)num_seqs * max_parts * num_kv_heads >= (1ll << 31))
         return fail(PA_ERR_UNSUPPORTED, "too many work units");
-    const pa::WsLayout L = pa::ws_layout(num_seqs, num_heads, head_dim, max_parts);
+    const pa::WsLayout L = pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts);
     if (workspace_bytes < L.total)
         return fail(PA_ERR_INVALID, "workspace %zu bytes < %zu needed", workspace_bytes, L.total);
 
@@ -219,6 +226,7 @@ pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_
     p.entries = reinterpret_cast<int4 *>(ws + L.entries);
     p.ml = reinterpret_cast<float2 *>(ws + L.ml);
     p.part_acc = reinterpret_cast<float *>(ws + L.acc);
+    p.merge_count = reinterpret_cast<int *>(ws + L.count);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int group = num_heads / num_kv_heads;

@@ -1,22 +1,23 @@
-// Paged decode attention for sm_100a: three launches per call.
+// Paged decode attention for sm_100a: two launches per call.
 //
 //  1. pa_plan_kernel   (1 CTA) cuts every sequence into partitions of P tokens
 //     and writes the work list, longest partitions first, so that the
-//     persistent attention kernel finishes with the short ones.
-//  2. pa_decode_kernel (one persistent CTA per SM) — every warp is an
+//     persistent attention kernel finishes with the short ones. It also
+//     zeroes the per-(sequence, KV head) merge counters.
+//  2. pa_decode_kernel (one persistent CTA per SM, launched with programmatic
+//     dependent launch so its set-up overlaps the plan) — every warp is an
 //     independent worker. It takes (sequence, KV head, partition) units from
 //     the work list with an atomic counter and streams the unit's 16-token K
 //     and V tiles, each one contiguous chunk of the pool, through a private
 //     ring of shared-memory stages filled by 1-D bulk copies (TMA) that
-//     complete on mbarriers. The block-table entries of a unit are loaded
-//     once into lane registers and handed to the copy-issuing lane by a
-//     shuffle. Per unit: K phase (scores of the G query heads of the KV head,
-//     kept in shared memory), exact max, exponentials, V phase (weighted sum).
-//     A unit that is a whole sequence writes the normalised output; otherwise
-//     it writes (max, sum, unnormalised output) partials.
-//  3. pa_merge_kernel  merges the partials of split sequences by the
-//     log-sum-exp identity and writes their outputs.
-//
+//     complete on mbarriers; K and V tiles alternate. The block-table entries
+//     of a unit are loaded once into lane registers and handed to the
+//     copy-issuing lane by a shuffle. Per tile: scores of the G query heads
+//     of the KV head, online softmax, weighted sum of the values. A unit that
+//     is a whole sequence writes the normalised output; otherwise it writes
+//     (max, sum, unnormalised output) partials, and the last warp to finish a
+//     (sequence, KV head) merges its partitions by the log-sum-exp identity.
+
 // The arithmetic is the definition in "别再让GPU内存拖后腿了：vLLM的PagedAttention
 // 如何像操作系统一样管理KV Cache", section 3.1: scores of the query against every
 // page, softmax over the concatenation with the 1/sqrt(dim) scale, weighted sum
@@ -47,24 +48,28 @@ struct DecodeParams {
     int4 *entries;   // {seq, partition, tokens, partitions of seq}
     float2 *ml;      // [seq][head][part] (max in log2 units, sum of weights)
     float *part_acc; // [seq][head][part][D] unnormalised outputs
+    int *merge_count;// [seq][kv head] finished partitions
 };
 
 // Workspace layout: header (counter, entry count), work list, partials.
 struct WsLayout {
-    size_t entries, ml, acc, total;
+    size_t entries, ml, acc, count, total;
 };
 
 inline __host__ __device__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline __host__ __device__ WsLayout ws_layout(int B, int H, int D, int max_parts) {
+inline __host__ __device__ WsLayout ws_layout(int B, int H, int Hkv, int D, int max_parts) {
     WsLayout L;
     size_t off = 256;
     L.entries = off;
     off = align256(off + sizeof(int4) * (size_t)B * max_parts);
+    L.count = off;
+    off = align256(off + sizeof(int) * (size_t)B * Hkv);
+    const size_t parts = max_parts > 1 ? (size_t)max_parts : 0;  // no partials without a split
     L.ml = off;
-    off = align256(off + sizeof(float2) * (size_t)B * H * max_parts);
+    off = align256(off + sizeof(float2) * (size_t)B * H * parts);
     L.acc = off;
-    off = align256(off + sizeof(float) * (size_t)B * H * max_parts * D);
+    off = align256(off + sizeof(float) * (size_t)B * H * parts * D);
     L.total = off;
     return L;
 }
@@ -87,9 +92,12 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
     __shared__ int s_bin_next[PLAN_MAX_BINS];
     __shared__ int s_warp[32];
     __shared__ int s_carry;
+    // Let the attention kernel launch now; it waits for this grid's results.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int P = p.partition, tiles = P / 16;
     for (int i = tid; i < PLAN_MAX_BINS; i += PLAN_THREADS) s_bin_count[i] = 0;
+    for (int i = tid; i < p.num_seqs * p.num_kv_heads; i += PLAN_THREADS) p.merge_count[i] = 0;
     if (tid == 0) s_carry = 0;
     __syncthreads();
 
@@ -152,13 +160,16 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
 }
 
 // ---- 2. attention -------------------------------------------------------------
-// Lane geometry of the K phase. A 16-token tile row is D elements = NV vectors
-// of 16 bytes. Each lane holds VPL vectors of the row (so G*VPL*8 = 64 query
-// values in registers) for TPL tokens; DG lanes share a token and their
-// partial dot products are summed through a small shared-memory transpose.
-// After it each lane owns R = G/2 (token, head) scores (G = 1: one, shared by
-// a lane pair). DG < 8 rotates each lane's vector order by its token group so
-// that the 8 lanes of a shared-memory phase hit distinct banks.
+// Lane geometry of the score computation. A 16-token tile row is D elements =
+// NV vectors of 16 bytes. Each lane holds VPL vectors of the row (so
+// G*VPL*8 = 64 query values in registers) for TPL tokens; DG lanes share a
+// token and their partial dot products are summed through a small
+// shared-memory transpose, after which each lane owns R = G/2 (token, head)
+// scores (G = 1: one score, shared by a lane pair). DG < 8 rotates each lane's
+// vector order by its token group so that the 8 lanes of a shared-memory phase
+// hit distinct banks. The weighted sum uses another mapping: lane l owns row
+// elements [l*EPL, (l+1)*EPL) of every head, for all 16 tokens of the tile, so
+// no cross-lane reduction is needed at the end.
 template <int D, int G>
 struct Geo {
     static constexpr int NV = D / 8;
@@ -169,29 +180,91 @@ struct Geo {
     static constexpr int V = TPL * G;
     static constexpr int R = G >= 2 ? G / 2 : 1;
     static constexpr bool ROT = DG < 8;
-    static constexpr int EPL = D / 32;  // V phase: elements of a row per lane
+    static constexpr int NACC = TPL * G >= 4 ? 1 : 4 / (TPL * G);  // independent FMA chains
+    static constexpr int EPL = D / 32;
     static constexpr int TILE_BYTES = 16 * D * 2;
     static constexpr int Q_BYTES = G * D * 2;
     static constexpr int XROW = (V % 4 == 0) ? V + 4 : V + 1;
     static constexpr int XTG = DG * XROW + ((V % 4 == 0) ? 16 : 0);
     static constexpr int XB_BYTES = G >= 2 ? ((TG * XTG * 4 + 15) & ~15) : 0;
+    static constexpr int SC_BYTES = G * 16 * 4;  // probabilities of one tile, [head][token]
+    static constexpr int BAR_BYTES = 16;         // up to 2 mbarriers per 16 bytes, see warp_smem_bytes
     static_assert(TG * DG == 32 && TPL * TG == 16, "lane geometry");
     static_assert(G == 1 || V == DG * R, "reduction geometry");
 };
 
 template <int D, int G, int NS>
-__host__ __device__ constexpr int warp_smem_bytes(int partition) {
-    return NS * Geo<D, G>::TILE_BYTES + 2 * Geo<D, G>::Q_BYTES + Geo<D, G>::XB_BYTES + 16 * ((NS * 8 + 15) / 16) +
-           ((partition * G * 4 + 15) & ~15);
+__host__ __device__ constexpr int warp_smem_bytes() {
+    return NS * Geo<D, G>::TILE_BYTES + 2 * Geo<D, G>::Q_BYTES + Geo<D, G>::XB_BYTES + Geo<D, G>::SC_BYTES +
+           16 * ((NS * 8 + 15) / 16);
 }
 
-constexpr int DECODE_MAX_WARPS = 12;
+// Build-time tuning: stages of the per-warp ring and the warp cap per CTA.
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 4
+#endif
+#ifndef PA_DECODE_MAX_WARPS
+#define PA_DECODE_MAX_WARPS 12
+#endif
+constexpr int DECODE_STAGES = PA_DECODE_STAGES;
+constexpr int DECODE_MAX_WARPS = PA_DECODE_MAX_WARPS;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
+// The running maximum of a head is only raised when a score exceeds it by more
+// than this many log2 units, so exponentials stay <= 2^8 and rescaling of the
+// accumulators is rare. The final normalisation uses the same reference, so the
+// result is the exact softmax in real arithmetic.
+constexpr float LAZY_MAX_LOG2 = 8.0f;
 
 struct Unit {
     int s, kvh, part, ntok, nparts, ntiles, tbl, slot;
     bool valid;
 };
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// Merge of the partitions of one (sequence, KV head) by the log-sum-exp
+// identity: out = sum_j 2^(m_j - M) acc_j / sum_j 2^(m_j - M) l_j.
+template <int D, int G, typename T>
+__device__ __forceinline__ void merge_partitions(const DecodeParams &p, size_t head0, int nparts, int lane) {
+    constexpr int EPL = D / 32;
+    T *out = static_cast<T *>(p.out);
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+        const size_t row0 = (head0 + g) * p.max_parts;
+        float M = -INFINITY;
+        for (int j = lane; j < nparts; j += 32) M = fmaxf(M, __ldcg(&p.ml[row0 + j].x));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
+        float L = 0.f, o[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[e] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < nparts; ++j) {
+            const float2 ml = __ldcg(&p.ml[row0 + j]);
+            const float w = exp2f(ml.x - M);
+            L = fmaf(w, ml.y, L);
+            const float *a = p.part_acc + (row0 + j) * D + lane * EPL;
+            if constexpr (EPL == 4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(a));
+                o[0] = fmaf(w, v.x, o[0]); o[1] = fmaf(w, v.y, o[1]);
+                o[2] = fmaf(w, v.z, o[2]); o[3] = fmaf(w, v.w, o[3]);
+            } else {
+                const float2 v = __ldcg(reinterpret_cast<const float2 *>(a));
+                o[0] = fmaf(w, v.x, o[0]); o[1] = fmaf(w, v.y, o[1]);
+            }
+        }
+        const float inv = 1.f / L;
+        T *dst = out + (head0 + g) * D + lane * EPL;
+        if constexpr (EPL == 4) {
+            uint2 w;
+            w.x = Elem<T>::pack(o[0] * inv, o[1] * inv);
+            w.y = Elem<T>::pack(o[2] * inv, o[3] * inv);
+            *reinterpret_cast<uint2 *>(dst) = w;
+        } else {
+            *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(o[0] * inv, o[1] * inv);
+        }
+    }
+}
 
 template <int D, int G, typename T, int NS>
 __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(const DecodeParams p) {
@@ -199,14 +272,13 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int P = p.partition;
     const int Hkv = p.num_kv_heads, H = p.num_heads, bs = p.block_size;
 
-    uint8_t *ring = smem + (size_t)warp * warp_smem_bytes<D, G, NS>(P);
+    uint8_t *ring = smem + (size_t)warp * warp_smem_bytes<D, G, NS>();
     uint8_t *qbuf = ring + NS * Gm::TILE_BYTES;
     float *xb = reinterpret_cast<float *>(qbuf + 2 * Gm::Q_BYTES);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(xb) + Gm::XB_BYTES);
-    float *sc = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 16 * ((NS * 8 + 15) / 16));
+    float *sc = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(xb) + Gm::XB_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sc) + Gm::SC_BYTES);
     const uint32_t ring_s = smem_u32(ring), qbuf_s = smem_u32(qbuf), bar_s = smem_u32(bars);
 
     if (lane == 0) {
@@ -214,14 +286,16 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
         fence_barrier_init();
     }
     __syncwarp();
+    const uint64_t policy = l2_policy_evict_first();
+    // The work list is written by the plan kernel that precedes this one.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const T *kpool = static_cast<const T *>(p.k_pool);
     const T *vpool = static_cast<const T *>(p.v_pool);
     const T *qg = static_cast<const T *>(p.q);
     const int total_units = *p.num_entries * Hkv;
-    const uint64_t policy = l2_policy_evict_first();
 
-    // K-phase lane geometry.
+    // Score-phase lane geometry.
     const int tg = lane / Gm::DG, dg = lane % Gm::DG;
     int voff[Gm::VPL];
 #pragma unroll
@@ -247,14 +321,15 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
         x.nparts = ent.w;
         x.ntiles = (x.ntok + 15) >> 4;
         const int nblk = (x.ntok + bs - 1) / bs;
-        x.tbl = lane < nblk ? p.block_tables[(size_t)x.s * p.max_blocks_per_seq + x.part * (P / bs) + lane] : 0;
+        x.tbl = lane < nblk ? p.block_tables[(size_t)x.s * p.max_blocks_per_seq + x.part * (p.partition / bs) + lane]
+                            : 0;
     };
 
-    // Issue item `it` of a unit: items [0, ntiles) are its K tiles, the rest
-    // its V tiles; item 0 also brings the unit's G query rows.
-    auto issue = [&](int s, int kvh, int ntiles, int tbl, int qslot, int it, uint32_t stage) {
-        const bool is_v = it >= ntiles;
-        const int tok = 16 * (is_v ? it - ntiles : it);
+    // Item `it` of a unit: even items are K tiles, odd items V tiles (tile it/2);
+    // item 0 also brings the unit's G query rows.
+    auto issue = [&](int s, int kvh, int tbl, int qslot, int it, uint32_t stage) {
+        const bool is_v = it & 1;
+        const int tok = 16 * (it >> 1);
         const int bi = tok / bs;
         const int pb = __shfl_sync(FULL_MASK, tbl, bi);
         if (lane == 0) {
@@ -306,9 +381,9 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
             pitem = 0;
         }
         if (prod_on_nxt)
-            issue(nxt.s, nxt.kvh, nxt.ntiles, nxt.tbl, nxt.slot, pitem, issued % NS);
+            issue(nxt.s, nxt.kvh, nxt.tbl, nxt.slot, pitem, issued % NS);
         else
-            issue(cur.s, cur.kvh, cur.ntiles, cur.tbl, cur.slot, pitem, issued % NS);
+            issue(cur.s, cur.kvh, cur.tbl, cur.slot, pitem, issued % NS);
         ++pitem;
         ++issued;
     };
@@ -329,16 +404,23 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
 
     for (int i = 0; i < NS; ++i) produce();
 
-    float qf[G][Gm::VPL * 8];
-    float acc[G][Gm::EPL];
-    float Mg[G], Lg[G];
+    float2 qf[G][Gm::VPL * 4];     // query pairs, pre-scaled by scale*log2(e)
+    float2 acc[G][Gm::EPL];        // (even-token, odd-token) partial sums of p*v
 
     for (;;) {
-        // ---------------- K phase: scores of this unit -----------------------
-        float mx[Gm::R];
+        float Mg[G];               // reference maximum per head (log2 units)
+        float ls[Gm::R];           // this lane's sum of its owned probabilities
 #pragma unroll
-        for (int r = 0; r < Gm::R; ++r) mx[r] = -INFINITY;
+        for (int g = 0; g < G; ++g) {
+            Mg[g] = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < Gm::EPL; ++e) acc[g][e] = f2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int r = 0; r < Gm::R; ++r) ls[r] = 0.f;
+
         for (int k = 0; k < cur.ntiles; ++k) {
+            // ------------------------------ scores of tile k ----------------
             if (!wait_item()) return;
             const uint8_t *tile = ring + (consumed % NS) * Gm::TILE_BYTES;
             if (k == 0) {
@@ -347,10 +429,13 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
                 for (int g = 0; g < G; ++g)
 #pragma unroll
                     for (int c = 0; c < Gm::VPL; ++c) {
-                        float f[8];
-                        unpack8<T>(*reinterpret_cast<const uint4 *>(qs + g * D * 2 + voff[c]), f);
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(qs + g * D * 2 + voff[c]);
+                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) qf[g][c * 8 + e] = f[e] * p.qscale;
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 v = Elem<T>::pair(w[j]);
+                            qf[g][c * 4 + j] = f2(v.x * p.qscale, v.y * p.qscale);
+                        }
                     }
             }
             const int valid = min(16, cur.ntok - 16 * k);
@@ -358,16 +443,31 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
 #pragma unroll
             for (int i = 0; i < Gm::TPL; ++i) {
                 const uint8_t *row = tile + (tg + Gm::TG * i) * (D * 2);
+                float2 a2[G][Gm::NACC];
 #pragma unroll
-                for (int g = 0; g < G; ++g) part[i][g] = 0.f;
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int n = 0; n < Gm::NACC; ++n) a2[g][n] = f2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < Gm::VPL; ++c) {
-                    float f[8];
-                    unpack8<T>(*reinterpret_cast<const uint4 *>(row + voff[c]), f);
+                    const uint4 raw = *reinterpret_cast<const uint4 *>(row + voff[c]);
+                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                    for (int g = 0; g < G; ++g)
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 kv = Elem<T>::pair(w[j]);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) part[i][g] = fmaf(qf[g][c * 8 + e], f[e], part[i][g]);
+                        for (int g = 0; g < G; ++g) {
+                            float2 &a = a2[g][(c * 4 + j) % Gm::NACC];
+                            a = __ffma2_rn(qf[g][c * 4 + j], kv, a);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float sum = 0.f;
+#pragma unroll
+                    for (int n = 0; n < Gm::NACC; ++n) sum += a2[g][n].x + a2[g][n].y;
+                    part[i][g] = sum;
                 }
             }
             float sred[Gm::R];
@@ -404,51 +504,103 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
                     }
                 }
             }
+            // Tokens past the context (stale or never-written slots) get -inf.
             const bool tvalid = t_own < valid;
+            float mown[Gm::R];
+            bool raise = false;
 #pragma unroll
             for (int r = 0; r < Gm::R; ++r) {
-                const float s = tvalid ? sred[r] : -INFINITY;
-                mx[r] = fmaxf(mx[r], s);
-                if (owner) sc[(g0 + r) * P + 16 * k + t_own] = s;
+                sred[r] = tvalid ? sred[r] : -INFINITY;
+                mown[r] = 0.f;
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+                    if (g == g0 + r) mown[r] = Mg[g];
+                raise |= !(sred[r] <= mown[r] + LAZY_MAX_LOG2);
+            }
+            // ------------------------------ online softmax ------------------
+            if (__any_sync(FULL_MASK, raise)) {
+                float tm[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    tm[g] = -INFINITY;
+#pragma unroll
+                    for (int r = 0; r < Gm::R; ++r)
+                        if (g == g0 + r) tm[g] = fmaxf(tm[g], sred[r]);
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) tm[g] = fmaxf(tm[g], __shfl_xor_sync(FULL_MASK, tm[g], o));
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float mn = fmaxf(Mg[g], tm[g]);
+                    const float alpha = exp2f(Mg[g] - mn);  // 0 on the first tile (Mg = -inf)
+                    Mg[g] = mn;
+#pragma unroll
+                    for (int e = 0; e < Gm::EPL; ++e) acc[g][e] = __fmul2_rn(acc[g][e], f2(alpha, alpha));
+#pragma unroll
+                    for (int r = 0; r < Gm::R; ++r)
+                        if (g == g0 + r) {
+                            ls[r] *= alpha;
+                            mown[r] = mn;
+                        }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < Gm::R; ++r) {
+                const float e = exp2f(sred[r] - mown[r]);
+                ls[r] += e;
+                if (owner) sc[(g0 + r) * 16 + t_own] = e;
+            }
+            ++consumed;
+            __syncwarp();
+            produce();
+
+            // ------------------------------ values of tile k ----------------
+            if (!wait_item()) return;
+            tile = ring + (consumed % NS) * Gm::TILE_BYTES;
+#pragma unroll
+            for (int t4 = 0; t4 < 4; ++t4) {
+                float4 pq[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) pq[g] = *reinterpret_cast<const float4 *>(sc + g * 16 + 4 * t4);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int t = 4 * t4 + 2 * h2;
+                    const uint8_t *src = tile + t * (D * 2) + lane * (Gm::EPL * 2);
+                    float2 vp[Gm::EPL];  // (token t, token t+1) of each owned element
+                    if constexpr (Gm::EPL == 4) {
+                        uint2 r0 = *reinterpret_cast<const uint2 *>(src);
+                        uint2 r1 = *reinterpret_cast<const uint2 *>(src + D * 2);
+                        if (t >= valid) r0 = make_uint2(0, 0);       // never multiply stale slots
+                        if (t + 1 >= valid) r1 = make_uint2(0, 0);
+                        const float2 a = Elem<T>::pair(r0.x), b = Elem<T>::pair(r0.y);
+                        const float2 c = Elem<T>::pair(r1.x), d = Elem<T>::pair(r1.y);
+                        vp[0] = f2(a.x, c.x); vp[1] = f2(a.y, c.y);
+                        vp[2] = f2(b.x, d.x); vp[3] = f2(b.y, d.y);
+                    } else {
+                        uint32_t r0 = *reinterpret_cast<const uint32_t *>(src);
+                        uint32_t r1 = *reinterpret_cast<const uint32_t *>(src + D * 2);
+                        if (t >= valid) r0 = 0;
+                        if (t + 1 >= valid) r1 = 0;
+                        const float2 a = Elem<T>::pair(r0), c = Elem<T>::pair(r1);
+                        vp[0] = f2(a.x, c.x); vp[1] = f2(a.y, c.y);
+                    }
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float2 pp = h2 ? f2(pq[g].z, pq[g].w) : f2(pq[g].x, pq[g].y);
+#pragma unroll
+                        for (int e = 0; e < Gm::EPL; ++e) acc[g][e] = __ffma2_rn(pp, vp[e], acc[g][e]);
+                    }
+                }
             }
             ++consumed;
             __syncwarp();
             produce();
         }
 
-        // ---------------- exact max, exponentials, sums ----------------------
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float m = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < Gm::R; ++r)
-                if (g == g0 + r) m = mx[r];
-            Mg[g] = m;
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1)
-#pragma unroll
-            for (int g = 0; g < G; ++g) Mg[g] = fmaxf(Mg[g], __shfl_xor_sync(FULL_MASK, Mg[g], o));
-        float mown[Gm::R], ls[Gm::R];
-#pragma unroll
-        for (int r = 0; r < Gm::R; ++r) {
-            ls[r] = 0.f;
-            mown[r] = 0.f;
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-                if (g == g0 + r) mown[r] = Mg[g];
-        }
-        if (owner) {
-            for (int k = 0; k < cur.ntiles; ++k) {
-#pragma unroll
-                for (int r = 0; r < Gm::R; ++r) {
-                    float *a = sc + (g0 + r) * P + 16 * k + t_own;
-                    const float e = exp2f(*a - mown[r]);
-                    *a = e;
-                    ls[r] += e;
-                }
-            }
-        }
+        // ---------------- totals and store -------------------------------------
+        float Lg[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             float l = 0.f;
@@ -461,52 +613,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
         for (int o = 16; o >= 1; o >>= 1)
 #pragma unroll
             for (int g = 0; g < G; ++g) Lg[g] += __shfl_xor_sync(FULL_MASK, Lg[g], o);
-        __syncwarp();
 
-        // ---------------- V phase: weighted sum of values --------------------
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < Gm::EPL; ++e) acc[g][e] = 0.f;
-        for (int k = 0; k < cur.ntiles; ++k) {
-            if (!wait_item()) return;
-            const uint8_t *tile = ring + (consumed % NS) * Gm::TILE_BYTES;
-            const int valid = min(16, cur.ntok - 16 * k);
-#pragma unroll
-            for (int t4 = 0; t4 < 4; ++t4) {
-                float pq[G][4];
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float4 v = *reinterpret_cast<const float4 *>(sc + g * P + 16 * k + 4 * t4);
-                    pq[g][0] = v.x; pq[g][1] = v.y; pq[g][2] = v.z; pq[g][3] = v.w;
-                }
-#pragma unroll
-                for (int tt = 0; tt < 4; ++tt) {
-                    const int t = 4 * t4 + tt;
-                    if (t < valid) {
-                        const uint8_t *src = tile + t * (D * 2) + lane * (Gm::EPL * 2);
-                        float f[Gm::EPL];
-                        if constexpr (Gm::EPL == 4) {
-                            const uint2 raw = *reinterpret_cast<const uint2 *>(src);
-                            const float2 a = Elem<T>::pair(raw.x), b = Elem<T>::pair(raw.y);
-                            f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-                        } else {
-                            const float2 a = Elem<T>::pair(*reinterpret_cast<const uint32_t *>(src));
-                            f[0] = a.x; f[1] = a.y;
-                        }
-#pragma unroll
-                        for (int g = 0; g < G; ++g)
-#pragma unroll
-                            for (int e = 0; e < Gm::EPL; ++e) acc[g][e] = fmaf(pq[g][tt], f[e], acc[g][e]);
-                    }
-                }
-            }
-            ++consumed;
-            __syncwarp();
-            produce();
-        }
-
-        // ---------------- store ---------------------------------------------
         const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;
         if (cur.nparts == 1) {
             T *out = static_cast<T *>(p.out);
@@ -516,11 +623,12 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
                 T *dst = out + (head0 + g) * D + lane * Gm::EPL;
                 if constexpr (Gm::EPL == 4) {
                     uint2 w;
-                    w.x = Elem<T>::pack(acc[g][0] * inv, acc[g][1] * inv);
-                    w.y = Elem<T>::pack(acc[g][2] * inv, acc[g][3] * inv);
+                    w.x = Elem<T>::pack((acc[g][0].x + acc[g][0].y) * inv, (acc[g][1].x + acc[g][1].y) * inv);
+                    w.y = Elem<T>::pack((acc[g][2].x + acc[g][2].y) * inv, (acc[g][3].x + acc[g][3].y) * inv);
                     *reinterpret_cast<uint2 *>(dst) = w;
                 } else {
-                    *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(acc[g][0] * inv, acc[g][1] * inv);
+                    *reinterpret_cast<uint32_t *>(dst) =
+                        Elem<T>::pack((acc[g][0].x + acc[g][0].y) * inv, (acc[g][1].x + acc[g][1].y) * inv);
                 }
             }
         } else {
@@ -529,10 +637,22 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
                 const size_t row = (head0 + g) * p.max_parts + cur.part;
                 float *dst = p.part_acc + row * D + lane * Gm::EPL;
                 if constexpr (Gm::EPL == 4)
-                    *reinterpret_cast<float4 *>(dst) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+                    *reinterpret_cast<float4 *>(dst) =
+                        make_float4(acc[g][0].x + acc[g][0].y, acc[g][1].x + acc[g][1].y,
+                                    acc[g][2].x + acc[g][2].y, acc[g][3].x + acc[g][3].y);
                 else
-                    *reinterpret_cast<float2 *>(dst) = make_float2(acc[g][0], acc[g][1]);
-                if (lane == g) p.ml[row] = make_float2(Mg[g], Lg[g]);
+                    *reinterpret_cast<float2 *>(dst) = f2(acc[g][0].x + acc[g][0].y, acc[g][1].x + acc[g][1].y);
+                if (lane == g) p.ml[row] = f2(Mg[g], Lg[g]);
+            }
+            // The last partition of this (sequence, KV head) to finish merges all.
+            __threadfence();
+            __syncwarp();
+            int done = 0;
+            if (lane == 0) done = atomicAdd(&p.merge_count[(size_t)cur.s * Hkv + cur.kvh], 1);
+            done = __shfl_sync(FULL_MASK, done, 0);
+            if (done == cur.nparts - 1) {
+                __threadfence();
+                merge_partitions<D, G, T>(p, head0, cur.nparts, lane);
             }
         }
 
@@ -541,57 +661,6 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
         if (!prod_on_nxt) break;
         cur = nxt;
         prod_on_nxt = false;
-    }
-}
-
-// ---- 3. merge of split sequences ---------------------------------------------
-constexpr int MERGE_WARPS = 8;
-
-template <int D, typename T>
-__global__ void __launch_bounds__(MERGE_WARPS * 32) pa_merge_kernel(const DecodeParams p) {
-    constexpr int EPL = D / 32;
-    const int lane = threadIdx.x & 31;
-    const long wid = (long)blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);
-    if (wid >= (long)p.num_seqs * p.num_heads) return;
-    const int s = (int)(wid / p.num_heads);
-    const int ctx = clamped_context(p, s, false);
-    const int nparts = (ctx + p.partition - 1) / p.partition;
-    if (nparts <= 1) return;  // written by the attention kernel (or zeroed by the plan)
-    T *dst = static_cast<T *>(p.out) + (size_t)wid * D + lane * EPL;
-    float o[EPL];
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) o[e] = 0.f;
-    if (nparts > 1) {
-        const float2 *ml = p.ml + (size_t)wid * p.max_parts;
-        const float *acc = p.part_acc + (size_t)wid * p.max_parts * D + lane * EPL;
-        float M = -INFINITY;
-        for (int j = 0; j < nparts; ++j) M = fmaxf(M, ml[j].x);
-        float L = 0.f;
-#pragma unroll 4
-        for (int j = 0; j < nparts; ++j) {
-            const float2 v = ml[j];
-            const float w = exp2f(v.x - M);
-            L = fmaf(w, v.y, L);
-            if constexpr (EPL == 4) {
-                const float4 a = *reinterpret_cast<const float4 *>(acc + (size_t)j * D);
-                o[0] = fmaf(w, a.x, o[0]); o[1] = fmaf(w, a.y, o[1]);
-                o[2] = fmaf(w, a.z, o[2]); o[3] = fmaf(w, a.w, o[3]);
-            } else {
-                const float2 a = *reinterpret_cast<const float2 *>(acc + (size_t)j * D);
-                o[0] = fmaf(w, a.x, o[0]); o[1] = fmaf(w, a.y, o[1]);
-            }
-        }
-        const float inv = 1.f / L;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) o[e] *= inv;
-    }
-    if constexpr (EPL == 4) {
-        uint2 w;
-        w.x = Elem<T>::pack(o[0], o[1]);
-        w.y = Elem<T>::pack(o[2], o[3]);
-        *reinterpret_cast<uint2 *>(dst) = w;
-    } else {
-        *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(o[0], o[1]);
     }
 }
 

@@ -24,7 +24,9 @@ def test_host_only_entry_points():
     assert pa.pa_decode_partition_size(4, 2, 2, 64, 16, 33, 0) == 48        # one partition
     assert pa.pa_decode_partition_size(4, 2, 2, 64, 16, 33, 24) == 0        # not a multiple of 16
     assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 100, 0) == 112    # group 8: one partition
-    assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 8192, 0) == 256   # group 8: 8 KB of scores
+    assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 8192, 0) == 512   # 512-token partitions
+    assert pa.pa_decode_partition_size(4, 32, 4, 128, 64, 8192, 2048) == 2048  # 32 blocks of 64
+    assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 8192, 1024) == 0     # > 32 blocks
     assert pa.pa_decode_partition_size(4, 24, 4, 128, 16, 100, 0) == 0      # group 6 unsupported
     n = pa.pa_decode_workspace_size(8, 32, 8, 128, 64, 32768, 512)
     parts = 32768 // 512
