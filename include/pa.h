@@ -176,6 +176,36 @@ PA_API pa_status pa_device_errors(unsigned int *flags, int clear, pa_stream_t st
 /* Number of SMs the library sizes its persistent grids for (current device). */
 PA_API int pa_num_sms(void);
 
+/* Size of the fixed scratch array behind pa_decode_noalloc (16 MiB). */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * pa_decode without a caller-provided workspace, for callers that cannot
+ * allocate device memory at decode time (a plugin whose host pre-partitions
+ * all device memory, a real-time loop that must not take cudaMalloc's implicit
+ * synchronisation, a process with a memory budget fixed at start-up). The
+ * pages this library follows describe no such entry point; it is an addition.
+ *
+ * Arguments, layouts and results are those of pa_decode. The scratch lives in
+ * one file-scope device array of PA_NOALLOC_SCRATCH_BYTES that every GPU which
+ * loads the library holds until the process exits; nothing is allocated.
+ * Sizes whose pa_decode_workspace_size() exceeds the array are rejected with
+ * PA_ERR_UNSUPPORTED before anything is launched (pa_last_error() says why).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. All calls share the one array: calls that overlap on the GPU
+ * (different streams, or different host threads without ordering) race and
+ * give undefined results. Calls ordered on one stream are safe; each call
+ * re-initialises the parts of the array that must start at zero.
+ */
+PA_API pa_status pa_decode_noalloc(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                   const int32_t *block_tables, const int32_t *context_lens,
+                                   int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int max_blocks_per_seq, int num_blocks,
+                                   int max_context_len, float scale, int dtype, int partition_size,
+                                   pa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint), _I, _P]
         L.pa_num_sms.restype = _I
         L.pa_num_sms.argtypes = []
+        L.pa_decode_noalloc.restype = _I
+        L.pa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]
         _lib = L
     return _lib
 
@@ -194,3 +196,20 @@ def pa_device_errors(clear: bool = True, stream=None) -> int:
 
 def pa_num_sms() -> int:
     return int(lib().pa_num_sms())
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def pa_decode_noalloc(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len,
+                      partition_size=0, stream=None) -> torch.Tensor:
+    """pa_decode with the library's fixed scratch array instead of a workspace
+    (for callers that cannot allocate at decode time; see include/pa.h)."""
+    B, H, D = q.shape
+    NB, Hkv, bs, _ = k_pool.shape
+    _check(lib().pa_decode_noalloc(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
+        B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
+        int(partition_size), _stream(stream)))
+    return out

@@ -2,8 +2,8 @@
 
     python -m paged_kv_cache_372_b200.build [--force] [--verbose]
 
-nvcc compiles the single translation unit csrc/pa_api.cu (which includes the
-kernel headers) for sm_100a only. The result lands in ``_lib/`` next to this
+nvcc compiles csrc/pa_api.cu (which includes the kernel headers) and
+csrc/pa_noalloc.cu for sm_100a only. The result lands in ``_lib/`` next to this
 file, so it travels with the source tree.
 """
 from __future__ import annotations
@@ -54,7 +54,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     tmp = target + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE,
-           os.path.join(CSRC, "pa_api.cu"), "-o", tmp]
+           os.path.join(CSRC, "pa_api.cu"), os.path.join(CSRC, "pa_noalloc.cu"), "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     cmd += extra or []

@@ -140,6 +140,9 @@ pa_status dispatch_group(pa::DecodeParams &p, int group, cudaStream_t stream) {
 
 }  // namespace
 
+// Lets other translation units of the library record pa_last_error() text.
+void pa_internal_set_last_error(const char *msg) { g_last_error = msg ? msg : ""; }
+
 extern "C" {
 
 const char *pa_status_string(int status) {
