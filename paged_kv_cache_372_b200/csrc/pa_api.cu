@@ -11,6 +11,9 @@
 #include "pa_cache.cuh"
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
+#include "pa_decode_mma.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace {
 
@@ -127,13 +130,99 @@ pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
     return PA_OK;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+pa_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled *out) {
+    static std::mutex mu;
+    static PFN_cuTensorMapEncodeTiled fn = nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !ptr)
+            return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(ptr);
+    }
+    *out = fn;
+    return PA_OK;
+}
+
+// A pool [num_blocks][num_kv_heads][block_size][D] as a 2-D tensor of
+// rows x D elements, read in boxes of 16 rows x 64 columns (128 bytes) with
+// the 128-byte shared-memory swizzle.
+template <typename T>
+pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, int D) {
+    PFN_cuTensorMapEncodeTiled enc;
+    pa_status st = tensor_map_encoder(&enc);
+    if (st != PA_OK) return st;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, pa::MmaType<T>::tma_type, 2, const_cast<void *>(pool), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PA_OK;
+}
+
+template <int D, int G, typename T>
+pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
+    constexpr int NS = pa::DECODE_MMA_STAGES;
+    DeviceInfo info;
+    pa_status st = device_info(&info);
+    if (st != PA_OK) return st;
+    const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
+    if (rows >= (1ll << 31)) return fail(PA_ERR_UNSUPPORTED, "pool has %lld rows, above 2^31", rows);
+    CUtensorMap tmk, tmv;
+    if ((st = encode_pool_map<T>(&tmk, p.k_pool, rows, D)) != PA_OK) return st;
+    if ((st = encode_pool_map<T>(&tmv, p.v_pool, rows, D)) != PA_OK) return st;
+    int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS>();
+    if (warps > pa::DECODE_MAX_WARPS) warps = pa::DECODE_MAX_WARPS;
+    if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "not enough shared memory for one warp");
+    const int smem = pa::mma_smem_bytes<D, G, NS>(warps);
+    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+
+    pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(info.sms);
+    cfg.blockDim = dim3(warps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, p, tmk, tmv);
+    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+    return PA_OK;
+}
+
 template <int D, typename T>
 pa_status dispatch_group(pa::DecodeParams &p, int group, cudaStream_t stream) {
+    if (group >= pa::DECODE_TENSOR_MIN_GROUP) {
+        switch (group) {
+            case 2: return launch_decode_mma<D, 2, T>(p, stream);
+            case 4: return launch_decode_mma<D, 4, T>(p, stream);
+            case 8: return launch_decode_mma<D, 8, T>(p, stream);
+        }
+    }
     switch (group) {
         case 1: return launch_decode<D, 1, T>(p, stream);
+#if PA_DECODE_TENSOR_MIN_GROUP > 2
         case 2: return launch_decode<D, 2, T>(p, stream);
+#endif
+#if PA_DECODE_TENSOR_MIN_GROUP > 4
         case 4: return launch_decode<D, 4, T>(p, stream);
+#endif
+#if PA_DECODE_TENSOR_MIN_GROUP > 8
         case 8: return launch_decode<D, 8, T>(p, stream);
+#endif
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }

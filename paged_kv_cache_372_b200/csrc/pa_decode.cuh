@@ -206,8 +206,18 @@ __host__ __device__ constexpr int warp_smem_bytes() {
 #ifndef PA_DECODE_MAX_WARPS
 #define PA_DECODE_MAX_WARPS 12
 #endif
+// Ring stages (each one 16-token K+V tile) of the tensor-core kernel, and the
+// smallest head group that uses it (smaller groups use the CUDA-core kernel).
+#ifndef PA_DECODE_MMA_STAGES
+#define PA_DECODE_MMA_STAGES 2
+#endif
+#ifndef PA_DECODE_TENSOR_MIN_GROUP
+#define PA_DECODE_TENSOR_MIN_GROUP 2
+#endif
 constexpr int DECODE_STAGES = PA_DECODE_STAGES;
 constexpr int DECODE_MAX_WARPS = PA_DECODE_MAX_WARPS;
+constexpr int DECODE_MMA_STAGES = PA_DECODE_MMA_STAGES;
+constexpr int DECODE_TENSOR_MIN_GROUP = PA_DECODE_TENSOR_MIN_GROUP;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
 // The running maximum of a head is only raised when a score exceeds it by more
 // than this many log2 units, so exponentials stay <= 2^8 and rescaling of the

@@ -1,0 +1,454 @@
+// Paged decode attention on tensor cores, for grouped-query heads (G >= 2).
+//
+// Same work list, unit scheduling, online softmax and split merge as
+// pa_decode_kernel (pa_decode.cuh); the per-tile arithmetic differs. With G
+// query heads per KV head, one 16-token tile gives two small dense products
+// per warp, each a single mma.sync m16n8k16 per 16-wide slice:
+//
+//   S^T[16 tokens x 8 heads]  = K_tile[16 x D] . Q^T[D x 8]       (D/16 MMAs)
+//   O^T[D x 8 heads]         += V_tile^T[D x 16] . P^T[16 x 8]    (D/16 MMAs)
+//
+// heads padded to N = 8 with zero query rows. K and V tiles arrive by tiled
+// TMA (cp.async.bulk.tensor, 128-byte swizzle) so the ldmatrix fragment loads
+// are bank-conflict free; the probabilities P go from the S accumulators to
+// the B operand of the second product by an in-register 8x8 transpose
+// (movmatrix). Scores, softmax state and O^T stay in fp32; P is rounded to the
+// input type for the second product and the softmax denominator sums the
+// same rounded values.
+#pragma once
+
+#include <cuda.h>
+
+#include "pa_decode.cuh"
+
+namespace pa {
+
+template <int D, int G>
+struct MmaGeo {
+    static_assert(G == 2 || G == 4 || G == 8, "tensor-core path covers grouped heads");
+    static constexpr int KS = D / 16;                    // 16-wide slices of a row
+    static constexpr int NBOX = D / 64;                  // 128-byte TMA boxes per row
+    static constexpr int HALF_BYTES = 16 * D * 2;        // one K (or V) tile
+    static constexpr int STAGE_BYTES = 2 * HALF_BYTES;   // K then V of one tile
+    static constexpr int Q_BYTES = G * D * 2;
+};
+
+template <int D, int G, int NS>
+__host__ __device__ constexpr int mma_smem_bytes(int warps) {
+    // 1024 bytes of slack re-align the base for the 128-byte swizzle pattern.
+    return 1024 + warps * (NS * MmaGeo<D, G>::STAGE_BYTES + 2 * MmaGeo<D, G>::Q_BYTES) + warps * NS * 8;
+}
+
+template <int D, int G, int NS>
+__host__ __device__ constexpr int mma_warp_bytes() {
+    return NS * MmaGeo<D, G>::STAGE_BYTES + 2 * MmaGeo<D, G>::Q_BYTES + NS * 8;
+}
+
+template <typename T>
+struct MmaType;
+template <>
+struct MmaType<__nv_bfloat16> {
+    static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    static constexpr CUtensorMapDataType tma_type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+};
+template <>
+struct MmaType<__half> {
+    static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    static constexpr CUtensorMapDataType tma_type = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
+// Tiled 2-D TMA load of one box {x = column, y = row} (no multicast).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` inside a tile loaded as
+// NBOX boxes of [16 rows][64 columns] with the 128-byte swizzle: within each
+// 1024-byte group of 8 rows the chunk index is XORed with the row index.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    return (uint32_t)((chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+// Merge of one (sequence, KV head)'s partitions, partial layout
+// [part][D][G] floats and [part][G] (max, sum) pairs.
+template <int D, int G, typename T>
+__device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, size_t head0, int nparts, int lane) {
+    constexpr int EPL = D / 32;
+    const float2 *ml = p.ml + group * p.max_parts * G;
+    const float *acc = p.part_acc + group * p.max_parts * (size_t)(D * G);
+    float M[G], L[G], o[EPL][G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        M[g] = -INFINITY;
+        L[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[e][g] = 0.f;
+    }
+    for (int j = 0; j < nparts; ++j)
+#pragma unroll
+        for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __ldcg(&ml[j * G + g].x));
+#pragma unroll 2
+    for (int j = 0; j < nparts; ++j) {
+        float w[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float2 v = __ldcg(&ml[j * G + g]);
+            w[g] = exp2f(v.x - M[g]);
+            L[g] = fmaf(w[g], v.y, L[g]);
+        }
+        const float *a = acc + (size_t)j * D * G + lane * EPL * G;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+#pragma unroll
+            for (int g = 0; g < G; g += 2) {
+                const float2 v = __ldcg(reinterpret_cast<const float2 *>(a + e * G + g));
+                o[e][g] = fmaf(w[g], v.x, o[e][g]);
+                o[e][g + 1] = fmaf(w[g + 1], v.y, o[e][g + 1]);
+            }
+    }
+    T *out = static_cast<T *>(p.out);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const float inv = 1.f / L[g];
+        T *dst = out + (head0 + g) * D + lane * EPL;
+        if constexpr (EPL == 4) {
+            uint2 w;
+            w.x = Elem<T>::pack(o[0][g] * inv, o[1][g] * inv);
+            w.y = Elem<T>::pack(o[2][g] * inv, o[3][g] * inv);
+            *reinterpret_cast<uint2 *>(dst) = w;
+        } else {
+            *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(o[0][g] * inv, o[1][g] * inv);
+        }
+    }
+}
+
+template <int D, int G, typename T, int NS>
+__global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
+    pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v) {
+    using Gm = MmaGeo<D, G>;
+    extern __shared__ uint8_t smem_raw[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int warps = blockDim.x >> 5;
+    const int Hkv = p.num_kv_heads, H = p.num_heads, bs = p.block_size;
+    const int g8 = lane >> 2, t4 = lane & 3;  // mma fragment row / column-pair index
+
+    // Shared memory: [rings of all warps][query buffers][mbarriers], base 1024-aligned.
+    const uint32_t raw_s = smem_u32(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    uint8_t *base = smem_raw + (base_s - raw_s);
+    const uint32_t ring_s = base_s + warp * NS * Gm::STAGE_BYTES;
+    uint8_t *ring = base + warp * NS * Gm::STAGE_BYTES;
+    const uint32_t qbuf_s = base_s + warps * NS * Gm::STAGE_BYTES + warp * 2 * Gm::Q_BYTES;
+    const uint8_t *qbuf = base + warps * NS * Gm::STAGE_BYTES + warp * 2 * Gm::Q_BYTES;
+    const uint32_t bar_s = base_s + warps * (NS * Gm::STAGE_BYTES + 2 * Gm::Q_BYTES) + warp * NS * 8;
+
+    if (lane == 0) {
+        for (int i = 0; i < NS; ++i) mbar_init(bar_s + 8 * i, 1);
+        fence_barrier_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+    }
+    __syncwarp();
+    const uint64_t policy = l2_policy_evict_first();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    const T *qg = static_cast<const T *>(p.q);
+    const int total_units = *p.num_entries * Hkv;
+
+    auto fetch = [&](Unit &x) {
+        int u = 0;
+        if (lane == 0) u = atomicAdd(p.counter, 1);
+        u = __shfl_sync(FULL_MASK, u, 0);
+        x.valid = u < total_units;
+        if (!x.valid) return;
+        const int e = u / Hkv;
+        x.kvh = u - e * Hkv;
+        const int4 ent = p.entries[e];
+        x.s = ent.x;
+        x.part = ent.y;
+        x.ntok = ent.z;
+        x.nparts = ent.w;
+        x.ntiles = (x.ntok + 15) >> 4;
+        const int nblk = (x.ntok + bs - 1) / bs;
+        x.tbl = lane < nblk ? p.block_tables[(size_t)x.s * p.max_blocks_per_seq + x.part * (p.partition / bs) + lane]
+                            : 0;
+    };
+
+    // Item `it` of a unit is its tile `it`: the K and V rows of 16 tokens;
+    // item 0 also brings the unit's G query rows.
+    auto issue = [&](int s, int kvh, int tbl, int qslot, int it, uint32_t stage) {
+        const int tok = 16 * it;
+        const int bi = tok / bs;
+        const int pb = __shfl_sync(FULL_MASK, tbl, bi);
+        if (lane == 0) {
+            const uint32_t bar = bar_s + 8 * stage;
+            const bool ok = (unsigned)pb < (unsigned)p.num_blocks;
+            if (!ok) raise_error(PA_DEVERR_BLOCK_ID);
+            const uint32_t bytes = (ok ? Gm::STAGE_BYTES : 0) + (it == 0 ? Gm::Q_BYTES : 0);
+            fence_proxy_async_smem();
+            if (bytes) {
+                mbar_arrive_expect_tx(bar, bytes);
+                if (ok) {
+                    const int row = (pb * Hkv + kvh) * bs + (tok - bi * bs);
+                    const uint32_t dst = ring_s + stage * Gm::STAGE_BYTES;
+#pragma unroll
+                    for (int b = 0; b < Gm::NBOX; ++b) {
+                        tma_load_2d(dst + b * 2048, &tm_k, 64 * b, row, bar, policy);
+                        tma_load_2d(dst + Gm::HALF_BYTES + b * 2048, &tm_v, 64 * b, row, bar, policy);
+                    }
+                }
+                if (it == 0)
+                    bulk_load(qbuf_s + qslot * Gm::Q_BYTES, qg + ((size_t)s * H + kvh * G) * D, Gm::Q_BYTES, bar,
+                              policy);
+            } else {
+                mbar_arrive(bar);
+            }
+        }
+    };
+
+    Unit cur, nxt;
+    fetch(cur);
+    if (!cur.valid) return;
+    cur.slot = 0;
+    nxt.valid = false;
+    int next_slot = 1;
+    bool prod_on_nxt = false, exhausted = false;
+    int pitem = 0;
+    uint32_t issued = 0, consumed = 0;
+
+    auto produce = [&]() {
+        if (exhausted) return;
+        if (pitem >= (prod_on_nxt ? nxt.ntiles : cur.ntiles)) {
+            if (prod_on_nxt) return;
+            fetch(nxt);
+            if (!nxt.valid) {
+                exhausted = true;
+                return;
+            }
+            nxt.slot = next_slot;
+            next_slot ^= 1;
+            prod_on_nxt = true;
+            pitem = 0;
+        }
+        if (prod_on_nxt)
+            issue(nxt.s, nxt.kvh, nxt.tbl, nxt.slot, pitem, issued % NS);
+        else
+            issue(cur.s, cur.kvh, cur.tbl, cur.slot, pitem, issued % NS);
+        ++pitem;
+        ++issued;
+    };
+
+    auto wait_item = [&]() -> bool {
+        const uint32_t stage = consumed % NS, parity = (consumed / NS) & 1;
+        bool ok = mbar_wait_bounded(bar_s + 8 * stage, parity, WAIT_LIMIT_NS);
+        ok = __all_sync(FULL_MASK, ok);
+        if (!ok) {
+            if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+            for (uint32_t c = consumed; c < issued; ++c)
+                mbar_wait_bounded(bar_s + 8 * (c % NS), (c / NS) & 1, WAIT_LIMIT_NS);
+        }
+        return ok;
+    };
+
+    for (int i = 0; i < NS; ++i) produce();
+
+    // Heads this lane's accumulator columns belong to, and whether they exist.
+    const int h0 = 2 * t4, h1 = 2 * t4 + 1;
+    const bool hv0 = h0 < G, hv1 = h1 < G;
+
+    for (;;) {
+        uint32_t qb[Gm::KS][2];  // B fragments of Q^T: query head g8, 2 columns
+        float o[Gm::KS][4];      // O^T fragments: rows d = 16*i + g8 (+8), heads h0, h1
+        float M0 = -INFINITY, M1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < Gm::KS; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+
+        for (int k = 0; k < cur.ntiles; ++k) {
+            if (!wait_item()) return;
+            const uint32_t stage = consumed % NS;
+            const uint32_t ks_s = ring_s + stage * Gm::STAGE_BYTES;
+            const uint32_t vs_s = ks_s + Gm::HALF_BYTES;
+            if (k == 0) {
+                const uint8_t *qs = qbuf + cur.slot * Gm::Q_BYTES;
+#pragma unroll
+                for (int i = 0; i < Gm::KS; ++i) {
+                    const int d = 16 * i + 2 * t4;
+                    qb[i][0] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
+                    qb[i][1] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 8) * 2) : 0u;
+                }
+            }
+            const int valid = min(16, cur.ntok - 16 * k);
+
+            // ---------------- S^T = K . Q^T ------------------------------------
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+                const int csel = lane >> 4;
+#pragma unroll
+                for (int i = 0; i < Gm::KS; ++i) {
+                    uint32_t a[4];
+                    ldsm_x4(a, ks_s + swz(row, 2 * i + csel));
+                    MmaType<T>::mma(s, a, qb[i][0], qb[i][1]);
+                }
+            }
+            // s[0], s[1]: token g8, heads h0, h1; s[2], s[3]: token g8 + 8.
+            const bool v_lo = g8 < valid, v_hi = g8 + 8 < valid;
+            float x0 = v_lo ? s[0] * p.qscale : -INFINITY;
+            float x1 = v_lo ? s[1] * p.qscale : -INFINITY;
+            float x2 = v_hi ? s[2] * p.qscale : -INFINITY;
+            float x3 = v_hi ? s[3] * p.qscale : -INFINITY;
+            bool raise = (hv0 && !(fmaxf(x0, x2) <= M0 + LAZY_MAX_LOG2)) ||
+                         (hv1 && !(fmaxf(x1, x3) <= M1 + LAZY_MAX_LOG2));
+            if (__any_sync(FULL_MASK, raise)) {
+                float m0 = fmaxf(x0, x2), m1 = fmaxf(x1, x3);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    m0 = fmaxf(m0, __shfl_xor_sync(FULL_MASK, m0, off));
+                    m1 = fmaxf(m1, __shfl_xor_sync(FULL_MASK, m1, off));
+                }
+                const float n0 = fmaxf(M0, m0), n1 = fmaxf(M1, m1);
+                const float a0 = exp2f(M0 - n0), a1 = exp2f(M1 - n1);
+                M0 = n0;
+                M1 = n1;
+                l0 *= a0;
+                l1 *= a1;
+#pragma unroll
+                for (int i = 0; i < Gm::KS; ++i) {
+                    o[i][0] *= a0; o[i][1] *= a1;
+                    o[i][2] *= a0; o[i][3] *= a1;
+                }
+            }
+            // Padding heads (>= G) carry zero scores; give them weight 0.
+            const float p0 = hv0 ? exp2f(x0 - M0) : 0.f, p1 = hv1 ? exp2f(x1 - M1) : 0.f;
+            const float p2 = hv0 ? exp2f(x2 - M0) : 0.f, p3 = hv1 ? exp2f(x3 - M1) : 0.f;
+            const uint32_t w_lo = Elem<T>::pack(p0, p1), w_hi = Elem<T>::pack(p2, p3);
+            {
+                const float2 r_lo = Elem<T>::pair(w_lo), r_hi = Elem<T>::pair(w_hi);
+                l0 += r_lo.x + r_hi.x;
+                l1 += r_lo.y + r_hi.y;
+            }
+            // P^T B fragments: head g8, tokens 2*t4 (+1) and 8 + 2*t4 (+1).
+            const uint32_t pb0 = movmatrix_trans(w_lo), pb1 = movmatrix_trans(w_hi);
+
+            // ---------------- O^T += V^T . P^T ----------------------------------
+            if (valid < 16) {
+                // Stale or never-written slots past the context must not reach
+                // the product (their weight is 0 but 0 * NaN is NaN): zero them.
+                uint8_t *vt = ring + stage * Gm::STAGE_BYTES + Gm::HALF_BYTES;
+                for (int idx = lane; idx < (16 - valid) * Gm::NBOX * 8; idx += 32) {
+                    const int r = valid + idx / (Gm::NBOX * 8);
+                    const int c = idx % (Gm::NBOX * 8);
+                    *reinterpret_cast<uint4 *>(vt + swz(r, c)) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
+                __syncwarp();
+            }
+            {
+                const int row = (lane & 7) + 8 * (lane >> 4);
+                const int csel = (lane >> 3) & 1;
+#pragma unroll
+                for (int i = 0; i < Gm::KS; ++i) {
+                    uint32_t a[4];
+                    ldsm_x4_trans(a, vs_s + swz(row, 2 * i + csel));
+                    MmaType<T>::mma(o[i], a, pb0, pb1);
+                }
+            }
+            ++consumed;
+            __syncwarp();
+            produce();
+        }
+
+        // ---------------- totals and store -------------------------------------
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l0 += __shfl_xor_sync(FULL_MASK, l0, off);
+            l1 += __shfl_xor_sync(FULL_MASK, l1, off);
+        }
+        const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;
+        if (cur.nparts == 1) {
+            const float i0 = hv0 ? 1.f / l0 : 0.f, i1 = hv1 ? 1.f / l1 : 0.f;
+            T *out = static_cast<T *>(p.out) + head0 * D;
+#pragma unroll
+            for (int i = 0; i < Gm::KS; ++i) {
+                // [d][head] pairs -> transpose -> [head g8][d = 2*t4, 2*t4 + 1]
+                const uint32_t lo = movmatrix_trans(Elem<T>::pack(o[i][0] * i0, o[i][1] * i1));
+                const uint32_t hi = movmatrix_trans(Elem<T>::pack(o[i][2] * i0, o[i][3] * i1));
+                if (g8 < G) {
+                    *reinterpret_cast<uint32_t *>(out + g8 * D + 16 * i + 2 * t4) = lo;
+                    *reinterpret_cast<uint32_t *>(out + g8 * D + 16 * i + 8 + 2 * t4) = hi;
+                }
+            }
+        } else {
+            const size_t group = (size_t)cur.s * Hkv + cur.kvh;
+            const size_t row = group * p.max_parts + cur.part;
+            float *acc = p.part_acc + row * (size_t)(D * G);
+#pragma unroll
+            for (int i = 0; i < Gm::KS; ++i) {
+                const int d = 16 * i + g8;
+                if (hv1) {
+                    *reinterpret_cast<float2 *>(acc + d * G + h0) = make_float2(o[i][0], o[i][1]);
+                    *reinterpret_cast<float2 *>(acc + (d + 8) * G + h0) = make_float2(o[i][2], o[i][3]);
+                }
+            }
+            if (g8 == 0 && hv1) {
+                p.ml[row * G + h0] = make_float2(M0, l0);
+                p.ml[row * G + h1] = make_float2(M1, l1);
+            }
+            __threadfence();
+            __syncwarp();
+            int done = 0;
+            if (lane == 0) done = atomicAdd(&p.merge_count[group], 1);
+            done = __shfl_sync(FULL_MASK, done, 0);
+            if (done == cur.nparts - 1) {
+                __threadfence();
+                mma_merge<D, G, T>(p, group, head0, cur.nparts, lane);
+            }
+        }
+
+        while (!prod_on_nxt && !exhausted) produce();
+        if (!prod_on_nxt) break;
+        cur = nxt;
+        prod_on_nxt = false;
+    }
+}
+
+}  // namespace pa
