@@ -100,9 +100,11 @@ PA_API const char *pa_last_error(void);
  *
  * Long contexts are split into partitions of partition_size tokens whose
  * partial results (max, sum, unnormalised output) are merged by the
- * log-sum-exp identity. partition_size = 0 picks one automatically (the whole
- * context when max_context_len <= 512, else 512); otherwise it must be a
- * multiple of 16 and of block_size, with partition_size / block_size <= 32.
+ * log-sum-exp identity. partition_size = 0 picks one automatically: 32
+ * blocks for grouped heads (group >= 2), 256 tokens for one query head per
+ * KV head, or the whole context when max_context_len fits in it. Otherwise it
+ * must be a multiple of 16 and of block_size, with
+ * partition_size / block_size <= 32.
  *
  * max_context_len bounds every context_lens entry (larger ones are clamped and
  * flagged) and sizes the workspace. scale multiplies q.k (1/sqrt(head_dim) for

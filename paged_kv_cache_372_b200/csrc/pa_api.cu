@@ -63,13 +63,15 @@ pa_status device_info(DeviceInfo *out) {
     return PA_OK;
 }
 
-// Largest partition the attention kernel takes: the unit's block-table slice
+// Largest partition the attention kernels take: the unit's block-table slice
 // fits one register per lane (<= 32 blocks).
 int partition_cap(int block_size) { return 32 * block_size; }
 
-// Partition used when the caller passes 0: a whole sequence when every
-// context fits 512 tokens, else 512-token partitions.
-constexpr int kAutoPartition = 512;
+// Partition used when the caller passes 0 (a whole sequence when every
+// context fits in it). The tensor-core kernel streams fast enough per warp
+// that long units (32 blocks) are best; the CUDA-core kernel (one query head
+// per KV head) needs more, shorter units to keep every warp busy.
+int auto_partition(int group, int block_size) { return group >= pa::DECODE_TENSOR_MIN_GROUP ? 32 * block_size : 256; }
 
 bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_size) {
     if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return false;
@@ -80,12 +82,12 @@ bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_si
 }
 
 // Resolves partition_size (0 = auto). Returns 0 for an invalid request.
-int resolve_partition(int block_size, int max_context_len, int requested) {
+int resolve_partition(int group, int block_size, int max_context_len, int requested) {
     if (requested > 0) {
         if (requested % 16 || requested % block_size || requested > partition_cap(block_size)) return 0;
         return requested;
     }
-    const int auto_p = kAutoPartition - kAutoPartition % block_size;
+    const int auto_p = auto_partition(group, block_size);
     if (max_context_len <= auto_p) {
         const int need = max_context_len > 0 ? max_context_len : 1;
         return ((need + block_size - 1) / block_size) * block_size;
@@ -251,7 +253,7 @@ int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int 
                              int max_context_len, int partition_size) {
     if (num_seqs < 0 || max_context_len < 0 || partition_size < 0) return 0;
     if (!shape_supported(num_heads, num_kv_heads, head_dim, block_size)) return 0;
-    return resolve_partition(block_size, max_context_len, partition_size);
+    return resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size);
 }
 
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
@@ -281,7 +283,7 @@ pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
         return fail(PA_ERR_INVALID, "misaligned pointer (16 B tensors, 4 B int arrays, 256 B workspace)");
-    const int P = resolve_partition(block_size, max_context_len, partition_size);
+    const int P = resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size);
     if (P == 0)
         return fail(PA_ERR_INVALID, "partition_size %d (multiple of 16 and of block_size, at most %d)",
                     partition_size, partition_cap(block_size));

@@ -230,10 +230,130 @@ struct Unit {
     bool valid;
 };
 
+// Hands out work-list units to one warp. Claiming a unit is a chain of three
+// dependent global accesses (atomic cursor -> work-list entry -> the unit's
+// block-table slice, one entry per lane); step() advances the chain for the
+// next unit by one link, so that called once per issued tile it has the next
+// unit ready before the warp needs it, and take() only finishes what is left.
+struct UnitSource {
+    const DecodeParams *p;
+    int lane, total_units, Hkv, bs, blocks_per_part;
+    int state;  // 0 idle, 1 cursor claimed, 2 entry loaded, 3 table loaded, 4 list exhausted
+    int u, tbl;
+    int4 ent;
+
+    __device__ void init(const DecodeParams &params, int lane_id, int total) {
+        p = &params;
+        lane = lane_id;
+        total_units = total;
+        Hkv = params.num_kv_heads;
+        bs = params.block_size;
+        blocks_per_part = params.partition / params.block_size;
+        state = 0;
+        u = 0;
+        tbl = 0;
+        ent = make_int4(0, 0, 0, 0);
+    }
+
+    __device__ __forceinline__ void step() {
+        if (state == 0) {
+            int v = 0;
+            if (lane == 0) v = atomicAdd(p->counter, 1);
+            u = v;  // lane 0 only; broadcast in the next link
+            state = 1;
+        } else if (state == 1) {
+            u = __shfl_sync(FULL_MASK, u, 0);
+            if (u >= total_units) {
+                state = 4;
+                return;
+            }
+            ent = p->entries[u / Hkv];
+            state = 2;
+        } else if (state == 2) {
+            const int nblk = (ent.z + bs - 1) / bs;
+            tbl = lane < nblk ? p->block_tables[(size_t)ent.x * p->max_blocks_per_seq + ent.y * blocks_per_part + lane]
+                              : 0;
+            state = 3;
+        }
+    }
+
+    // Finishes claiming the next unit; x.valid is false once the list is done.
+    __device__ __forceinline__ void take(Unit &x) {
+        while (state < 3) step();
+        x.valid = state == 3;
+        if (!x.valid) return;
+        const int e = u / Hkv;
+        x.kvh = u - e * Hkv;
+        x.s = ent.x;
+        x.part = ent.y;
+        x.ntok = ent.z;
+        x.nparts = ent.w;
+        x.ntiles = (ent.z + 15) >> 4;
+        x.tbl = tbl;
+        state = 0;
+    }
+};
+
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
-// Merge of the partitions of one (sequence, KV head) by the log-sum-exp
-// identity: out = sum_j 2^(m_j - M) acc_j / sum_j 2^(m_j - M) l_j.
+// Merge of the partitions of one head by the log-sum-exp identity:
+//   out = sum_j 2^(m_j - M) acc_j / sum_j 2^(m_j - M) l_j,  M = max_j m_j.
+// ml(j) returns partition j's (m, l); acc(j) points at this lane's EPL floats
+// of partition j's unnormalised output. Lane j computes partition j's weight
+// (32 partitions per round) and the weights reach the other lanes by shuffle,
+// so the output loop only waits on its own independent loads.
+template <int EPL, typename ML, typename ACC>
+__device__ __forceinline__ void merge_head(int nparts, int lane, ML ml, ACC acc, float (&o)[EPL]) {
+    float M = -INFINITY;
+    for (int j = lane; j < nparts; j += 32) M = fmaxf(M, ml(j).x);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
+    float L = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) o[e] = 0.f;
+    for (int base = 0; base < nparts; base += 32) {
+        float w = 0.f;
+        if (base + lane < nparts) {
+            const float2 v = ml(base + lane);
+            w = exp2f(v.x - M);
+            L = fmaf(w, v.y, L);
+        }
+        const int n = min(32, nparts - base);
+#pragma unroll 8
+        for (int jj = 0; jj < n; ++jj) {
+            const float wj = __shfl_sync(FULL_MASK, w, jj);
+            const float *a = acc(base + jj);
+            if constexpr (EPL == 4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(a));
+                o[0] = fmaf(wj, v.x, o[0]); o[1] = fmaf(wj, v.y, o[1]);
+                o[2] = fmaf(wj, v.z, o[2]); o[3] = fmaf(wj, v.w, o[3]);
+            } else {
+                const float2 v = __ldcg(reinterpret_cast<const float2 *>(a));
+                o[0] = fmaf(wj, v.x, o[0]); o[1] = fmaf(wj, v.y, o[1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(FULL_MASK, L, off);
+    const float inv = 1.f / L;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) o[e] *= inv;
+}
+
+template <int EPL, typename T>
+__device__ __forceinline__ void store_row(T *dst, const float (&o)[EPL]) {
+    if constexpr (EPL == 4) {
+        uint2 w;
+        w.x = Elem<T>::pack(o[0], o[1]);
+        w.y = Elem<T>::pack(o[2], o[3]);
+        *reinterpret_cast<uint2 *>(dst) = w;
+    } else {
+        *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(o[0], o[1]);
+    }
+}
+
+// Merge for the CUDA-core kernel's partial layout: [head][part][D] floats,
+// [head][part] (max, sum) pairs.
 template <int D, int G, typename T>
 __device__ __forceinline__ void merge_partitions(const DecodeParams &p, size_t head0, int nparts, int lane) {
     constexpr int EPL = D / 32;
@@ -241,38 +361,11 @@ __device__ __forceinline__ void merge_partitions(const DecodeParams &p, size_t h
 #pragma unroll 1
     for (int g = 0; g < G; ++g) {
         const size_t row0 = (head0 + g) * p.max_parts;
-        float M = -INFINITY;
-        for (int j = lane; j < nparts; j += 32) M = fmaxf(M, __ldcg(&p.ml[row0 + j].x));
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
-        float L = 0.f, o[EPL];
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) o[e] = 0.f;
-#pragma unroll 4
-        for (int j = 0; j < nparts; ++j) {
-            const float2 ml = __ldcg(&p.ml[row0 + j]);
-            const float w = exp2f(ml.x - M);
-            L = fmaf(w, ml.y, L);
-            const float *a = p.part_acc + (row0 + j) * D + lane * EPL;
-            if constexpr (EPL == 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(a));
-                o[0] = fmaf(w, v.x, o[0]); o[1] = fmaf(w, v.y, o[1]);
-                o[2] = fmaf(w, v.z, o[2]); o[3] = fmaf(w, v.w, o[3]);
-            } else {
-                const float2 v = __ldcg(reinterpret_cast<const float2 *>(a));
-                o[0] = fmaf(w, v.x, o[0]); o[1] = fmaf(w, v.y, o[1]);
-            }
-        }
-        const float inv = 1.f / L;
-        T *dst = out + (head0 + g) * D + lane * EPL;
-        if constexpr (EPL == 4) {
-            uint2 w;
-            w.x = Elem<T>::pack(o[0] * inv, o[1] * inv);
-            w.y = Elem<T>::pack(o[2] * inv, o[3] * inv);
-            *reinterpret_cast<uint2 *>(dst) = w;
-        } else {
-            *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(o[0] * inv, o[1] * inv);
-        }
+        float o[EPL];
+        merge_head<EPL>(
+            nparts, lane, [&](int j) { return __ldcg(&p.ml[row0 + j]); },
+            [&](int j) { return p.part_acc + (row0 + j) * D + lane * EPL; }, o);
+        store_row<EPL>(out + (head0 + g) * D + lane * EPL, o);
     }
 }
 
@@ -316,24 +409,9 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
     const int g0 = G >= 2 ? (dg & 1) * Gm::R : 0;
     const bool owner = G >= 2 || dg == 0;
 
-    auto fetch = [&](Unit &x) {
-        int u = 0;
-        if (lane == 0) u = atomicAdd(p.counter, 1);
-        u = __shfl_sync(FULL_MASK, u, 0);
-        x.valid = u < total_units;
-        if (!x.valid) return;
-        const int e = u / Hkv;
-        x.kvh = u - e * Hkv;
-        const int4 ent = p.entries[e];
-        x.s = ent.x;
-        x.part = ent.y;
-        x.ntok = ent.z;
-        x.nparts = ent.w;
-        x.ntiles = (x.ntok + 15) >> 4;
-        const int nblk = (x.ntok + bs - 1) / bs;
-        x.tbl = lane < nblk ? p.block_tables[(size_t)x.s * p.max_blocks_per_seq + x.part * (p.partition / bs) + lane]
-                            : 0;
-    };
+    UnitSource src;
+    src.init(p, lane, total_units);
+    auto fetch = [&](Unit &x) { src.take(x); };
 
     // Item `it` of a unit: even items are K tiles, odd items V tiles (tile it/2);
     // item 0 also brings the unit's G query rows.
@@ -396,6 +474,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
             issue(cur.s, cur.kvh, cur.tbl, cur.slot, pitem, issued % NS);
         ++pitem;
         ++issued;
+        src.step();  // one link of the next unit's claim per issued item
     };
 
     // Wait for the consumer's next item; on a timeout flag it, wait (bounded)

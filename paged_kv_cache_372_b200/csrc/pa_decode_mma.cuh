@@ -104,56 +104,75 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)((chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
-// Merge of one (sequence, KV head)'s partitions, partial layout
-// [part][D][G] floats and [part][G] (max, sum) pairs.
+// Merge of one (sequence, KV head)'s partitions for this kernel's partial
+// layout: [part][D][G] floats and [part][G] (max, sum) pairs (head-innermost,
+// so the accumulator fragments store as pairs). All G heads in one pass: lane
+// j computes partition j's G weights (32 partitions per round), the weights
+// reach the other lanes by shuffle, and each lane reads its EPL x G contiguous
+// floats of every partition with vector loads.
 template <int D, int G, typename T>
 __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, size_t head0, int nparts, int lane) {
     constexpr int EPL = D / 32;
+    constexpr int NV4 = EPL * G / 4;  // float4 loads per partition per lane
     const float2 *ml = p.ml + group * p.max_parts * G;
     const float *acc = p.part_acc + group * p.max_parts * (size_t)(D * G);
-    float M[G], L[G], o[EPL][G];
+    float M[G], L[G], o[EPL * G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         M[g] = -INFINITY;
         L[g] = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) o[e][g] = 0.f;
     }
-    for (int j = 0; j < nparts; ++j)
+#pragma unroll
+    for (int i = 0; i < EPL * G; ++i) o[i] = 0.f;
+    for (int j = lane; j < nparts; j += 32)
 #pragma unroll
         for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __ldcg(&ml[j * G + g].x));
-#pragma unroll 2
-    for (int j = 0; j < nparts; ++j) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __shfl_xor_sync(FULL_MASK, M[g], off));
+    for (int base = 0; base < nparts; base += 32) {
         float w[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float2 v = __ldcg(&ml[j * G + g]);
-            w[g] = exp2f(v.x - M[g]);
-            L[g] = fmaf(w[g], v.y, L[g]);
-        }
-        const float *a = acc + (size_t)j * D * G + lane * EPL * G;
+        for (int g = 0; g < G; ++g) w[g] = 0.f;
+        if (base + lane < nparts) {
 #pragma unroll
-        for (int e = 0; e < EPL; ++e)
-#pragma unroll
-            for (int g = 0; g < G; g += 2) {
-                const float2 v = __ldcg(reinterpret_cast<const float2 *>(a + e * G + g));
-                o[e][g] = fmaf(w[g], v.x, o[e][g]);
-                o[e][g + 1] = fmaf(w[g + 1], v.y, o[e][g + 1]);
+            for (int g = 0; g < G; ++g) {
+                const float2 v = __ldcg(&ml[(base + lane) * G + g]);
+                w[g] = exp2f(v.x - M[g]);
+                L[g] = fmaf(w[g], v.y, L[g]);
             }
+        }
+        const int n = min(32, nparts - base);
+#pragma unroll 4
+        for (int jj = 0; jj < n; ++jj) {
+            const float4 *a = reinterpret_cast<const float4 *>(acc + (size_t)(base + jj) * D * G + lane * EPL * G);
+            float4 v[NV4];
+#pragma unroll
+            for (int i = 0; i < NV4; ++i) v[i] = __ldcg(a + i);
+            float wj[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) wj[g] = __shfl_sync(FULL_MASK, w[g], jj);
+#pragma unroll
+            for (int i = 0; i < NV4; ++i) {
+                const float f[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) o[4 * i + c] = fmaf(wj[(4 * i + c) % G], f[c], o[4 * i + c]);
+            }
+        }
     }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) L[g] += __shfl_xor_sync(FULL_MASK, L[g], off);
     T *out = static_cast<T *>(p.out);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         const float inv = 1.f / L[g];
-        T *dst = out + (head0 + g) * D + lane * EPL;
-        if constexpr (EPL == 4) {
-            uint2 w;
-            w.x = Elem<T>::pack(o[0][g] * inv, o[1][g] * inv);
-            w.y = Elem<T>::pack(o[2][g] * inv, o[3][g] * inv);
-            *reinterpret_cast<uint2 *>(dst) = w;
-        } else {
-            *reinterpret_cast<uint32_t *>(dst) = Elem<T>::pack(o[0][g] * inv, o[1][g] * inv);
-        }
+        float r[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) r[e] = o[e * G + g] * inv;
+        store_row<EPL>(out + (head0 + g) * D + lane * EPL, r);
     }
 }
 
@@ -192,24 +211,9 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     const T *qg = static_cast<const T *>(p.q);
     const int total_units = *p.num_entries * Hkv;
 
-    auto fetch = [&](Unit &x) {
-        int u = 0;
-        if (lane == 0) u = atomicAdd(p.counter, 1);
-        u = __shfl_sync(FULL_MASK, u, 0);
-        x.valid = u < total_units;
-        if (!x.valid) return;
-        const int e = u / Hkv;
-        x.kvh = u - e * Hkv;
-        const int4 ent = p.entries[e];
-        x.s = ent.x;
-        x.part = ent.y;
-        x.ntok = ent.z;
-        x.nparts = ent.w;
-        x.ntiles = (x.ntok + 15) >> 4;
-        const int nblk = (x.ntok + bs - 1) / bs;
-        x.tbl = lane < nblk ? p.block_tables[(size_t)x.s * p.max_blocks_per_seq + x.part * (p.partition / bs) + lane]
-                            : 0;
-    };
+    UnitSource src;
+    src.init(p, lane, total_units);
+    auto fetch = [&](Unit &x) { src.take(x); };
 
     // Item `it` of a unit is its tile `it`: the K and V rows of 16 tokens;
     // item 0 also brings the unit's G query rows.
@@ -273,6 +277,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             issue(cur.s, cur.kvh, cur.tbl, cur.slot, pitem, issued % NS);
         ++pitem;
         ++issued;
+        src.step();  // one link of the next unit's claim per issued item
     };
 
     auto wait_item = [&]() -> bool {

@@ -80,9 +80,22 @@ class Workload:
         return self.num_kv_heads * self.block_size * self.head_dim * 2
 
     def kv_bytes(self, step: int = 0) -> int:
-        """Algorithmic K+V bytes one decode reads: valid tokens only."""
+        """Algorithmic K+V bytes one decode reads: valid tokens only, counted
+        once per sequence (logical bytes; shared blocks count every time)."""
         return int(self.steps[step].context_lens.astype(np.int64).sum()) * \
             self.num_kv_heads * self.head_dim * 2 * 2
+
+    def kv_bytes_unique(self, step: int = 0) -> int:
+        """K+V bytes of the distinct physical block slots one decode reads:
+        a block shared by several sequences counts once (its longest use)."""
+        st = self.steps[step]
+        used = {}
+        for s, n in enumerate(st.context_lens):
+            n = int(n)
+            for j in range(-(-n // self.block_size)):
+                b = int(st.block_tables[s, j])
+                used[b] = max(used.get(b, 0), min(self.block_size, n - j * self.block_size))
+        return sum(used.values()) * self.num_kv_heads * self.head_dim * 2 * 2
 
 
 def _pool(num_blocks, hkv, bs, d, dtype, gen):
