@@ -85,10 +85,14 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# The files that define the decode kernels and how they are launched.
+KERNEL_SOURCES = ("pa_common.cuh", "pa_decode.cuh", "pa_decode_mma.cuh", "pa_launch.cuh")
+
+
 def source_digest() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_372_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -277,7 +281,8 @@ def run_ours(args, world, rank, local):
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "kernel": "pa_decode call (plan + attention launches; split merge fused)",
                      "bytes": "unique K+V bytes of valid tokens per call",
-                     "traffic": profiled_traffic(wl.name)},
+                     "traffic": profiled_traffic(wl.name if args.partition is None
+                                                 else f"{wl.name}@P{args.partition}")},
         "gpu_launches": launches,
         "clocks": clk,
     }

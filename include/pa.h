@@ -178,6 +178,15 @@ PA_API pa_status pa_device_errors(unsigned int *flags, int clear, pa_stream_t st
 /* Number of SMs the library sizes its persistent grids for (current device). */
 PA_API int pa_num_sms(void);
 
+/*
+ * Self-test of the kernels' bounded device-side waits: launches one warp that
+ * waits on an mbarrier nothing will ever complete, for at most limit_ns
+ * nanoseconds (1 ms .. 10 s), then sets PA_DEVERR_TIMEOUT and returns — the
+ * same path every pipeline wait in pa_decode takes if a copy never lands.
+ * Asynchronous; read the result with pa_device_errors().
+ */
+PA_API pa_status pa_selftest_bounded_wait(unsigned long long limit_ns, pa_stream_t stream);
+
 /* Size of the fixed scratch array behind pa_decode_noalloc (16 MiB). */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
 

@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint), _I, _P]
         L.pa_num_sms.restype = _I
         L.pa_num_sms.argtypes = []
+        L.pa_selftest_bounded_wait.restype = _I
+        L.pa_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _P]
         L.pa_decode_noalloc.restype = _I
         L.pa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]
         _lib = L
@@ -196,6 +198,11 @@ def pa_device_errors(clear: bool = True, stream=None) -> int:
 
 def pa_num_sms() -> int:
     return int(lib().pa_num_sms())
+
+
+def pa_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self-test kernel (sets DEVERR_TIMEOUT when it ends)."""
+    _check(lib().pa_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

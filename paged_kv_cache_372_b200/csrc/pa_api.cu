@@ -13,8 +13,6 @@
 #include "pa_decode.cuh"
 #include "pa_decode_mma.cuh"
 
-#include <cudaTypedefs.h>
-
 namespace {
 
 thread_local std::string g_last_error;
@@ -63,170 +61,26 @@ pa_status device_info(DeviceInfo *out) {
     return PA_OK;
 }
 
-// Largest partition the attention kernels take: the unit's block-table slice
-// fits one register per lane (<= 32 blocks).
-int partition_cap(int block_size) { return 32 * block_size; }
-
-// Partition used when the caller passes 0 (a whole sequence when every
-// context fits in it). The tensor-core kernel streams fast enough per warp
-// that long units (32 blocks) are best; the CUDA-core kernel (one query head
-// per KV head) needs more, shorter units to keep every warp busy.
-int auto_partition(int group, int block_size) { return group >= pa::DECODE_TENSOR_MIN_GROUP ? 32 * block_size : 256; }
-
-bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_size) {
-    if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return false;
-    const int g = num_heads / num_kv_heads;
-    if (g != 1 && g != 2 && g != 4 && g != 8) return false;
-    if (head_dim != 64 && head_dim != 128) return false;
-    return block_size == 16 || block_size == 32 || block_size == 64;
-}
-
-// Resolves partition_size (0 = auto). Returns 0 for an invalid request.
-int resolve_partition(int group, int block_size, int max_context_len, int requested) {
-    if (requested > 0) {
-        if (requested % 16 || requested % block_size || requested > partition_cap(block_size)) return 0;
-        return requested;
-    }
-    const int auto_p = auto_partition(group, block_size);
-    if (max_context_len <= auto_p) {
-        const int need = max_context_len > 0 ? max_context_len : 1;
-        return ((need + block_size - 1) / block_size) * block_size;
-    }
-    return auto_p;
-}
-
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
-template <int D, int G, typename T>
-pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
-    constexpr int NS = pa::DECODE_STAGES;
-    DeviceInfo info;
-    pa_status st = device_info(&info);
-    if (st != PA_OK) return st;
-    const int per_warp = pa::warp_smem_bytes<D, G, NS>();
-    int warps = info.smem_optin / per_warp;
-    if (warps > pa::DECODE_MAX_WARPS) warps = pa::DECODE_MAX_WARPS;
-    if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "%d bytes of shared memory per warp", per_warp);
-    const int smem = warps * per_warp;
-    auto kernel = pa::pa_decode_kernel<D, G, T, NS>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+}  // namespace
 
-    pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
-    // Programmatic dependent launch: the attention CTAs start their set-up
-    // while the plan kernel runs and wait for its results in-kernel.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(info.sms);
-    cfg.blockDim = dim3(warps * 32);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, p);
-    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
-    return PA_OK;
-}
+#include "pa_launch.cuh"
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
-pa_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled *out) {
-    static std::mutex mu;
-    static PFN_cuTensorMapEncodeTiled fn = nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
-        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !ptr)
-            return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(ptr);
+namespace {
+
+// One warp waits, with a limit, on an mbarrier that never completes.
+__global__ void pa_bounded_wait_probe(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t bar_s = pa::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        pa::mbar_init(bar_s, 1);
+        pa::fence_barrier_init();
     }
-    *out = fn;
-    return PA_OK;
-}
-
-// A pool [num_blocks][num_kv_heads][block_size][D] as a 2-D tensor of
-// rows x D elements, read in boxes of 16 rows x 64 columns (128 bytes) with
-// the 128-byte shared-memory swizzle.
-template <typename T>
-pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, int D) {
-    PFN_cuTensorMapEncodeTiled enc;
-    pa_status st = tensor_map_encoder(&enc);
-    if (st != PA_OK) return st;
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, 16};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, pa::MmaType<T>::tma_type, 2, const_cast<void *>(pool), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return PA_OK;
-}
-
-template <int D, int G, typename T>
-pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
-    constexpr int NS = pa::DECODE_MMA_STAGES;
-    DeviceInfo info;
-    pa_status st = device_info(&info);
-    if (st != PA_OK) return st;
-    const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
-    if (rows >= (1ll << 31)) return fail(PA_ERR_UNSUPPORTED, "pool has %lld rows, above 2^31", rows);
-    CUtensorMap tmk, tmv;
-    if ((st = encode_pool_map<T>(&tmk, p.k_pool, rows, D)) != PA_OK) return st;
-    if ((st = encode_pool_map<T>(&tmv, p.v_pool, rows, D)) != PA_OK) return st;
-    int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS>();
-    if (warps > pa::DECODE_MAX_WARPS) warps = pa::DECODE_MAX_WARPS;
-    if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "not enough shared memory for one warp");
-    const int smem = pa::mma_smem_bytes<D, G, NS>(warps);
-    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-
-    pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(info.sms);
-    cfg.blockDim = dim3(warps * 32);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, p, tmk, tmv);
-    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
-    return PA_OK;
-}
-
-template <int D, typename T>
-pa_status dispatch_group(pa::DecodeParams &p, int group, cudaStream_t stream) {
-    if (group >= pa::DECODE_TENSOR_MIN_GROUP) {
-        switch (group) {
-            case 2: return launch_decode_mma<D, 2, T>(p, stream);
-            case 4: return launch_decode_mma<D, 4, T>(p, stream);
-            case 8: return launch_decode_mma<D, 8, T>(p, stream);
-        }
-    }
-    switch (group) {
-        case 1: return launch_decode<D, 1, T>(p, stream);
-#if PA_DECODE_TENSOR_MIN_GROUP > 2
-        case 2: return launch_decode<D, 2, T>(p, stream);
-#endif
-#if PA_DECODE_TENSOR_MIN_GROUP > 4
-        case 4: return launch_decode<D, 4, T>(p, stream);
-#endif
-#if PA_DECODE_TENSOR_MIN_GROUP > 8
-        case 8: return launch_decode<D, 8, T>(p, stream);
-#endif
-    }
-    return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
+    __syncwarp();
+    bool ok = pa::mbar_wait_bounded(bar_s, 0, limit_ns);
+    ok = __all_sync(pa::FULL_MASK, ok);
+    if (!ok && threadIdx.x == 0) pa::raise_error(PA_DEVERR_TIMEOUT);
 }
 
 }  // namespace
@@ -400,6 +254,16 @@ pa_status pa_device_errors(unsigned int *flags, int clear, pa_stream_t stream) {
     }
     if (flags) *flags = v;
     return v ? PA_ERR_DEVICE_CHECK : PA_OK;
+}
+
+pa_status pa_selftest_bounded_wait(unsigned long long limit_ns, pa_stream_t stream) {
+    g_last_error.clear();
+    if (limit_ns < 1000000ull || limit_ns > 10000000000ull)
+        return fail(PA_ERR_INVALID, "limit %llu ns outside [1 ms, 10 s]", limit_ns);
+    pa_bounded_wait_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "bounded-wait probe launch");
+    return PA_OK;
 }
 
 int pa_num_sms(void) {

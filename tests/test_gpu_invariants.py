@@ -190,3 +190,20 @@ def test_cpu_tensors_are_rejected():
     with pytest.raises(ValueError):
         pa.pa_decode(torch.empty_like(st.q), st.q, wl.k_pool, wl.v_pool,
                      torch.as_tensor(st.block_tables), torch.as_tensor(st.context_lens), wl.scale, 33)
+
+
+def test_bounded_wait_runs_out_reports_and_leaves_the_context_usable():
+    """A device-side wait that nothing completes ends at its limit with
+    DEVERR_TIMEOUT instead of hanging; decoding works afterwards."""
+    import time
+    pa.pa_device_errors(clear=True)
+    t0 = time.perf_counter()
+    pa.pa_selftest_bounded_wait(20_000_000)          # 20 ms
+    flags = pa.pa_device_errors(clear=True)
+    elapsed = time.perf_counter() - t0
+    assert flags & pa.DEVERR_TIMEOUT
+    assert 0.015 < elapsed < 5.0
+    wl = workloads.tiny(0)
+    st = wl.steps[0]
+    out = decode(wl, wl.k_pool.cuda(), wl.v_pool.cuda(), st.block_tables, st.context_lens)
+    assert torch.isfinite(out.float()).all() and pa.pa_device_errors() == 0
