@@ -207,12 +207,14 @@ __host__ __device__ constexpr int warp_smem_bytes() {
 #define PA_DECODE_MAX_WARPS 12
 #endif
 // Ring stages (each one 16-token K+V tile) of the tensor-core kernel, and the
-// smallest head group that uses it (smaller groups use the CUDA-core kernel).
+// smallest head group that uses it; smaller groups use the CUDA-core kernel
+// (by default every group uses the tensor-core kernel; building with
+// -DPA_DECODE_TENSOR_MIN_GROUP=16 selects the CUDA-core kernel everywhere).
 #ifndef PA_DECODE_MMA_STAGES
 #define PA_DECODE_MMA_STAGES 2
 #endif
 #ifndef PA_DECODE_TENSOR_MIN_GROUP
-#define PA_DECODE_TENSOR_MIN_GROUP 2
+#define PA_DECODE_TENSOR_MIN_GROUP 1
 #endif
 constexpr int DECODE_STAGES = PA_DECODE_STAGES;
 constexpr int DECODE_MAX_WARPS = PA_DECODE_MAX_WARPS;

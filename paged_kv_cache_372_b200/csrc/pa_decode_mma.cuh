@@ -1,4 +1,4 @@
-// Paged decode attention on tensor cores, for grouped-query heads (G >= 2).
+// Paged decode attention on tensor cores (the default kernel, any head group).
 //
 // Same work list, unit scheduling, online softmax and split merge as
 // pa_decode_kernel (pa_decode.cuh); the per-tile arithmetic differs. With G
@@ -25,7 +25,7 @@ namespace pa {
 
 template <int D, int G>
 struct MmaGeo {
-    static_assert(G == 2 || G == 4 || G == 8, "tensor-core path covers grouped heads");
+    static_assert(G == 1 || G == 2 || G == 4 || G == 8, "head group size");
     static constexpr int KS = D / 16;                    // 16-wide slices of a row
     static constexpr int NBOX = D / 64;                  // 128-byte TMA boxes per row
     static constexpr int HALF_BYTES = 16 * D * 2;        // one K (or V) tile
@@ -113,7 +113,8 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 template <int D, int G, typename T>
 __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, size_t head0, int nparts, int lane) {
     constexpr int EPL = D / 32;
-    constexpr int NV4 = EPL * G / 4;  // float4 loads per partition per lane
+    constexpr int VW = EPL * G >= 4 ? 4 : EPL * G;  // floats per vector load (4 or 2)
+    constexpr int NV4 = EPL * G / VW;               // vector loads per partition per lane
     const float2 *ml = p.ml + group * p.max_parts * G;
     const float *acc = p.part_acc + group * p.max_parts * (size_t)(D * G);
     float M[G], L[G], o[EPL * G];
@@ -146,19 +147,23 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
         const int n = min(32, nparts - base);
 #pragma unroll 4
         for (int jj = 0; jj < n; ++jj) {
-            const float4 *a = reinterpret_cast<const float4 *>(acc + (size_t)(base + jj) * D * G + lane * EPL * G);
-            float4 v[NV4];
+            const float *a = acc + (size_t)(base + jj) * D * G + lane * EPL * G;
+            float f[EPL * G];
 #pragma unroll
-            for (int i = 0; i < NV4; ++i) v[i] = __ldcg(a + i);
+            for (int i = 0; i < NV4; ++i) {
+                if constexpr (VW == 4) {
+                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(a) + i);
+                    f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
+                } else {
+                    const float2 v = __ldcg(reinterpret_cast<const float2 *>(a) + i);
+                    f[2 * i] = v.x; f[2 * i + 1] = v.y;
+                }
+            }
             float wj[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) wj[g] = __shfl_sync(FULL_MASK, w[g], jj);
 #pragma unroll
-            for (int i = 0; i < NV4; ++i) {
-                const float f[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-                for (int c = 0; c < 4; ++c) o[4 * i + c] = fmaf(wj[(4 * i + c) % G], f[c], o[4 * i + c]);
-            }
+            for (int c = 0; c < EPL * G; ++c) o[c] = fmaf(wj[c % G], f[c], o[c]);
         }
     }
 #pragma unroll
@@ -429,15 +434,18 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
 #pragma unroll
             for (int i = 0; i < Gm::KS; ++i) {
                 const int d = 16 * i + g8;
-                if (hv1) {
+                if constexpr (G == 1) {
+                    if (hv0) {
+                        acc[d] = o[i][0];
+                        acc[d + 8] = o[i][2];
+                    }
+                } else if (hv1) {
                     *reinterpret_cast<float2 *>(acc + d * G + h0) = make_float2(o[i][0], o[i][1]);
                     *reinterpret_cast<float2 *>(acc + (d + 8) * G + h0) = make_float2(o[i][2], o[i][3]);
                 }
             }
-            if (g8 == 0 && hv1) {
-                p.ml[row * G + h0] = make_float2(M0, l0);
-                p.ml[row * G + h1] = make_float2(M1, l1);
-            }
+            if (g8 == 0 && hv0) p.ml[row * G + h0] = make_float2(M0, l0);
+            if (g8 == 0 && hv1) p.ml[row * G + h1] = make_float2(M1, l1);
             __threadfence();
             __syncwarp();
             int done = 0;

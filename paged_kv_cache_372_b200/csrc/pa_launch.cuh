@@ -15,10 +15,9 @@ namespace {
 int partition_cap(int block_size) { return 32 * block_size; }
 
 // Partition used when the caller passes 0 (a whole sequence when every
-// context fits in it). The tensor-core kernel streams fast enough per warp
-// that long units (32 blocks) are best; the CUDA-core kernel (one query head
-// per KV head) needs more, shorter units to keep every warp busy.
-int auto_partition(int group, int block_size) { return group >= pa::DECODE_TENSOR_MIN_GROUP ? 32 * block_size : 256; }
+// context fits in it): 32 blocks for grouped heads, 256 tokens for one query
+// head per KV head (measured best on the benchmark workloads).
+int auto_partition(int group, int block_size) { return group >= 2 ? 32 * block_size : 256; }
 
 bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_size) {
     if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return false;
@@ -154,13 +153,18 @@ template <int D, typename T>
 pa_status dispatch_group(pa::DecodeParams &p, int group, cudaStream_t stream) {
     if (group >= pa::DECODE_TENSOR_MIN_GROUP) {
         switch (group) {
+#if PA_DECODE_TENSOR_MIN_GROUP <= 1
+            case 1: return launch_decode_mma<D, 1, T>(p, stream);
+#endif
             case 2: return launch_decode_mma<D, 2, T>(p, stream);
             case 4: return launch_decode_mma<D, 4, T>(p, stream);
             case 8: return launch_decode_mma<D, 8, T>(p, stream);
         }
     }
     switch (group) {
+#if PA_DECODE_TENSOR_MIN_GROUP > 1
         case 1: return launch_decode<D, 1, T>(p, stream);
+#endif
 #if PA_DECODE_TENSOR_MIN_GROUP > 2
         case 2: return launch_decode<D, 2, T>(p, stream);
 #endif

@@ -22,6 +22,7 @@ def test_host_only_entry_points():
     # partition choice and workspace size are pure host functions
     assert pa.pa_decode_partition_size(8, 32, 8, 128, 64, 32768, 512) == 512
     assert pa.pa_decode_partition_size(4, 2, 2, 64, 16, 33, 0) == 48        # one partition
+    assert pa.pa_decode_partition_size(64, 32, 32, 128, 16, 2048, 0) == 256  # one head per KV head
     assert pa.pa_decode_partition_size(4, 2, 2, 64, 16, 33, 24) == 0        # not a multiple of 16
     assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 100, 0) == 112    # group 8: one partition
     assert pa.pa_decode_partition_size(4, 32, 4, 128, 16, 8192, 0) == 512   # 512-token partitions
