@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--unfused", action="store_true",
+                    help="separate cache-write launch instead of pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
@@ -73,6 +75,19 @@ L2_BYTES = 126 * 1024 * 1024
 
 def needs_flush(wl) -> bool:
     return wl.kv_bytes_unique() < 4 * L2_BYTES
+
+
+def appends_at_last_positions(wl) -> bool:
+    """True when every step's first num_seqs new tokens are each sequence's
+    last position, so the fused append + decode entry point applies."""
+    for st in wl.steps:
+        B = st.q.shape[0]
+        for s in range(B):
+            n = int(st.context_lens[s])
+            if n == 0 or st.slot_mapping[s] != st.block_tables[s, (n - 1) // wl.block_size] * wl.block_size + \
+                    (n - 1) % wl.block_size:
+                return False
+    return True
 
 
 def measured_peaks():
@@ -212,17 +227,31 @@ def run_ours(args, world, rank, local):
     flush = needs_flush(wl)
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
 
+    fused = not args.unfused and appends_at_last_positions(wl)
+    for d in dev_steps:
+        d["k_dec"], d["v_dec"] = d["k"][:B].contiguous(), d["v"][:B].contiguous()
+        d["k_extra"], d["v_extra"], d["slots_extra"] = d["k"][B:], d["v"][B:], d["slots"][B:]
+
     def step(i, ev=None):
         d = dev_steps[i % nsteps]
         n = 0
         if d["pairs"].shape[0]:
             pa.pa_copy_blocks([kp, vp], d["pairs"])
             n += 1
-        pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
-        n += 1
+        if fused:
+            if d["slots_extra"].shape[0]:
+                pa.pa_reshape_and_cache(d["k_extra"], d["v_extra"], kp, vp, d["slots_extra"])
+                n += 1
+        else:
+            pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
+            n += 1
         if ev is not None:
             ev[0].record(stream)
-        pa.pa_decode(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws)
+        if fused:
+            pa.pa_decode_append(d["out"], d["q"], d["k_dec"], d["v_dec"], kp, vp, d["tables"], d["ctx"], wl.scale,
+                                max_ctx, P, ws)
+        else:
+            pa.pa_decode(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws)
         if ev is not None:
             ev[1].record(stream)
         return n + launches_per_decode
@@ -279,24 +308,28 @@ def run_ours(args, world, rank, local):
         "hbm_frac_of_nominal_8000": achieved / 8000.0,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
-                     "kernel": "pa_decode call (plan + attention launches; split merge fused)",
+                     "kernel": ("pa_decode_append call (plan + attention launches; cache write and split "
+                                "merge fused)" if fused else
+                                "pa_decode call (plan + attention launches; split merge fused)"),
                      "bytes": "unique K+V bytes of valid tokens per call",
                      "traffic": profiled_traffic(wl.name if args.partition is None
                                                  else f"{wl.name}@P{args.partition}")},
         "gpu_launches": launches,
+        "step": ("pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_append"
+                 if fused else "pa_copy_blocks (if any), pa_reshape_and_cache, pa_decode"),
         "clocks": clk,
     }
     if rank == 0 and not args.no_e2e:
-        result["e2e"] = run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world)
+        result["e2e"] = run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused)
     elif not args.no_e2e:
-        run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world)
+        run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused)
     pa.pa_device_errors()
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(wl)
     return result
 
 
-def run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world):
+def run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused):
     """Same metric through the public API with host buffers: every step copies its
     inputs from pinned host memory and reads the output back."""
     nsteps = len(wl.steps)
@@ -318,9 +351,15 @@ def run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world):
         d = {k: h[k].to(dev, non_blocking=True) for k in ("q", "k", "v", "slots", "tables", "ctx", "pairs")}
         if d["pairs"].shape[0]:
             pa.pa_copy_blocks([kp, vp], d["pairs"])
-        pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
         out = torch.empty_like(d["q"])
-        pa.pa_decode(out, d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws)
+        if fused:
+            if d["slots"].shape[0] > B:
+                pa.pa_reshape_and_cache(d["k"][B:], d["v"][B:], kp, vp, d["slots"][B:])
+            pa.pa_decode_append(out, d["q"], d["k"][:B], d["v"][:B], kp, vp, d["tables"], d["ctx"], wl.scale,
+                                max_ctx, P, ws)
+        else:
+            pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
+            pa.pa_decode(out, d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws)
         h["out"].copy_(out, non_blocking=True)
 
     for i in range(args.warmup):

@@ -121,6 +121,34 @@ PA_API pa_status pa_decode(void *out, const void *q, const void *k_pool, const v
                     int max_context_len, float scale, int dtype, int partition_size,
                     void *workspace, size_t workspace_bytes, pa_stream_t stream);
 
+/*
+ * Fused append + decode: for every sequence s with context_lens[s] >= 1,
+ * first writes k_new[s][h][:] and v_new[s][h][:] (all KV heads h) into the
+ * slot of position context_lens[s] - 1, i.e.
+ *   slot = block_tables[s][pos / block_size] * block_size + pos % block_size,
+ * then attends exactly as pa_decode. Same result, pool contents included, as
+ * pa_reshape_and_cache with those slots followed by pa_decode, in one pass:
+ * the attention unit that holds the last position writes the row and uses it
+ * directly, so the new row is neither written by a separate launch nor read
+ * back.
+ *
+ * Defined by: the m.nxbn.cn VLLM explainer, section 一 — each decode step
+ * computes only the new token's K/V, appends it to the cache and attends over
+ * the cache.
+ *
+ * k_new, v_new: [num_seqs][num_kv_heads][head_dim], fp16/bf16 like the pools,
+ * 16-byte aligned. context_lens are post-append lengths. The appended slot's
+ * block must be private to the sequence (a shared tail is copied first with
+ * pa_copy_blocks). Other arguments as pa_decode.
+ */
+PA_API pa_status pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                                  void *k_pool, void *v_pool, const int32_t *block_tables,
+                                  const int32_t *context_lens, int num_seqs, int num_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int num_blocks, int max_context_len,
+                                  float scale, int dtype, int partition_size, void *workspace,
+                                  size_t workspace_bytes, pa_stream_t stream);
+
 /* Workspace bytes pa_decode needs for these sizes (0 if the shape is invalid). */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
                                 int head_dim, int block_size, int max_context_len,

@@ -51,6 +51,9 @@ def lib() -> ctypes.CDLL:
         L.pa_decode.restype = _I
         L.pa_decode.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                                 _P, _SZ, _P]
+        L.pa_decode_append.restype = _I
+        L.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                                       _I, _P, _SZ, _P]
         L.pa_decode_workspace_size.restype = _SZ
         L.pa_decode_workspace_size.argtypes = [_I] * 7
         L.pa_decode_partition_size.restype = _I
@@ -150,6 +153,26 @@ def pa_decode(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_con
         B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
         int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+    return out
+
+
+def pa_decode_append(out, q, k_new, v_new, k_pool, v_pool, block_tables, context_lens, scale, max_context_len,
+                     partition_size=0, workspace=None, stream=None) -> torch.Tensor:
+    """Write k_new/v_new [B][Hkv][D] at each sequence's last position, then pa_decode."""
+    B, H, D = q.shape
+    NB, Hkv, bs, _ = k_pool.shape
+    if tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D):
+        raise ValueError("k_new and v_new must be [B][Hkv][D]")
+    if k_new.dtype != q.dtype or v_new.dtype != q.dtype or k_pool.dtype != q.dtype or v_pool.dtype != q.dtype:
+        raise ValueError("q, k_new, v_new and the pools must share one dtype")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device)
+    _check(lib().pa_decode_append(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_new, "k_new"), _cuda(v_new, "v_new"), _cuda(k_pool, "k_pool"),
+        _cuda(v_pool, "v_pool"), _cuda(block_tables, "block_tables", torch.int32),
+        _cuda(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, block_tables.shape[1], NB,
+        int(max_context_len), float(scale), _DTYPES[q.dtype], int(partition_size), _cuda(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
 
 

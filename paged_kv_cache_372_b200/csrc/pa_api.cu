@@ -119,10 +119,15 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
     return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts).total;
 }
 
-pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_pool, const int32_t *block_tables,
-                    const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                    int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
-                    int dtype, int partition_size, void *workspace, size_t workspace_bytes, pa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v_new, const void *k_pool,
+                      const void *v_pool, const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                      int num_blocks, int max_context_len, float scale, int dtype, int partition_size,
+                      void *workspace, size_t workspace_bytes, pa_stream_t stream) {
     g_last_error.clear();
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 || partition_size < 0)
         return fail(PA_ERR_INVALID, "negative or zero size argument");
@@ -150,11 +155,16 @@ pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_
     if (workspace_bytes < L.total)
         return fail(PA_ERR_INVALID, "workspace %zu bytes < %zu needed", workspace_bytes, L.total);
 
+    if ((k_new || v_new) && (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)))
+        return fail(PA_ERR_INVALID, "k_new/v_new null or misaligned");
+
     pa::DecodeParams p;
     p.out = out;
     p.q = q;
     p.k_pool = k_pool;
     p.v_pool = v_pool;
+    p.k_new = k_new;
+    p.v_new = v_new;
     p.block_tables = block_tables;
     p.context_lens = context_lens;
     p.num_seqs = num_seqs;
@@ -182,6 +192,33 @@ pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_
         return dtype == PA_F16 ? dispatch_group<128, __half>(p, group, s)
                                : dispatch_group<128, __nv_bfloat16>(p, group, s);
     return dtype == PA_F16 ? dispatch_group<64, __half>(p, group, s) : dispatch_group<64, __nv_bfloat16>(p, group, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_pool, const int32_t *block_tables,
+                    const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                    int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                    int dtype, int partition_size, void *workspace, size_t workspace_bytes, pa_stream_t stream) {
+    return decode_impl(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new, void *k_pool,
+                           void *v_pool, const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                           int num_blocks, int max_context_len, float scale, int dtype, int partition_size,
+                           void *workspace, size_t workspace_bytes, pa_stream_t stream) {
+    if (num_seqs > 0 && (!k_new || !v_new)) {
+        g_last_error = "k_new/v_new null";
+        return PA_ERR_INVALID;
+    }
+    return decode_impl(out, q, k_new, v_new, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void *v_pool, const int64_t *slot_mapping,

@@ -36,6 +36,8 @@ struct DecodeParams {
     const void *q;
     const void *k_pool;
     const void *v_pool;
+    const void *k_new;  // [num_seqs][num_kv_heads][head_dim] rows appended at each
+    const void *v_new;  // sequence's last position first; null for plain decode
     const int32_t *block_tables;
     const int32_t *context_lens;
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks;
@@ -156,6 +158,33 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
             uint4 *row = static_cast<uint4 *>(p.out) + (size_t)s * nvec;
             for (int i = 0; i < nvec; ++i) row[i] = make_uint4(0, 0, 0, 0);
         }
+    }
+}
+
+// ---- append (used with the CUDA-core kernel) ---------------------------------
+// Writes k_new/v_new[s][h] into the slot of sequence s's last position
+// (context_len - 1): slot = table[s][pos / bs] * bs + pos % bs. One thread per
+// 16-byte vector of K and the matching vector of V.
+__global__ void __launch_bounds__(256) pa_append_kernel(const DecodeParams p) {
+    const int vpr = p.head_dim / 8;
+    const long long total = (long long)p.num_seqs * p.num_kv_heads * vpr;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const long long row = i / vpr;
+        const int vec = (int)(i - row * vpr);
+        const int s = (int)(row / p.num_kv_heads);
+        const int h = (int)(row - (long long)s * p.num_kv_heads);
+        const int ctx = clamped_context(p, s, false);
+        if (ctx == 0) continue;
+        const int pos = ctx - 1;
+        const int pb = p.block_tables[(size_t)s * p.max_blocks_per_seq + pos / p.block_size];
+        if ((unsigned)pb >= (unsigned)p.num_blocks) {
+            raise_error(PA_DEVERR_BLOCK_ID);
+            continue;
+        }
+        const size_t dst = (((size_t)pb * p.num_kv_heads + h) * p.block_size + pos % p.block_size) * vpr + vec;
+        static_cast<uint4 *>(const_cast<void *>(p.k_pool))[dst] = static_cast<const uint4 *>(p.k_new)[i];
+        static_cast<uint4 *>(const_cast<void *>(p.v_pool))[dst] = static_cast<const uint4 *>(p.v_new)[i];
     }
 }
 

@@ -302,6 +302,10 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     // Heads this lane's accumulator columns belong to, and whether they exist.
     const int h0 = 2 * t4, h1 = 2 * t4 + 1;
     const bool hv0 = h0 < G, hv1 = h1 < G;
+    // Fused append: the unit that holds a sequence's last token writes the new
+    // K/V row into the pool and uses it in place of the tile's old contents.
+    constexpr int NVR = D / 8;  // 16-byte vectors per row
+    const bool append = p.k_new != nullptr;
 
     for (;;) {
         uint32_t qb[Gm::KS][2];  // B fragments of Q^T: query head g8, 2 columns
@@ -311,6 +315,15 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
         for (int i = 0; i < Gm::KS; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+        // Lanes [0, NVR) hold one 16-byte vector of the new K row, lanes
+        // [NVR, 2*NVR) of the new V row; loaded now, used at the last tile.
+        const bool app_unit = append && cur.part == cur.nparts - 1;
+        uint4 newrow = make_uint4(0, 0, 0, 0);
+        if (app_unit && lane < 2 * NVR) {
+            const size_t rowoff = ((size_t)cur.s * Hkv + cur.kvh) * D;
+            const T *src = static_cast<const T *>(lane < NVR ? p.k_new : p.v_new);
+            newrow = *reinterpret_cast<const uint4 *>(src + rowoff + (lane % NVR) * 8);
+        }
 
         for (int k = 0; k < cur.ntiles; ++k) {
             if (!wait_item()) return;
@@ -327,6 +340,24 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 }
             }
             const int valid = min(16, cur.ntok - 16 * k);
+            if (app_unit && k == cur.ntiles - 1) {
+                const int tok = cur.ntok - 1;  // the sequence's last position, in this tile
+                const int pb = __shfl_sync(FULL_MASK, cur.tbl, tok / bs);
+                if (lane < 2 * NVR) {
+                    const int half = lane / NVR, c = lane % NVR;
+                    uint8_t *st = ring + stage * Gm::STAGE_BYTES + half * Gm::HALF_BYTES;
+                    *reinterpret_cast<uint4 *>(st + swz(tok & 15, c)) = newrow;
+                    if ((unsigned)pb < (unsigned)p.num_blocks) {
+                        T *pool = static_cast<T *>(const_cast<void *>(half ? p.v_pool : p.k_pool));
+                        *reinterpret_cast<uint4 *>(pool + (((size_t)pb * Hkv + cur.kvh) * bs + tok % bs) * D + c * 8) =
+                            newrow;
+                    } else if (lane == 0) {
+                        raise_error(PA_DEVERR_BLOCK_ID);
+                    }
+                }
+                fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
+                __syncwarp();
+            }
 
             // ---------------- S^T = K . Q^T ------------------------------------
             float s[4] = {0.f, 0.f, 0.f, 0.f};

@@ -56,6 +56,13 @@ pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
+    if (p.k_new) {
+        // The CUDA-core kernel has no fused append: write the new rows first.
+        const long long total = (long long)p.num_seqs * p.num_kv_heads * (D / 8);
+        long long blocks = (total + 255) / 256;
+        if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
+        pa::pa_append_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
+    }
     pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
     // Programmatic dependent launch: the attention CTAs start their set-up
     // while the plan kernel runs and wait for its results in-kernel.

@@ -58,3 +58,28 @@ def max_err(gpu_out: torch.Tensor, ref: np.ndarray) -> float:
 def pools_equal(kp_gpu, vp_gpu, kp_ref, vp_ref) -> bool:
     return (np.array_equal(bits_of(kp_gpu.cpu()), kp_ref)
             and np.array_equal(bits_of(vp_gpu.cpu()), vp_ref))
+
+
+def gpu_step_fused(wl, step, kp, vp, partition_size=None, workspace=None):
+    """The same step with the fused append + decode entry point: copies, then
+    any extra (prefill) tokens through pa_reshape_and_cache, then
+    pa_decode_append for each sequence's new token."""
+    st = wl.steps[step]
+    dev = kp.device
+    B = st.q.shape[0]
+    bs = wl.block_size
+    for s in range(B):  # the workloads append each sequence's token at its last position
+        n = int(st.context_lens[s])
+        assert st.slot_mapping[s] == st.block_tables[s, (n - 1) // bs] * bs + (n - 1) % bs
+    if len(st.copy_pairs):
+        pa.pa_copy_blocks([kp, vp], torch.from_numpy(st.copy_pairs).to(dev))
+    if len(st.slot_mapping) > B:
+        pa.pa_reshape_and_cache(st.k_new[B:].to(dev), st.v_new[B:].to(dev), kp, vp,
+                                torch.from_numpy(st.slot_mapping[B:]).to(dev))
+    q = st.q.to(dev)
+    out = torch.empty_like(q)
+    P = wl.partition_size if partition_size is None else partition_size
+    pa.pa_decode_append(out, q, st.k_new[:B].contiguous().to(dev), st.v_new[:B].contiguous().to(dev), kp, vp,
+                        torch.from_numpy(st.block_tables).to(dev), torch.from_numpy(st.context_lens).to(dev),
+                        wl.scale, int(st.context_lens.max()), P, workspace)
+    return out

@@ -97,3 +97,25 @@ def test_shapes(shape, block_size):
                                 inputs.normal((nb, hkv, block_size, D), dtype, gen), [st])
         for P in (0, block_size * max(1, 64 // block_size)):
             run_and_compare(wl, partition_size=P)
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("llama7b", {"num_seqs": 8}), ("llama3_8b", {"num_seqs": 16}),
+                                     ("beam", {"groups": 2, "steps": 4}),
+                                     ("long32k", {"num_seqs": 2, "ctx_len": 3000, "prefill_tokens": 64})])
+def test_fused_append_matches_oracle_and_unfused_path(name, kw):
+    """pa_decode_append = cache write of the last positions + pa_decode: same
+    pools bit for bit, same outputs bit for bit, oracle within tolerance."""
+    wl = workloads.build(name, 21, **kw)
+    kf, vf = H.to_gpu(wl)                 # fused path state
+    ku, vu = H.to_gpu(wl)                 # unfused path state
+    okp, ovp = H.oracle_state(wl)
+    for i in range(len(wl.steps)):
+        fused = H.gpu_step_fused(wl, i, kf, vf)
+        unfused = H.gpu_step(wl, i, ku, vu)
+        ref = H.oracle_step(wl, i, okp, ovp)
+        torch.cuda.synchronize()
+        assert pa.pa_device_errors() == 0
+        assert torch.equal(kf, ku) and torch.equal(vf, vu), f"pools differ at step {i}"
+        assert H.pools_equal(kf, vf, okp, ovp)
+        assert torch.equal(fused, unfused), f"outputs differ at step {i}"
+        assert H.max_err(fused, ref) <= H.TOL[wl.dtype]
