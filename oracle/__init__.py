@@ -73,6 +73,8 @@ class Oracle:
         L.oracle_reshape_and_cache.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I]
         L.oracle_copy_blocks.restype = None
         L.oracle_copy_blocks.argtypes = [_P, _I, _P, _I, ctypes.c_size_t]
+        L.oracle_swap_blocks.restype = None
+        L.oracle_swap_blocks.argtypes = [_P, _P, _I, _P, _I, ctypes.c_size_t]
         L.oracle_slot_mapping.restype = None
         L.oracle_slot_mapping.argtypes = [_P, _P, _I, _P, _P, _I, _I]
 
@@ -140,6 +142,20 @@ class Oracle:
         self.lib.oracle_copy_blocks(arr, len(pools), _ptr(pairs), pairs.shape[0],
                                     int(block_bytes))
 
+    def swap_blocks(self, dst_pools, src_pools, src_dst_pairs, block_bytes: int) -> None:
+        """In place on each dst pool: dst_pools[i][dst] = src_pools[i][src] per pair."""
+        pairs = np.ascontiguousarray(src_dst_pairs, dtype=np.int64).reshape(-1, 2)
+        assert len(dst_pools) == len(src_pools)
+        for d, s_ in zip(dst_pools, src_pools):
+            assert d.flags.c_contiguous and s_.flags.c_contiguous
+            if pairs.size:
+                assert pairs[:, 0].min() >= 0 and pairs[:, 0].max() < s_.nbytes // block_bytes
+                assert pairs[:, 1].min() >= 0 and pairs[:, 1].max() < d.nbytes // block_bytes
+        n = max(1, len(dst_pools))
+        darr = (ctypes.c_void_p * n)(*[a.ctypes.data for a in dst_pools])
+        sarr = (ctypes.c_void_p * n)(*[a.ctypes.data for a in src_pools])
+        self.lib.oracle_swap_blocks(darr, sarr, len(dst_pools), _ptr(pairs), pairs.shape[0], int(block_bytes))
+
     def slot_mapping(self, block_tables, seq_ids, positions, block_size: int) -> np.ndarray:
         block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
         seq_ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
@@ -176,6 +192,10 @@ def copy_blocks(*args, **kwargs):
 
 def slot_mapping(*args, **kwargs):
     return get().slot_mapping(*args, **kwargs)
+
+
+def swap_blocks(*args, **kwargs):
+    return get().swap_blocks(*args, **kwargs)
 
 
 def to_double(*args, **kwargs):

@@ -216,6 +216,25 @@ void oracle_copy_blocks(uint8_t *const *pools, int num_pools,
 }
 
 /*
+ * Swap copies between two sets of pools (e.g. GPU blocks out to a host pool
+ * and back), as in "vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理",
+ * section 抢占与恢复 (swapping a preempted request's blocks to CPU memory over
+ * PCIe and back): for each (src, dst) pair in order and each pool index i,
+ * block dst of dst_pools[i] becomes a byte copy of block src of src_pools[i].
+ */
+void oracle_swap_blocks(uint8_t *const *dst_pools, const uint8_t *const *src_pools, int num_pools,
+                        const int64_t *src_dst_pairs, int num_pairs, size_t block_bytes)
+{
+    for (int p = 0; p < num_pairs; p++) {
+        const int64_t src = src_dst_pairs[2 * p];
+        const int64_t dst = src_dst_pairs[2 * p + 1];
+        for (int i = 0; i < num_pools; i++)
+            memcpy(dst_pools[i] + (size_t)dst * block_bytes,
+                   src_pools[i] + (size_t)src * block_bytes, block_bytes);
+    }
+}
+
+/*
  * Slot of token position pos of a sequence: the page table maps logical page
  * pos / block_size to a physical page; the slot is that page's first slot plus
  * the offset inside the page.

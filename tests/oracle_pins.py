@@ -253,6 +253,25 @@ def pin_copy_blocks(orc, seed=9):
         assert np.array_equal(p, w)
 
 
+def pin_swap_blocks(orc, seed=11):
+    """Cross-pool block copies vs numpy slice assignment; the source is untouched."""
+    rng = np.random.default_rng(seed)
+    src = [rng.integers(0, 256, (9, 2, 4, 8), dtype=np.uint8) for _ in range(2)]
+    dst = [rng.integers(0, 256, (5, 2, 4, 8), dtype=np.uint8) for _ in range(2)]
+    bb = 2 * 4 * 8
+    pairs = np.array([[7, 0], [2, 4], [8, 1]], dtype=np.int64)
+    want = [d.copy() for d in dst]
+    before = [x.copy() for x in src]
+    for w, x in zip(want, src):
+        for a, b in pairs:
+            w[b] = x[a]
+    orc.swap_blocks(dst, src, pairs, bb)
+    for d, w in zip(dst, want):
+        assert np.array_equal(d, w)
+    for x, b in zip(src, before):
+        assert np.array_equal(x, b)
+
+
 def pin_slot_mapping(orc, seed=10):
     rng = np.random.default_rng(seed)
     bs, B, W = 16, 5, 6
@@ -271,4 +290,4 @@ def pin_slot_mapping(orc, seed=10):
 ALL_PINS = [pin_decode_f16, pin_decode_bf16, pin_bruteforce, pin_sdpa, pin_single_token,
             pin_equal_keys, pin_two_token_closed_form, pin_block_permutation,
             pin_shared_equals_duplicated, pin_tail_slots_ignored, pin_gqa_mapping,
-            pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_slot_mapping]
+            pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_swap_blocks, pin_slot_mapping]

@@ -39,6 +39,8 @@ MUTATIONS = {
                            "const size_t src = ((size_t)t * num_kv_heads + (num_kv_heads - 1 - h)) * head_dim;"),
     "copy_direction": ("const int64_t src = src_dst_pairs[2 * p];\n        const int64_t dst = src_dst_pairs[2 * p + 1];",
                        "const int64_t src = src_dst_pairs[2 * p + 1];\n        const int64_t dst = src_dst_pairs[2 * p];"),
+    "swap_pool_index": ("memcpy(dst_pools[i] + (size_t)dst * block_bytes,\n                   src_pools[i] + (size_t)src * block_bytes, block_bytes);",
+                        "memcpy(dst_pools[i] + (size_t)dst * block_bytes,\n                   src_pools[num_pools - 1 - i] + (size_t)src * block_bytes, block_bytes);"),
     "slot_offset": ("slots[i] = (int64_t)table[pos / block_size] * block_size + pos % block_size;",
                     "slots[i] = (int64_t)table[pos / block_size] * block_size + (pos + 1) % block_size;"),
 }
