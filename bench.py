@@ -1,7 +1,7 @@
 """Benchmark of the paged decode hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload llama7b|llama3_8b|beam|long32k|tiny] [--seed S]
+                    [--workload llama7b|llama3_8b|beam|long32k|tiny|swap] [--seed S]
 
 One step is the whole hot path once over one batch: copy-on-write block
 copies (when the workload has any), the cache write of the step's new tokens,
@@ -15,7 +15,8 @@ Under torchrun every rank runs its own replica of the workload on its own GPU
 with the max-over-ranks device time.
 
 --impl reference times the fp64 CPU oracle on the host cores over a bounded
-sample of the same workload (rank 0 only).
+sample of the same workload (rank 0 only). --workload swap measures
+pa_swap_blocks between the GPU pools and page-locked host memory instead.
 """
 from __future__ import annotations
 
@@ -410,6 +411,63 @@ def cpu_baseline(wl, budget_s=10.0, n_seqs=None):
                       f"{reps} repetitions, {dt:.3f} s each"}
 
 
+def run_swap(args, world, rank, local):
+    """pa_swap_blocks between the GPU pools and a page-locked host pool: a
+    shuffled set of whole blocks out and back, against one contiguous
+    cudaMemcpyAsync of the same bytes over the same link (the roofline)."""
+    import paged_kv_cache_372_b200 as pa
+    from paged_kv_cache_372_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    nb, hkv, bs, d = 8192, 8, 16, 128                      # llama3_8b-shaped blocks, 32 KiB per pool
+    gen = inputs.generator(args.seed + 7000)
+    kp = inputs.normal((nb, hkv, bs, d), "bf16", gen).to(dev)
+    vp = inputs.normal((nb, hkv, bs, d), "bf16", gen).to(dev)
+    hk = torch.empty((nb, hkv, bs, d), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    n = nb // 2                                           # half the pool moves each way
+    src = torch.tensor(inputs.choice(nb, n, gen), dtype=torch.int64)
+    dst = torch.tensor(inputs.choice(nb, n, gen), dtype=torch.int64)
+    out_pairs = torch.stack([src, dst], 1).to(dev)
+    in_pairs = torch.stack([dst, src], 1).to(dev)
+    moved = 2 * n * kp[0].numel() * 2
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / args.steps
+
+    ms_out = timed(lambda: pa.pa_swap_blocks([hk, hv], [kp, vp], out_pairs))
+    ms_in = timed(lambda: pa.pa_swap_blocks([kp, vp], [hk, hv], in_pairs))
+    assert pa.pa_device_errors() == 0
+    flat_d = torch.empty(moved, dtype=torch.uint8, device=dev)
+    flat_h = torch.empty(moved, dtype=torch.uint8).pin_memory()
+    ms_d2h = timed(lambda: flat_h.copy_(flat_d, non_blocking=True))
+    ms_h2d = timed(lambda: flat_d.copy_(flat_h, non_blocking=True))
+    gbs = lambda ms: moved / (ms * 1e-3) / 1e9
+    value = 2 * moved / ((ms_out + ms_in) * 1e-3) / 1e9
+    link = 2 * moved / ((ms_d2h + ms_h2d) * 1e-3) / 1e9
+    return {"metric": "block swap GPU<->page-locked host (pa_swap_blocks), GB/s", "value": value, "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_out + ms_in,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": "swap", "blocks_each_way": n, "block_bytes_per_pool":
+                                            kp[0].numel() * 2, "pools": 2, "bytes_each_way": moved},
+            "swap_out_gbs": gbs(ms_out), "swap_in_gbs": gbs(ms_in),
+            "roofline": {"bound": "host link", "achieved": value, "peak": link, "unit": "GB/s",
+                         "frac": value / link,
+                         "peak_source": "measured: one contiguous cudaMemcpyAsync of the same bytes each way",
+                         "memcpy_d2h_gbs": gbs(ms_d2h), "memcpy_h2d_gbs": gbs(ms_h2d)},
+            "gpu_launches": 2 * args.steps}
+
+
 def run_reference(args, world, rank):
     """The oracle, as it stands, on the host cores: each step is a bounded sample
     (8 sequences) of the same workload."""
@@ -450,7 +508,7 @@ def main():
             if rank == 0:
                 print(json.dumps(run_reference(args, world, rank)), flush=True)
             return
-        res = run_ours(args, world, rank, local)
+        res = run_swap(args, world, rank, local) if args.workload == "swap" else run_ours(args, world, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -197,6 +197,30 @@ PA_API pa_status pa_copy_blocks(void *const *pools, int num_pools, const int64_t
                          pa_stream_t stream);
 
 /*
+ * Swap copies of whole blocks between two sets of pools: for each pair p and
+ * each pool index i, block dst of dst_pools[i] becomes a byte copy of block
+ * src of src_pools[i] (block = block_bytes bytes). Used to move a preempted
+ * sequence's blocks from the GPU pools to host pools and back.
+ *
+ * Defined by: "vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理", section
+ * 抢占与恢复 — preemption by swapping moves a request's KV blocks over PCIe to
+ * CPU memory and back when it resumes.
+ *
+ * dst_pools, src_pools: HOST arrays of num_pools pointers, each to device
+ * memory or to page-locked host memory (cudaHostAlloc / cudaMallocHost /
+ * cudaHostRegister), 16-byte aligned; pageable host memory is rejected with
+ * PA_ERR_INVALID. src_dst_pairs: [num_pairs][2] int64 in device or page-locked
+ * host memory. Source ids must be < num_src_blocks and destination ids <
+ * num_dst_blocks (others are skipped and flagged PA_DEVERR_PAIR). block_bytes
+ * is a multiple of 16. Destinations must be distinct; the two sides must not
+ * overlap. Asynchronous on `stream`; host memory must stay valid until the
+ * copy has finished.
+ */
+PA_API pa_status pa_swap_blocks(void *const *dst_pools, const void *const *src_pools, int num_pools,
+                                const int64_t *src_dst_pairs, int num_pairs, size_t block_bytes,
+                                int num_src_blocks, int num_dst_blocks, pa_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns the current device's error word in
  * *flags (PA_DEVERR_* bits) and clears it when `clear` is non-zero. Returns
  * PA_ERR_DEVICE_CHECK when any bit was set, PA_OK otherwise.

@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.pa_reshape_and_cache.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
         L.pa_copy_blocks.restype = _I
         L.pa_copy_blocks.argtypes = [ctypes.POINTER(_P), _I, _P, _I, _SZ, _I, _P]
+        L.pa_swap_blocks.restype = _I
+        L.pa_swap_blocks.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_P), _I, _P, _I, _SZ, _I, _I, _P]
         L.pa_device_errors.restype = _I
         L.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint), _I, _P]
         L.pa_num_sms.restype = _I
@@ -208,6 +210,38 @@ def pa_copy_blocks(pools, src_dst_pairs, stream=None) -> None:
     ptrs = (_P * len(pools))(*[_cuda(t, "pool") for t in pools])
     _check(lib().pa_copy_blocks(ptrs, len(pools), _cuda(pairs, "src_dst_pairs", torch.int64),
                                 pairs.shape[0], block_bytes, nb, _stream(stream)))
+
+
+def pa_swap_blocks(dst_pools, src_pools, src_dst_pairs, stream=None) -> None:
+    """dst_pools[i][dst] = src_pools[i][src] for each (src, dst) row of src_dst_pairs.
+
+    Pools are CUDA tensors or page-locked CPU tensors (``pin_memory()``) with the
+    same block size; src_dst_pairs is an int64 [P][2] CUDA or page-locked tensor.
+    """
+    dst_pools, src_pools = list(dst_pools), list(src_pools)
+    if len(dst_pools) != len(src_pools):
+        raise ValueError("dst_pools and src_pools differ in length")
+    if not dst_pools:
+        return
+    block_bytes = dst_pools[0][0].numel() * dst_pools[0].element_size()
+
+    def ptr(t, name):
+        if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous tensor")
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError(f"{name} must be a CUDA tensor or page-locked (pin_memory) CPU tensor")
+        return t.data_ptr()
+
+    for t in dst_pools + src_pools:
+        if t[0].numel() * t.element_size() != block_bytes:
+            raise ValueError("all pools must have the same block size")
+    pairs = src_dst_pairs
+    if pairs.dim() != 2 or pairs.shape[1] != 2 or pairs.dtype != torch.int64:
+        raise ValueError("src_dst_pairs must be int64 [P][2]")
+    dp = (_P * len(dst_pools))(*[ptr(t, "dst pool") for t in dst_pools])
+    sp = (_P * len(src_pools))(*[ptr(t, "src pool") for t in src_pools])
+    _check(lib().pa_swap_blocks(dp, sp, len(dst_pools), ptr(pairs, "src_dst_pairs"), pairs.shape[0],
+                                block_bytes, src_pools[0].shape[0], dst_pools[0].shape[0], _stream(stream)))
 
 
 def pa_device_errors(clear: bool = True, stream=None) -> int:

@@ -15,6 +15,9 @@ Behaviour, cited by page and section:
     whose reference count is above one is copied (new block, copy, table
     update) before a sequence appends into it; the last holder writes in place.
   * slot = block_table[pos // block_size] * block_size + pos % block_size.
+  * "vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理", section 抢占与恢复:
+    a preempted sequence's blocks can be swapped out to CPU memory and back;
+    ``swap_out`` / ``swap_in`` plan those copies against a host block pool.
 """
 from __future__ import annotations
 
@@ -135,3 +138,44 @@ class BlockManager:
                 count[b] += 1
         assert count == self.ref, "reference counts disagree with the tables"
         assert sorted(self.free) == [b for b in range(self.num_blocks) if count[b] == 0]
+
+
+@dataclass
+class HostPool:
+    """Free list of a page-locked host pool holding swapped-out blocks."""
+    num_blocks: int
+    free: list[int] = field(init=False)
+    tables: dict[int, list[int]] = field(init=False, default_factory=dict)
+    lens: dict[int, int] = field(init=False, default_factory=dict)
+
+    def __post_init__(self):
+        self.free = list(range(self.num_blocks))
+
+
+def swap_out(bm: BlockManager, host: HostPool, seq: int) -> list[tuple[int, int]]:
+    """Move sequence `seq` to the host pool: returns (gpu block, host block) copy
+    pairs and releases the GPU blocks (a shared block stays with its other holders)."""
+    table = bm.tables[seq]
+    if len(table) > len(host.free):
+        raise OutOfBlocks("no free blocks in the host pool")
+    pairs = [(g, host.free.pop()) for g in table]
+    host.tables[seq] = [c for _, c in pairs]
+    host.lens[seq] = bm.lens[seq]
+    bm.free_seq(seq)
+    return pairs
+
+
+def swap_in(bm: BlockManager, host: HostPool, seq: int) -> list[tuple[int, int]]:
+    """Bring sequence `seq` back into fresh GPU blocks: returns (host block, gpu
+    block) copy pairs and releases the host blocks."""
+    cpu = host.tables[seq]
+    if len(cpu) > len(bm.free):
+        raise OutOfBlocks("no free blocks in the pool")
+    if seq in bm.tables:
+        raise KeyError(f"sequence {seq} is resident")
+    del host.tables[seq]
+    gpu = [bm._pop() for _ in cpu]
+    bm.tables[seq] = gpu
+    bm.lens[seq] = host.lens.pop(seq)
+    host.free.extend(reversed(cpu))
+    return list(zip(cpu, gpu))

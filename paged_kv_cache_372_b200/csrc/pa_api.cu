@@ -277,6 +277,79 @@ pa_status pa_copy_blocks(void *const *pools, int num_pools, const int64_t *src_d
     return PA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Device-usable address of `p`: device memory as is, page-locked host memory
+// through its mapped device pointer; anything else (pageable host memory,
+// unknown pointers) is rejected so that no kernel touches an unmapped address.
+pa_status device_address(const void *p, const void **out, const char *what) {
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(PA_ERR_INVALID, "%s: not a CUDA-visible pointer", what);
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+        *out = p;
+        return PA_OK;
+    }
+    if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+        *out = a.devicePointer;
+        return PA_OK;
+    }
+    return fail(PA_ERR_INVALID, "%s: pageable host memory (use page-locked memory)", what);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_swap_blocks(void *const *dst_pools, const void *const *src_pools, int num_pools,
+                         const int64_t *src_dst_pairs, int num_pairs, size_t block_bytes, int num_src_blocks,
+                         int num_dst_blocks, pa_stream_t stream) {
+    g_last_error.clear();
+    if (num_pools < 0 || num_pairs < 0 || num_src_blocks <= 0 || num_dst_blocks <= 0)
+        return fail(PA_ERR_INVALID, "size argument");
+    if (num_pairs == 0 || num_pools == 0) return PA_OK;
+    if (num_pairs > 2147483647 / 2) return fail(PA_ERR_UNSUPPORTED, "too many pairs");
+    if (!dst_pools || !src_pools || !src_dst_pairs) return fail(PA_ERR_INVALID, "null pointer");
+    if (block_bytes == 0 || block_bytes % 16)
+        return fail(PA_ERR_INVALID, "block_bytes %zu not a multiple of 16", block_bytes);
+    if (!aligned(src_dst_pairs, 8)) return fail(PA_ERR_INVALID, "misaligned pairs");
+    const void *pairs = nullptr;
+    pa_status st = device_address(src_dst_pairs, &pairs, "src_dst_pairs");
+    if (st != PA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int first = 0; first < num_pools; first += pa::COPY_MAX_POOLS) {
+        const int n = num_pools - first < pa::COPY_MAX_POOLS ? num_pools - first : pa::COPY_MAX_POOLS;
+        pa::PoolList dst;
+        pa::ConstPoolList src;
+        for (int i = 0; i < pa::COPY_MAX_POOLS; ++i) {
+            dst.ptr[i] = nullptr;
+            src.ptr[i] = nullptr;
+        }
+        for (int i = 0; i < n; ++i) {
+            if (!dst_pools[first + i] || !src_pools[first + i] || !aligned(dst_pools[first + i], 16) ||
+                !aligned(src_pools[first + i], 16))
+                return fail(PA_ERR_INVALID, "pool %d null or misaligned", first + i);
+            const void *d = nullptr, *sp = nullptr;
+            if ((st = device_address(dst_pools[first + i], &d, "dst pool")) != PA_OK) return st;
+            if ((st = device_address(src_pools[first + i], &sp, "src pool")) != PA_OK) return st;
+            dst.ptr[i] = static_cast<uint4 *>(const_cast<void *>(d));
+            src.ptr[i] = static_cast<const uint4 *>(sp);
+        }
+        const dim3 grid((unsigned)num_pairs, (unsigned)n);
+        pa::pa_swap_blocks_kernel<<<grid, 256, 0, s>>>(dst, src, static_cast<const int64_t *>(pairs),
+                                                       (long long)(block_bytes / 16), (long long)num_src_blocks,
+                                                       (long long)num_dst_blocks);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pa_swap_blocks launch");
+    return PA_OK;
+}
+
 pa_status pa_device_errors(unsigned int *flags, int clear, pa_stream_t stream) {
     g_last_error.clear();
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -72,4 +72,35 @@ __global__ void __launch_bounds__(256) pa_copy_blocks_kernel(PoolList pools, con
     for (; i < vec_per_block; i += 256) to[i] = from[i];
 }
 
+// Cross-pool block copies for swapping: blockIdx.x = pair, blockIdx.y = pool
+// index; the CTA copies block src of src[pool] to block dst of dst[pool].
+// Either side may be page-locked host memory reached through unified
+// addressing, so each thread keeps four 16-byte loads in flight.
+struct ConstPoolList {
+    const uint4 *ptr[COPY_MAX_POOLS];
+};
+
+__global__ void __launch_bounds__(256) pa_swap_blocks_kernel(PoolList dst, ConstPoolList src,
+                                                             const int64_t *__restrict__ pairs,
+                                                             long long vec_per_block, long long num_src_blocks,
+                                                             long long num_dst_blocks) {
+    const int64_t s = pairs[2 * (size_t)blockIdx.x];
+    const int64_t d = pairs[2 * (size_t)blockIdx.x + 1];
+    if (s < 0 || s >= num_src_blocks || d < 0 || d >= num_dst_blocks) {
+        if (threadIdx.x == 0) raise_error(PA_DEVERR_PAIR);
+        return;
+    }
+    const uint4 *from = src.ptr[blockIdx.y] + (size_t)s * vec_per_block;
+    uint4 *to = dst.ptr[blockIdx.y] + (size_t)d * vec_per_block;
+    long long i = threadIdx.x;
+    for (; i + 3 * 256 < vec_per_block; i += 4 * 256) {
+        const uint4 a = from[i], b = from[i + 256], c = from[i + 512], e = from[i + 768];
+        to[i] = a;
+        to[i + 256] = b;
+        to[i + 512] = c;
+        to[i + 768] = e;
+    }
+    for (; i < vec_per_block; i += 256) to[i] = from[i];
+}
+
 }  // namespace pa

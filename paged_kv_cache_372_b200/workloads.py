@@ -23,6 +23,8 @@ Workloads (sizes as named):
              uniform in [16, 512]; H=32, Hkv=8, D=128, bs=16, bf16; each step
              keeps 2 parents per group and forks each into 4 beams, so appends
              into a shared partly-filled tail block copy it first.
+  beam256    the other reading of beam: all 8 sequences of a group fork 4 ways
+             (256 sequences per step; 8 of a group's 32 beams are kept later).
   long32k    8 seqs at ctx 32768, H=32, Hkv=8, D=128, bs=64, bf16, 512-token
              split-context partitions; the same step also writes 4096 prefill
              tokens into distinct random free slots.
@@ -38,7 +40,7 @@ import torch
 from . import inputs
 from .block_manager import BlockManager
 
-NAMES = ("tiny", "llama7b", "llama3_8b", "beam", "long32k")
+NAMES = ("tiny", "llama7b", "llama3_8b", "beam", "beam256", "long32k")
 
 
 @dataclass
@@ -191,31 +193,34 @@ def long32k(seed: int = 0, num_seqs: int = 8, ctx_len: int = 32768,
 
 
 def beam(seed: int = 0, groups: int = 8, width: int = 8, prefix: int = 1024,
-         steps: int = 8, parents: int = 2) -> Workload:
-    """Shared prefix + beam fork. Per step and group: keep `parents` beams, fork each
-    into width // parents children, free the rest, and append one token per child."""
+         steps: int = 8, parents: int = 2, initial: int | None = None, name: str = "beam") -> Workload:
+    """Shared prefix + beam fork. A group starts with `initial` sequences (default
+    `width`) sharing the prefix, each with its own suffix. Per step and group:
+    keep `parents` beams, fork each into width // parents children, free the
+    rest, and append one token per child."""
     gen = inputs.generator(seed + 4000)
     bs, hkv, heads, d, dtype = 16, 8, 32, 128, "bf16"
-    suffix = inputs.uniform_int(16, 512, groups * width, gen)
+    start = width if initial is None else initial
+    suffix = inputs.uniform_int(16, 512, groups * start, gen)
     need = groups * (prefix // bs) + sum(-(-x // bs) + 1 for x in suffix)
-    nb = int(math.ceil(1.25 * need)) + steps * groups * width
+    nb = int(math.ceil(1.25 * need)) + steps * groups * width * 2
     bm = BlockManager(nb, bs, inputs.permutation(nb, gen))
     live = []
     for g in range(groups):
-        root = g * width
+        root = g * start
         bm.allocate(root, prefix)
-        for j in range(1, width):
+        for j in range(1, start):
             bm.fork(root, root + j)
-        for j in range(width):
+        for j in range(start):
             for _ in range(suffix[root + j]):
                 bm.append_slot(root + j)
-        live.append([root + j for j in range(width)])
-    next_id = groups * width
+        live.append([root + j for j in range(start)])
+    next_id = groups * start
     plans = []
     for _ in range(steps):
         pairs, slots, order = [], [], []
         for g in range(groups):
-            keep = [live[g][i] for i in inputs.choice(width, parents, gen)]
+            keep = [live[g][i] for i in inputs.choice(len(live[g]), parents, gen)]
             children = []
             for p in keep:
                 for _ in range(width // parents):
@@ -235,7 +240,7 @@ def beam(seed: int = 0, groups: int = 8, width: int = 8, prefix: int = 1024,
         plans.append((order, pairs, slots, {s: list(bm.tables[s]) for s in order},
                       bm.context_lens(order)))
     width_blocks = max(len(t) for _, _, _, tabs, _ in plans for t in tabs.values())
-    wl = Workload("beam", dtype, heads, hkv, d, bs, nb, 0,
+    wl = Workload(name, dtype, heads, hkv, d, bs, nb, 0,
                   _pool(nb, hkv, bs, d, dtype, gen), _pool(nb, hkv, bs, d, dtype, gen))
     for order, pairs, slots, tabs, lens in plans:
         bt = np.full((len(order), width_blocks), -1, dtype=np.int32)
@@ -253,6 +258,13 @@ def beam(seed: int = 0, groups: int = 8, width: int = 8, prefix: int = 1024,
     return wl
 
 
+def beam256(seed: int = 0, steps: int = 8, groups: int = 8) -> Workload:
+    """The other reading of the beam workload: every one of a group's 8
+    sequences forks 4 ways (32 per group, 256 in all); later steps keep 8 of a
+    group's 32 beams and fork each 4 ways again."""
+    return beam(seed, groups=groups, width=32, prefix=1024, steps=steps, parents=8, initial=8, name="beam256")
+
+
 def build(name: str, seed: int = 0, **kw) -> Workload:
-    return {"tiny": tiny, "llama7b": llama7b, "llama3_8b": llama3_8b, "beam": beam,
+    return {"tiny": tiny, "llama7b": llama7b, "llama3_8b": llama3_8b, "beam": beam, "beam256": beam256,
             "long32k": long32k}[name](seed, **kw)

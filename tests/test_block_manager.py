@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 from paged_kv_cache_372_b200 import workloads
-from paged_kv_cache_372_b200.block_manager import BlockManager, OutOfBlocks
+from paged_kv_cache_372_b200.block_manager import BlockManager, HostPool, OutOfBlocks, swap_in, swap_out
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -142,3 +142,42 @@ def test_long_context_prefill_slots_are_free_and_distinct():
     assert len(set(pre.tolist())) == 256
     used = set(st.block_tables[st.block_tables >= 0].tolist())
     assert not (set((pre // 64).tolist()) & used)
+
+
+def test_swap_out_and_in_round_trip_keeps_tokens_and_refcounts():
+    bm = BlockManager(12, 16, list(range(12))[::-1])
+    host = HostPool(8)
+    bm.allocate(0, 40)                     # 3 blocks
+    bm.fork(0, 1)                          # shares them
+    before = list(bm.tables[0])
+    out_pairs = swap_out(bm, host, 0)
+    assert [g for g, _ in out_pairs] == before and len(set(c for _, c in out_pairs)) == 3
+    assert 0 not in bm.tables and all(bm.ref[b] == 1 for b in before)   # still held by seq 1
+    bm.check()
+    in_pairs = swap_in(bm, host, 0)
+    assert [c for c, _ in in_pairs] == [c for _, c in out_pairs]
+    assert bm.lens[0] == 40 and len(bm.tables[0]) == 3
+    assert not set(bm.tables[0]) & set(before)                          # fresh private blocks
+    assert sorted(host.free) == list(range(8))
+    bm.check()
+
+
+def test_swap_out_fails_cleanly_when_host_pool_is_full():
+    bm = BlockManager(8, 16)
+    host = HostPool(1)
+    bm.allocate(0, 40)
+    with pytest.raises(OutOfBlocks):
+        swap_out(bm, host, 0)
+    assert len(bm.tables[0]) == 3
+    bm.check()
+
+
+def test_beam256_workload_forks_every_beam():
+    wl = workloads.beam256(0, steps=2, groups=2)
+    for st in wl.steps:
+        assert st.q.shape[0] == 64                        # 2 groups x 32 beams
+        dst = st.copy_pairs[:, 1]
+        assert len(set(dst.tolist())) == len(dst)
+        assert not (set(dst.tolist()) & set(st.copy_pairs[:, 0].tolist()))
+    # first step: 8 parents per group, each forked 4 ways -> 3 copies per parent with a partial tail
+    assert 0 < len(wl.steps[0].copy_pairs) <= 2 * 8 * 3

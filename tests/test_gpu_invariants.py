@@ -207,3 +207,71 @@ def test_bounded_wait_runs_out_reports_and_leaves_the_context_usable():
     st = wl.steps[0]
     out = decode(wl, wl.k_pool.cuda(), wl.v_pool.cuda(), st.block_tables, st.context_lens)
     assert torch.isfinite(out.float()).all() and pa.pa_device_errors() == 0
+
+
+def test_swap_blocks_round_trip_through_pinned_host_memory():
+    """Swap a batch out to a page-locked host pool and back into fresh GPU
+    blocks: pools bit-exact against the oracle's copies, and the decode after
+    swap-in equals the decode before swap-out bit for bit."""
+    import oracle
+    from paged_kv_cache_372_b200.block_manager import BlockManager, HostPool, swap_in, swap_out
+    from tests.bruteforce import bits_of
+    wl = workloads.llama3_8b(9, num_seqs=12)
+    st = wl.steps[0]
+    nb, bs = wl.num_blocks, wl.block_size
+    bm = BlockManager(nb, bs, list(range(nb)))
+    used = set(st.block_tables[st.block_tables >= 0].tolist())
+    bm.free = [b for b in range(nb) if b not in used][::-1]
+    for s_, n in enumerate(st.context_lens):
+        k = -(-int(n) // bs)
+        bm.tables[s_] = [int(b) for b in st.block_tables[s_, :k]]
+        bm.lens[s_] = int(n)
+        for b in bm.tables[s_]:
+            bm.ref[b] += 1
+    bm.check()
+    kp, vp = wl.k_pool.cuda(), wl.v_pool.cuda()
+    before = decode(wl, kp, vp, st.block_tables, st.context_lens)
+    host = HostPool(len(used) + 8)
+    hk = torch.empty((host.num_blocks,) + tuple(wl.k_pool.shape[1:]), dtype=wl.k_pool.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    okp, ovp = bits_of(wl.k_pool).copy(), bits_of(wl.v_pool).copy()
+    ohk, ohv = np.zeros_like(bits_of(hk)), np.zeros_like(bits_of(hv))
+    hk.zero_(); hv.zero_()
+    seqs = list(range(len(st.context_lens)))
+    out_pairs = [pr for s_ in seqs for pr in swap_out(bm, host, s_)]
+    pairs = torch.tensor(out_pairs, dtype=torch.int64).cuda()
+    pa.pa_swap_blocks([hk, hv], [kp, vp], pairs)
+    torch.cuda.synchronize()
+    oracle.swap_blocks([ohk, ohv], [okp, ovp], np.array(out_pairs), wl.block_bytes)
+    assert np.array_equal(bits_of(hk), ohk) and np.array_equal(bits_of(hv), ohv)
+    kp.fill_(float("nan")); vp.fill_(float("nan"))          # the GPU copies are gone
+    torch.cuda.synchronize()
+    start_k, start_v = bits_of(kp.cpu()).copy(), bits_of(vp.cpu()).copy()
+    in_pairs = [pr for s_ in seqs for pr in swap_in(bm, host, s_)]
+    pairs_in = torch.tensor(in_pairs, dtype=torch.int64).pin_memory()   # pairs from host memory
+    pa.pa_swap_blocks([kp, vp], [hk, hv], pairs_in)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    oracle.swap_blocks([start_k, start_v], [ohk, ohv], np.array(in_pairs), wl.block_bytes)
+    assert np.array_equal(bits_of(kp.cpu()), start_k) and np.array_equal(bits_of(vp.cpu()), start_v)
+    width = max(len(t) for t in bm.tables.values())
+    tables = bm.block_table_array(seqs, width)
+    after = decode(wl, kp, vp, tables, st.context_lens)
+    assert torch.equal(before, after)
+
+
+def test_swap_blocks_rejects_pageable_host_memory():
+    wl = workloads.tiny(0)
+    kp = wl.k_pool.cuda()
+    pageable = torch.zeros_like(wl.k_pool)                 # not page-locked
+    with pytest.raises(ValueError):
+        pa.pa_swap_blocks([pageable], [kp], torch.tensor([[0, 1]], dtype=torch.int64).cuda())
+    L = pa.lib()
+    import ctypes
+    dst = (ctypes.c_void_p * 1)(pageable.data_ptr())
+    src = (ctypes.c_void_p * 1)(kp.data_ptr())
+    pairs = torch.tensor([[0, 1]], dtype=torch.int64).cuda()
+    st = L.pa_swap_blocks(dst, src, 1, pairs.data_ptr(), 1, kp[0].numel() * 2, 32, 32, None)
+    assert st == pa.PA_ERR_INVALID and b"pageable" in L.pa_last_error()
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0

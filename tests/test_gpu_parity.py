@@ -58,6 +58,10 @@ def test_beam_all_steps():
     run_and_compare(workloads.beam(0))
 
 
+def test_beam256_steps():
+    run_and_compare(workloads.beam256(0, steps=3))
+
+
 def test_long32k_full():
     run_and_compare(workloads.long32k(0))
 
