@@ -75,6 +75,16 @@ class Oracle:
         L.oracle_copy_blocks.argtypes = [_P, _I, _P, _I, ctypes.c_size_t]
         L.oracle_swap_blocks.restype = None
         L.oracle_swap_blocks.argtypes = [_P, _P, _I, _P, _I, ctypes.c_size_t]
+        L.oracle_e4m3_to_double.restype = ctypes.c_double
+        L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_paged_attention_fp8.restype = None
+        L.oracle_paged_attention_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                                 ctypes.c_double, _I, ctypes.c_double, ctypes.c_double, _I]
+        L.oracle_reshape_and_cache_fp8.restype = None
+        L.oracle_reshape_and_cache_fp8.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                                                   ctypes.c_float, ctypes.c_float]
         L.oracle_slot_mapping.restype = None
         L.oracle_slot_mapping.argtypes = [_P, _P, _I, _P, _P, _I, _I]
 
@@ -84,6 +94,55 @@ class Oracle:
         flat = np.ascontiguousarray(bits, dtype=np.uint16).ravel()
         f = self.lib.oracle_to_double
         return np.array([f(int(b), code) for b in flat], dtype=np.float64).reshape(np.shape(bits))
+
+    def e4m3_to_double(self, codes) -> np.ndarray:
+        flat = np.ascontiguousarray(codes, dtype=np.uint8).ravel()
+        f = self.lib.oracle_e4m3_to_double
+        return np.array([f(int(c)) for c in flat], dtype=np.float64).reshape(np.shape(codes))
+
+    def e4m3_encode(self, values) -> np.ndarray:
+        flat = np.ascontiguousarray(values, dtype=np.float32).ravel()
+        f = self.lib.oracle_e4m3_encode
+        return np.array([f(float(v)) for v in flat], dtype=np.uint8).reshape(np.shape(values))
+
+    def paged_attention_fp8(self, q, k_pool, v_pool, block_tables, context_lens, scale, q_dtype,
+                            k_scale, v_scale, num_threads: int = 0) -> np.ndarray:
+        """out[s][h][:] in fp64 over E4M3 pools (uint8 codes) with per-tensor scales."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        k_pool = np.ascontiguousarray(k_pool, dtype=np.uint8)
+        v_pool = np.ascontiguousarray(v_pool, dtype=np.uint8)
+        block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+        context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+        B, H, D = q.shape
+        NB, Hkv, bs, D2 = k_pool.shape
+        assert D2 == D and v_pool.shape == k_pool.shape and H % Hkv == 0
+        for s in range(B):
+            n = int(context_lens[s])
+            pages = -(-n // bs)
+            assert 0 <= n and pages <= block_tables.shape[1]
+            if pages:
+                used = block_tables[s, :pages]
+                assert used.min() >= 0 and used.max() < NB
+        out = np.zeros((B, H, D), dtype=np.float64)
+        self.lib.oracle_paged_attention_fp8(
+            _ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), _ptr(context_lens),
+            B, H, Hkv, D, bs, block_tables.shape[1], float(scale), dtype_code(q_dtype), float(k_scale),
+            float(v_scale), int(num_threads))
+        return out
+
+    def reshape_and_cache_fp8(self, k, v, k_pool, v_pool, slot_mapping, dtype, k_scale, v_scale) -> None:
+        """In place on uint8 E4M3 pools: code = encode(x / scale) in fp32."""
+        for a in (k_pool, v_pool):
+            assert a.dtype == np.uint8 and a.flags.c_contiguous
+        k = np.ascontiguousarray(k, dtype=np.uint16)
+        v = np.ascontiguousarray(v, dtype=np.uint16)
+        slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        T, Hkv, D = k.shape
+        NB, Hkv2, bs, D2 = k_pool.shape
+        assert Hkv2 == Hkv and D2 == D and v.shape == k.shape and slot_mapping.shape == (T,)
+        assert slot_mapping.max(initial=-1) < NB * bs
+        self.lib.oracle_reshape_and_cache_fp8(_ptr(k), _ptr(v), _ptr(k_pool), _ptr(v_pool), _ptr(slot_mapping),
+                                              T, Hkv, D, bs, dtype_code(dtype), float(k_scale), float(v_scale))
 
     def max_threads(self) -> int:
         return int(self.lib.oracle_max_threads())
@@ -196,6 +255,14 @@ def slot_mapping(*args, **kwargs):
 
 def swap_blocks(*args, **kwargs):
     return get().swap_blocks(*args, **kwargs)
+
+
+def paged_attention_fp8(*args, **kwargs):
+    return get().paged_attention_fp8(*args, **kwargs)
+
+
+def reshape_and_cache_fp8(*args, **kwargs):
+    return get().reshape_and_cache_fp8(*args, **kwargs)
 
 
 def to_double(*args, **kwargs):

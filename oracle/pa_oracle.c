@@ -71,6 +71,67 @@ double oracle_to_double(uint16_t bits, int dtype)
     return sign ? -mag : mag;
 }
 
+/*
+ * 8-bit E4M3 ("fp8 e4m3fn"): 1 sign bit, 4 exponent bits (bias 7), 3 fraction
+ * bits, no infinities, one NaN pattern per sign (exponent and fraction all
+ * ones), largest finite magnitude 448. Quantised KV cache of
+ * "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
+ * section 3.2 (内存压缩技术: store K/V in fewer bits). Decoded here from the
+ * bit fields.
+ */
+double oracle_e4m3_to_double(uint8_t code)
+{
+    const int sign = (code >> 7) & 1;
+    const int e = (code >> 3) & 0xf;
+    const int m = code & 7;
+    double mag;
+    if (e == 15 && m == 7)
+        mag = NAN;
+    else if (e == 0)
+        mag = ldexp((double)m, -9);          /* subnormal: m * 2^(1-7-3) */
+    else
+        mag = ldexp((double)(m + 8), e - 10);
+    return sign ? -mag : mag;
+}
+
+/*
+ * Nearest E4M3 code to y, ties to even, magnitudes past 448 saturated to 448
+ * (NaN stays NaN). Works on the value exactly (y is a float, so y * 2^k is
+ * exact in double).
+ */
+uint8_t oracle_e4m3_encode(float y)
+{
+    if (isnan(y))
+        return 0x7f;
+    const uint8_t sign = signbit(y) ? 0x80 : 0;
+    double a = fabs((double)y);
+    if (a >= 464.0)                         /* rounds past 448: saturate */
+        return sign | 0x7e;
+    int e;
+    if (a < ldexp(1.0, -6)) {               /* subnormal range, step 2^-9 */
+        double q = a * 512.0;
+        double r = floor(q);
+        double f = q - r;
+        if (f > 0.5 || (f == 0.5 && fmod(r, 2.0) == 1.0))
+            r += 1.0;
+        return sign | (uint8_t)r;           /* r == 8 is the smallest normal */
+    }
+    frexp(a, &e);                           /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                 /* a in [2^e, 2^(e+1)) */
+    double q = ldexp(a, 3 - e);             /* in [8, 16): 8 + fraction * 8 */
+    double r = floor(q);
+    double f = q - r;
+    if (f > 0.5 || (f == 0.5 && fmod(r, 2.0) == 1.0))
+        r += 1.0;
+    if (r == 16.0) {
+        r = 8.0;
+        e += 1;
+    }
+    if (e > 8 || (e == 8 && r > 14.0))      /* above 448 after rounding */
+        return sign | 0x7e;
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)r - 8));
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP
@@ -168,6 +229,112 @@ void oracle_paged_attention(double *out, const uint16_t *q,
         }
         free(scores);
         free(qd);
+    }
+}
+
+/*
+ * Paged decode attention over an E4M3 KV cache: the same computation as
+ * oracle_paged_attention with every key element k_scale * decode(code) and
+ * every value element v_scale * decode(code), in fp64.
+ */
+void oracle_paged_attention_fp8(double *out, const uint16_t *q,
+                                const uint8_t *k_pool, const uint8_t *v_pool,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int num_heads, int num_kv_heads,
+                                int head_dim, int block_size, int max_blocks_per_seq,
+                                double scale, int q_dtype, double k_scale, double v_scale,
+                                int num_threads)
+{
+    const int group = num_heads / num_kv_heads;
+    const long pairs = (long)num_seqs * num_heads;
+#ifdef _OPENMP
+    if (num_threads > 0)
+        omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long sh = 0; sh < pairs; sh++) {
+        const int s = (int)(sh / num_heads);
+        const int h = (int)(sh % num_heads);
+        const int kvh = h / group;
+        const int n = context_lens[s];
+        double *o = out + (size_t)sh * head_dim;
+        for (int d = 0; d < head_dim; d++)
+            o[d] = 0.0;
+        if (n <= 0)
+            continue;
+        double *qd = (double *)malloc(sizeof(double) * head_dim);
+        double *scores = (double *)malloc(sizeof(double) * n);
+        for (int d = 0; d < head_dim; d++)
+            qd[d] = oracle_to_double(q[(size_t)sh * head_dim + d], q_dtype);
+        const int pages = (n + block_size - 1) / block_size;
+        const int32_t *table = block_tables + (size_t)s * max_blocks_per_seq;
+        for (int i = 0; i < pages; i++) {
+            const size_t page = (size_t)table[i];
+            for (int r = 0; r < block_size; r++) {
+                const int t = i * block_size + r;
+                if (t >= n)
+                    break;
+                const uint8_t *key = k_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;
+                double dot = 0.0;
+                for (int d = 0; d < head_dim; d++)
+                    dot += qd[d] * (k_scale * oracle_e4m3_to_double(key[d]));
+                scores[t] = dot;
+            }
+        }
+        double mx = -INFINITY;
+        for (int t = 0; t < n; t++)
+            if (scale * scores[t] > mx)
+                mx = scale * scores[t];
+        double total = 0.0;
+        for (int t = 0; t < n; t++) {
+            scores[t] = exp(scale * scores[t] - mx);
+            total += scores[t];
+        }
+        for (int t = 0; t < n; t++)
+            scores[t] /= total;
+        for (int i = 0; i < pages; i++) {
+            const size_t page = (size_t)table[i];
+            for (int r = 0; r < block_size; r++) {
+                const int t = i * block_size + r;
+                if (t >= n)
+                    break;
+                const uint8_t *val = v_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;
+                for (int d = 0; d < head_dim; d++)
+                    o[d] += scores[t] * (v_scale * oracle_e4m3_to_double(val[d]));
+            }
+        }
+        free(scores);
+        free(qd);
+    }
+}
+
+/*
+ * Quantising cache write: like oracle_reshape_and_cache, but each element x
+ * (fp16/bf16) is stored as oracle_e4m3_encode(x / scale) with the division in
+ * fp32 (float operands, IEEE single, round to nearest).
+ */
+void oracle_reshape_and_cache_fp8(const uint16_t *k, const uint16_t *v,
+                                  uint8_t *k_pool, uint8_t *v_pool,
+                                  const int64_t *slot_mapping, int num_tokens,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int dtype, float k_scale, float v_scale)
+{
+    for (int t = 0; t < num_tokens; t++) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; h++) {
+            const size_t src = ((size_t)t * num_kv_heads + h) * head_dim;
+            const size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) * head_dim;
+            for (int d = 0; d < head_dim; d++) {
+                const float kx = (float)oracle_to_double(k[src + d], dtype);
+                const float vx = (float)oracle_to_double(v[src + d], dtype);
+                k_pool[dst + d] = oracle_e4m3_encode(kx / k_scale);
+                v_pool[dst + d] = oracle_e4m3_encode(vx / v_scale);
+            }
+        }
     }
 }
 

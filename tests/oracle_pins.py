@@ -15,6 +15,11 @@ What pins what:
                           unwritten tail slots, GQA head mapping)
   * cache write / copies  numpy fancy-index scatter and slice copies
   * slot mapping          enumeration of the contiguous token order
+  * E4M3 (fp8) codes      all 256 codes vs torch's float8_e4m3fn; encoding vs
+                          torch's cast (in range, exact midpoints), saturation
+                          closed forms, round trip of every finite code
+  * fp8 attention / write brute force over the numpy-dequantised cache; numpy
+                          float32 division + torch's cast
 """
 from __future__ import annotations
 
@@ -272,6 +277,83 @@ def pin_swap_blocks(orc, seed=11):
         assert np.array_equal(x, b)
 
 
+def _torch_e4m3_codes(x: np.ndarray) -> np.ndarray:
+    """float32 -> E4M3 codes through torch's own float8_e4m3fn cast (in-range values)."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy()
+
+
+def pin_e4m3_decode(orc):
+    codes = np.arange(256, dtype=np.uint8)
+    got = orc.e4m3_to_double(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref)) and np.isnan(got).sum() == 2
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+    assert got[0x7e] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def pin_e4m3_encode(orc, seed=12):
+    rng = np.random.default_rng(seed)
+    x = np.concatenate([rng.standard_normal(3000) * s for s in (1e-3, 0.05, 1.0, 20.0, 120.0)])
+    x = np.clip(x, -440.0, 440.0).astype(np.float32)
+    codes = np.arange(256, dtype=np.uint8)
+    vals = orc.e4m3_to_double(codes)
+    finite = codes[~np.isnan(vals)]
+    mids = []                                   # exact midpoints between neighbours: ties to even
+    pos = np.sort(vals[(vals >= 0) & ~np.isnan(vals)])
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids, vals[~np.isnan(vals)].astype(np.float32)])
+    assert np.array_equal(orc.e4m3_encode(x), _torch_e4m3_codes(x))
+    # saturation (no infinities in E4M3): past 448 the code is +-448
+    big = np.array([448.0, 449.0, 463.9, 464.0, 1e6, -500.0, np.inf, -np.inf], dtype=np.float32)
+    assert list(orc.e4m3_encode(big)) == [0x7e, 0x7e, 0x7e, 0x7e, 0x7e, 0xfe, 0x7e, 0xfe]
+    # every finite code round-trips
+    assert np.array_equal(orc.e4m3_encode(vals[finite].astype(np.float32)), finite)
+
+
+def _fp8_case(rng, B, H, Hkv, D, bs, ctx, dtype):
+    q, kp, vp, tab, cl = _case(rng, B, H, Hkv, D, bs, ctx, dtype)
+    k8 = rng.integers(0, 256, kp.shape, dtype=np.uint8)
+    v8 = rng.integers(0, 256, vp.shape, dtype=np.uint8)
+    for a in (k8, v8):                          # no NaN codes in the cache
+        a[(a & 0x7f) == 0x7f] = 0x10
+    return q, k8, v8, tab, cl
+
+
+def pin_fp8_attention_bruteforce(orc, seed=13):
+    """fp8 attention = attention over the dequantised cache (numpy dequantisation)."""
+    rng = np.random.default_rng(seed)
+    for B, H, Hkv, D, bs, ctx, dt in SHAPES:
+        q, k8, v8, tab, cl = _fp8_case(rng, B, H, Hkv, D, bs, ctx, dt)
+        ks, vs = 0.37, 1.9
+        got = orc.paged_attention_fp8(q, k8, v8, tab, cl, 1.0 / math.sqrt(D), dt, ks, vs)
+        deq = lambda a, sc: torch.from_numpy(a).view(torch.float8_e4m3fn).to(torch.float64).numpy() * sc
+        ref = contiguous_attention(decode(q, dt), deq(k8, ks), deq(v8, vs), tab, cl, 1.0 / math.sqrt(D))
+        # random codes span the whole E4M3 range (|v| up to 448 * vs): relative bound
+        assert np.abs(got - ref).max() <= ATOL * max(1.0, np.abs(ref).max())
+
+
+def pin_fp8_cache_write(orc, seed=14):
+    """Quantising write: code = E4M3(x / scale) with the division in float32."""
+    rng = np.random.default_rng(seed)
+    NB, Hkv, bs, D, T = 5, 2, 16, 32, 12
+    for dt in ("f16", "bf16"):
+        k = _rand_bits(rng, (T, Hkv, D), dt)
+        v = _rand_bits(rng, (T, Hkv, D), dt)
+        kp = rng.integers(0, 256, (NB, Hkv, bs, D), dtype=np.uint8)
+        vp = rng.integers(0, 256, (NB, Hkv, bs, D), dtype=np.uint8)
+        slots = rng.choice(NB * bs, T, replace=False).astype(np.int64)
+        ks, vs = np.float32(0.0213), np.float32(0.75)
+        ek, ev = kp.copy(), vp.copy()
+        kx = (decode(k, dt).astype(np.float32) / ks).astype(np.float32)
+        vx = (decode(v, dt).astype(np.float32) / vs).astype(np.float32)
+        ek[slots // bs, :, slots % bs, :] = _torch_e4m3_codes(np.clip(kx, -448, 448))
+        ev[slots // bs, :, slots % bs, :] = _torch_e4m3_codes(np.clip(vx, -448, 448))
+        orc.reshape_and_cache_fp8(k, v, kp, vp, slots, dt, float(ks), float(vs))
+        assert np.array_equal(kp, ek) and np.array_equal(vp, ev)
+
+
 def pin_slot_mapping(orc, seed=10):
     rng = np.random.default_rng(seed)
     bs, B, W = 16, 5, 6
@@ -290,4 +372,5 @@ def pin_slot_mapping(orc, seed=10):
 ALL_PINS = [pin_decode_f16, pin_decode_bf16, pin_bruteforce, pin_sdpa, pin_single_token,
             pin_equal_keys, pin_two_token_closed_form, pin_block_permutation,
             pin_shared_equals_duplicated, pin_tail_slots_ignored, pin_gqa_mapping,
-            pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_swap_blocks, pin_slot_mapping]
+            pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_swap_blocks, pin_slot_mapping,
+            pin_e4m3_decode, pin_e4m3_encode, pin_fp8_attention_bruteforce, pin_fp8_cache_write]

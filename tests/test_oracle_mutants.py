@@ -41,6 +41,18 @@ MUTATIONS = {
                        "const int64_t src = src_dst_pairs[2 * p + 1];\n        const int64_t dst = src_dst_pairs[2 * p];"),
     "swap_pool_index": ("memcpy(dst_pools[i] + (size_t)dst * block_bytes,\n                   src_pools[i] + (size_t)src * block_bytes, block_bytes);",
                         "memcpy(dst_pools[i] + (size_t)dst * block_bytes,\n                   src_pools[num_pools - 1 - i] + (size_t)src * block_bytes, block_bytes);"),
+    "e4m3_bias": ("mag = ldexp((double)(m + 8), e - 10);", "mag = ldexp((double)(m + 8), e - 11);"),
+    "e4m3_subnormal_step": ("mag = ldexp((double)m, -9);", "mag = ldexp((double)m, -10);"),
+    "e4m3_ties_away": ("if (f > 0.5 || (f == 0.5 && fmod(r, 2.0) == 1.0))\n        r += 1.0;\n    if (r == 16.0)",
+                       "if (f >= 0.5)\n        r += 1.0;\n    if (r == 16.0)"),
+    "e4m3_saturation": ("if (a >= 464.0)                         /* rounds past 448: saturate */\n        return sign | 0x7e;",
+                        "if (a >= 464.0)                         /* rounds past 448: saturate */\n        return sign | 0x7d;"),
+    "fp8_key_scale_dropped": ("dot += qd[d] * (k_scale * oracle_e4m3_to_double(key[d]));",
+                              "dot += qd[d] * oracle_e4m3_to_double(key[d]);"),
+    "fp8_value_scale_dropped": ("o[d] += scores[t] * (v_scale * oracle_e4m3_to_double(val[d]));",
+                                "o[d] += scores[t] * oracle_e4m3_to_double(val[d]);"),
+    "fp8_write_scale_times": ("k_pool[dst + d] = oracle_e4m3_encode(kx / k_scale);",
+                              "k_pool[dst + d] = oracle_e4m3_encode(kx * k_scale);"),
     "slot_offset": ("slots[i] = (int64_t)table[pos / block_size] * block_size + pos % block_size;",
                     "slots[i] = (int64_t)table[pos / block_size] * block_size + (pos + 1) % block_size;"),
 }
