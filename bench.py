@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--kv", default="auto", choices=["auto", "fp8"],
+                    help="fp8: E4M3 KV cache (pa_reshape_and_cache_fp8 + pa_decode_fp8)")
     ap.add_argument("--unfused", action="store_true",
                     help="separate cache-write launch instead of pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
@@ -72,6 +74,7 @@ def describe(wl) -> dict:
 
 
 L2_BYTES = 126 * 1024 * 1024
+FP8_SCALE = 0.0375  # N(0,1) values / 0.0375 stay well inside E4M3's +-448
 
 
 def needs_flush(wl) -> bool:
@@ -228,7 +231,19 @@ def run_ours(args, world, rank, local):
     flush = needs_flush(wl)
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
 
-    fused = not args.unfused and appends_at_last_positions(wl)
+    kv8 = args.kv == "fp8"
+    fused = not args.unfused and not kv8 and appends_at_last_positions(wl)
+    if kv8:
+        # The whole cache quantised once by the library's own E4M3 cache write.
+        NB, Hkv, bs, D = kp.shape
+        k8 = torch.empty((NB, Hkv, bs, D), dtype=torch.uint8, device=dev)
+        v8 = torch.empty_like(k8)
+        all_slots = torch.arange(NB * bs, dtype=torch.int64, device=dev)
+        pa.pa_reshape_and_cache_fp8(kp.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous(),
+                                    vp.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous(), k8, v8,
+                                    all_slots, FP8_SCALE, FP8_SCALE)
+        del kp, vp
+        kp, vp = k8, v8
     for d in dev_steps:
         d["k_dec"], d["v_dec"] = d["k"][:B].contiguous(), d["v"][:B].contiguous()
         d["k_extra"], d["v_extra"], d["slots_extra"] = d["k"][B:], d["v"][B:], d["slots"][B:]
@@ -239,7 +254,10 @@ def run_ours(args, world, rank, local):
         if d["pairs"].shape[0]:
             pa.pa_copy_blocks([kp, vp], d["pairs"])
             n += 1
-        if fused:
+        if kv8:
+            pa.pa_reshape_and_cache_fp8(d["k"], d["v"], kp, vp, d["slots"], FP8_SCALE, FP8_SCALE)
+            n += 1
+        elif fused:
             if d["slots_extra"].shape[0]:
                 pa.pa_reshape_and_cache(d["k_extra"], d["v_extra"], kp, vp, d["slots_extra"])
                 n += 1
@@ -248,7 +266,10 @@ def run_ours(args, world, rank, local):
             n += 1
         if ev is not None:
             ev[0].record(stream)
-        if fused:
+        if kv8:
+            pa.pa_decode_fp8(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, FP8_SCALE,
+                             FP8_SCALE, P, ws)
+        elif fused:
             pa.pa_decode_append(d["out"], d["q"], d["k_dec"], d["v_dec"], kp, vp, d["tables"], d["ctx"], wl.scale,
                                 max_ctx, P, ws)
         else:
@@ -291,15 +312,17 @@ def run_ours(args, world, rank, local):
     seqs = B * world
     value = seqs / (ms_per_step / 1e3)
 
-    kv_bytes = float(np.mean([wl.kv_bytes(i % nsteps) for i in range(args.steps)]))
+    eb = 0.5 if kv8 else 1.0   # kv_bytes counts 2-byte elements
+    kv_bytes = eb * float(np.mean([wl.kv_bytes(i % nsteps) for i in range(args.steps)]))
     uniq = [wl.kv_bytes_unique(i) for i in range(nsteps)]
-    kv_unique = float(np.mean([uniq[i % nsteps] for i in range(args.steps)]))
+    kv_unique = eb * float(np.mean([uniq[i % nsteps] for i in range(args.steps)]))
     peak, peak_kind = measured_peaks()
     achieved = kv_unique / (decode_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": value, "unit": "seqs/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block pool)",
+        "vs_baseline": None, "dtype": (f"e4m3 KV cache, {wl.dtype} q/out" if kv8 else wl.dtype),
+        "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block pool)",
         "config": describe(wl),
         "kv_gbs": kv_unique * world / (ms_per_step * 1e-3) / 1e9,
         "decode_ms": decode_ms_max,
@@ -309,23 +332,28 @@ def run_ours(args, world, rank, local):
         "hbm_frac_of_nominal_8000": achieved / 8000.0,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
-                     "kernel": ("pa_decode_append call (plan + attention launches; cache write and split "
+                     "kernel": ("pa_decode_fp8 call (plan + attention launches; split merge fused)" if kv8 else
+                                "pa_decode_append call (plan + attention launches; cache write and split "
                                 "merge fused)" if fused else
                                 "pa_decode call (plan + attention launches; split merge fused)"),
                      "bytes": "unique K+V bytes of valid tokens per call",
                      "traffic": profiled_traffic(wl.name if args.partition is None
                                                  else f"{wl.name}@P{args.partition}")},
         "gpu_launches": launches,
-        "step": ("pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_append"
+        "step": ("pa_copy_blocks (if any), pa_reshape_and_cache_fp8, pa_decode_fp8" if kv8 else
+                 "pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_append"
                  if fused else "pa_copy_blocks (if any), pa_reshape_and_cache, pa_decode"),
         "clocks": clk,
     }
-    if rank == 0 and not args.no_e2e:
-        result["e2e"] = run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused)
-    elif not args.no_e2e:
-        run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused)
+    if kv8:
+        result["config"]["kv_cache"] = f"E4M3 codes, k_scale = v_scale = {FP8_SCALE}"
+        result["config"]["kv_bytes_per_step"] = int(kv_bytes)
+    if not args.no_e2e and not kv8:
+        e2e = run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused)
+        if rank == 0:
+            result["e2e"] = e2e
     pa.pa_device_errors()
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu and not kv8:
         result["cpu_baseline"] = cpu_baseline(wl)
     return result
 

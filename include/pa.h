@@ -149,6 +149,42 @@ PA_API pa_status pa_decode_append(void *out, const void *q, const void *k_new, c
                                   float scale, int dtype, int partition_size, void *workspace,
                                   size_t workspace_bytes, pa_stream_t stream);
 
+/*
+ * Paged decode attention over an 8-bit E4M3 ("fp8 e4m3fn") KV cache with
+ * per-tensor scales: key element = k_scale * E4M3 code, value element =
+ * v_scale * E4M3 code; otherwise exactly pa_decode (q and out stay fp16/bf16
+ * by `dtype`). k_pool, v_pool: uint8 codes [num_blocks][num_kv_heads]
+ * [block_size][head_dim], written by pa_reshape_and_cache_fp8. head_dim 128.
+ * The products run on tensor cores with the codes widened to fp16 (exact) and
+ * the queries converted to fp16 (exact for |q| in fp16's normal range); the
+ * workspace is sized by pa_decode_workspace_size as for pa_decode.
+ *
+ * Defined by: "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
+ * section 3.2 (内存压缩技术) — keep the KV cache in fewer bits to cut its
+ * memory; the attention itself is that of section 3.1.
+ */
+PA_API pa_status pa_decode_fp8(void *out, const void *q, const void *k_pool, const void *v_pool,
+                               const int32_t *block_tables, const int32_t *context_lens,
+                               int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                               int block_size, int max_blocks_per_seq, int num_blocks,
+                               int max_context_len, float scale, int dtype, float k_scale,
+                               float v_scale, int partition_size, void *workspace,
+                               size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * Quantising cache write for an E4M3 cache: like pa_reshape_and_cache, but
+ * each element x of k (v) is stored as the E4M3 code of x / k_scale
+ * (x / v_scale): fp32 division rounded to nearest, then round-to-nearest-even
+ * to E4M3 with magnitudes past 448 saturated to 448. k, v fp16/bf16 (dtype);
+ * pools uint8, 8-byte aligned. Same slot rules and error reporting as
+ * pa_reshape_and_cache. Defined by the same section 3.2.
+ */
+PA_API pa_status pa_reshape_and_cache_fp8(const void *k, const void *v, void *k_pool, void *v_pool,
+                                          const int64_t *slot_mapping, int num_tokens,
+                                          int num_kv_heads, int head_dim, int block_size,
+                                          int num_blocks, int dtype, float k_scale, float v_scale,
+                                          pa_stream_t stream);
+
 /* Workspace bytes pa_decode needs for these sizes (0 if the shape is invalid). */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
                                 int head_dim, int block_size, int max_context_len,

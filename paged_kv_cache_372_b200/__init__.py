@@ -54,6 +54,11 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_append.restype = _I
         L.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                        _I, _P, _SZ, _P]
+        L.pa_decode_fp8.restype = _I
+        L.pa_decode_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _F, _F, _I,
+                                    _P, _SZ, _P]
+        L.pa_reshape_and_cache_fp8.restype = _I
+        L.pa_reshape_and_cache_fp8.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P]
         L.pa_decode_workspace_size.restype = _SZ
         L.pa_decode_workspace_size.argtypes = [_I] * 7
         L.pa_decode_partition_size.restype = _I
@@ -176,6 +181,43 @@ def pa_decode_append(out, q, k_new, v_new, k_pool, v_pool, block_tables, context
         int(max_context_len), float(scale), _DTYPES[q.dtype], int(partition_size), _cuda(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+def pa_decode_fp8(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len, k_scale, v_scale,
+                  partition_size=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode over an E4M3 cache: k_pool, v_pool uint8 codes [NB][Hkv][bs][D];
+    element = scale * code (k_scale for keys, v_scale for values)."""
+    B, H, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch between q, out and the pools")
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("fp8 pools must be uint8 tensors of E4M3 codes")
+    if q.dtype not in _DTYPES or out.dtype != q.dtype:
+        raise ValueError("q and out must share one dtype, fp16 or bf16")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device)
+    _check(lib().pa_decode_fp8(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
+        B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
+        float(k_scale), float(v_scale), int(partition_size), _cuda(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def pa_reshape_and_cache_fp8(k, v, k_pool, v_pool, slot_mapping, k_scale, v_scale, stream=None) -> None:
+    """Quantising write: k_pool[slot] = E4M3(k[t] / k_scale) (and v) for t with slot >= 0."""
+    T, Hkv, D = k.shape
+    NB, Hkv2, bs, D2 = k_pool.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(v.shape) != tuple(k.shape) or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("shape mismatch between k, v and the pools")
+    if k.dtype not in _DTYPES or v.dtype != k.dtype or k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("k, v fp16/bf16; pools uint8")
+    _check(lib().pa_reshape_and_cache_fp8(
+        _cuda(k, "k"), _cuda(v, "v"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, bs, NB, _DTYPES[k.dtype], float(k_scale),
+        float(v_scale), _stream(stream)))
 
 
 def pa_reshape_and_cache(k, v, k_pool, v_pool, slot_mapping, stream=None) -> None:

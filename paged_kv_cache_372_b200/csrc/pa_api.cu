@@ -127,8 +127,12 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
                       const void *v_pool, const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                       int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
                       int num_blocks, int max_context_len, float scale, int dtype, int partition_size,
-                      void *workspace, size_t workspace_bytes, pa_stream_t stream) {
+                      void *workspace, size_t workspace_bytes, pa_stream_t stream, bool kv8 = false,
+                      float k_scale = 1.f, float v_scale = 1.f) {
     g_last_error.clear();
+    if (kv8 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "fp8 cache supports head_dim 128, got %d", head_dim);
+    if (kv8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || k_scale == INFINITY || v_scale == INFINITY))
+        return fail(PA_ERR_INVALID, "k_scale and v_scale must be positive and finite");
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 || partition_size < 0)
         return fail(PA_ERR_INVALID, "negative or zero size argument");
     if (dtype != PA_F16 && dtype != PA_BF16) return fail(PA_ERR_INVALID, "dtype %d", dtype);
@@ -177,7 +181,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     p.ctx_limit = ctx_limit;
     p.partition = P;
     p.max_parts = max_parts;
-    p.qscale = scale * 1.4426950408889634f;
+    p.qscale = scale * 1.4426950408889634f * k_scale;
+    p.v_scale = v_scale;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.counter = reinterpret_cast<int *>(ws);
     p.num_entries = reinterpret_cast<int *>(ws) + 1;
@@ -188,6 +193,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int group = num_heads / num_kv_heads;
+    if (kv8)
+        return dtype == PA_F16 ? dispatch_group_fp8<__half>(p, group, s) : dispatch_group_fp8<__nv_bfloat16>(p, group, s);
     if (head_dim == 128)
         return dtype == PA_F16 ? dispatch_group<128, __half>(p, group, s)
                                : dispatch_group<128, __nv_bfloat16>(p, group, s);
@@ -205,6 +212,16 @@ pa_status pa_decode(void *out, const void *q, const void *k_pool, const void *v_
     return decode_impl(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
                        num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
                        dtype, partition_size, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_fp8(void *out, const void *q, const void *k_pool, const void *v_pool, const int32_t *block_tables,
+                        const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                        int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                        int dtype, float k_scale, float v_scale, int partition_size, void *workspace,
+                        size_t workspace_bytes, pa_stream_t stream) {
+    return decode_impl(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream, true, k_scale, v_scale);
 }
 
 pa_status pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new, void *k_pool,
@@ -249,6 +266,45 @@ pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void 
         (long long)num_blocks * block_size);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pa_reshape_and_cache launch");
+    return PA_OK;
+}
+
+pa_status pa_reshape_and_cache_fp8(const void *k, const void *v, void *k_pool, void *v_pool,
+                                   const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                   int block_size, int num_blocks, int dtype, float k_scale, float v_scale,
+                                   pa_stream_t stream) {
+    g_last_error.clear();
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return fail(PA_ERR_INVALID, "size argument");
+    if (dtype != PA_F16 && dtype != PA_BF16) return fail(PA_ERR_INVALID, "dtype %d", dtype);
+    if (head_dim != 64 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d", head_dim);
+    if (block_size != 16 && block_size != 32 && block_size != 64)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d", block_size);
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || k_scale == INFINITY || v_scale == INFINITY)
+        return fail(PA_ERR_INVALID, "k_scale and v_scale must be positive and finite");
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !k_pool || !v_pool || !slot_mapping) return fail(PA_ERR_INVALID, "null pointer");
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_pool, 8) || !aligned(v_pool, 8) || !aligned(slot_mapping, 8))
+        return fail(PA_ERR_INVALID, "misaligned pointer");
+    DeviceInfo info;
+    pa_status st = device_info(&info);
+    if (st != PA_OK) return st;
+    const int vec_per_row = head_dim / 8;
+    const long long total = (long long)num_tokens * num_kv_heads * vec_per_row;
+    long long blocks = (total + 255) / 256;
+    if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == PA_F16)
+        pa::pa_reshape_fp8_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint2 *>(k_pool),
+            static_cast<uint2 *>(v_pool), slot_mapping, total, vec_per_row, num_kv_heads, block_size,
+            (long long)num_blocks * block_size, k_scale, v_scale);
+    else
+        pa::pa_reshape_fp8_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint2 *>(k_pool),
+            static_cast<uint2 *>(v_pool), slot_mapping, total, vec_per_row, num_kv_heads, block_size,
+            (long long)num_blocks * block_size, k_scale, v_scale);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pa_reshape_and_cache_fp8 launch");
     return PA_OK;
 }
 

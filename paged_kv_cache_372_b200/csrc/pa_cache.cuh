@@ -9,6 +9,8 @@
 // Both are bit copies. Out-of-range indices are skipped and flagged.
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "pa_common.cuh"
 
 namespace pa {
@@ -40,6 +42,53 @@ __global__ void __launch_bounds__(256) pa_reshape_kernel(const uint4 *__restrict
         const uint4 vv = v[i];
         k_pool[dst] = kv;
         v_pool[dst] = vv;
+    }
+}
+
+// Quantising cache write for an E4M3 (fp8) cache: code = E4M3(x / scale),
+// the division in fp32 (IEEE, round to nearest), the conversion rounding to
+// nearest even and saturating at +-448. One thread turns one 16-byte vector of
+// K (8 elements) into 8 codes, and the same for V.
+template <typename T>
+__global__ void __launch_bounds__(256) pa_reshape_fp8_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                                                             uint2 *__restrict__ k_pool, uint2 *__restrict__ v_pool,
+                                                             const int64_t *__restrict__ slot_mapping,
+                                                             long long total_vectors, int vec_per_row,
+                                                             int num_kv_heads, int block_size, long long num_slots,
+                                                             float k_scale, float v_scale) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vectors; i += stride) {
+        const long long row = i / vec_per_row;
+        const int vec = (int)(i - row * vec_per_row);
+        const long long t = row / num_kv_heads;
+        const int h = (int)(row - t * num_kv_heads);
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+            raise_error(PA_DEVERR_SLOT);
+            continue;
+        }
+        const int64_t blk = slot / block_size;
+        const int64_t off = slot - blk * block_size;
+        const size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * vec_per_row + vec;
+        const uint4 src[2] = {k[i], v[i]};
+        const float sc[2] = {k_scale, v_scale};
+        uint2 codes[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint32_t w[4] = {src[j].x, src[j].y, src[j].z, src[j].w};
+            uint32_t c[2] = {0u, 0u};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = Elem<T>::pair(w[q]);
+                const float2 y = make_float2(__fdiv_rn(f.x, sc[j]), __fdiv_rn(f.y, sc[j]));
+                const uint32_t two = (uint32_t)__nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+                c[q >> 1] |= two << (16 * (q & 1));
+            }
+            codes[j] = make_uint2(c[0], c[1]);
+        }
+        k_pool[dst] = codes[0];
+        v_pool[dst] = codes[1];
     }
 }
 

@@ -44,7 +44,8 @@ struct DecodeParams {
     int ctx_limit;   // context lengths are clamped to [0, ctx_limit]
     int partition;   // P, tokens per partition
     int max_parts;   // ceil(ctx_limit / P)
-    float qscale;    // scale * log2(e)
+    float qscale;    // scale * log2(e) (times k_scale for an fp8 cache)
+    float v_scale;   // fp8 cache: dequantisation scale of V (1 otherwise)
     int *counter;    // work-list cursor (reset by the plan kernel)
     int *num_entries;
     int4 *entries;   // {seq, partition, tokens, partitions of seq}

@@ -18,30 +18,56 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp8.h>
+
+#include <type_traits>
 
 #include "pa_decode.cuh"
 
 namespace pa {
 
-template <int D, int G>
+// KV8: the pools hold E4M3 (fp8) codes, one byte per element, dequantised
+// with per-tensor scales (k_scale folded into the score scale, v_scale into
+// the output scale).
+template <int D, int G, bool KV8 = false>
 struct MmaGeo {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "head group size");
-    static constexpr int KS = D / 16;                    // 16-wide slices of a row
-    static constexpr int NBOX = D / 64;                  // 128-byte TMA boxes per row
-    static constexpr int HALF_BYTES = 16 * D * 2;        // one K (or V) tile
-    static constexpr int STAGE_BYTES = 2 * HALF_BYTES;   // K then V of one tile
+    static_assert(!KV8 || D == 128, "fp8 cache: head_dim 128");
+    static constexpr int EB = KV8 ? 1 : 2;                // bytes per pool element
+    static constexpr int KS = D / 16;                     // 16-wide slices of a row
+    static constexpr int NBOX = D * EB / 128;             // 128-byte TMA boxes per row
+    static constexpr int HALF_BYTES = 16 * D * EB;        // one K (or V) tile
+    static constexpr int STAGE_BYTES = 2 * HALF_BYTES;    // K then V of one tile
     static constexpr int Q_BYTES = G * D * 2;
 };
 
-template <int D, int G, int NS>
+template <int D, int G, int NS, bool KV8 = false>
 __host__ __device__ constexpr int mma_smem_bytes(int warps) {
     // 1024 bytes of slack re-align the base for the 128-byte swizzle pattern.
-    return 1024 + warps * (NS * MmaGeo<D, G>::STAGE_BYTES + 2 * MmaGeo<D, G>::Q_BYTES) + warps * NS * 8;
+    return 1024 + warps * (NS * MmaGeo<D, G, KV8>::STAGE_BYTES + 2 * MmaGeo<D, G, KV8>::Q_BYTES) + warps * NS * 8;
 }
 
-template <int D, int G, int NS>
+template <int D, int G, int NS, bool KV8 = false>
 __host__ __device__ constexpr int mma_warp_bytes() {
-    return NS * MmaGeo<D, G>::STAGE_BYTES + 2 * MmaGeo<D, G>::Q_BYTES + NS * 8;
+    return NS * MmaGeo<D, G, KV8>::STAGE_BYTES + 2 * MmaGeo<D, G, KV8>::Q_BYTES + NS * 8;
+}
+
+// Two E4M3 codes (low byte first) -> two f16 (exact: every E4M3 value is an f16).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// Two 16-bit query elements of type T -> f16x2 (bf16 -> f16 is exact in f16's
+// normal range, which decode queries stay within).
+template <typename T>
+__device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
+    if constexpr (std::is_same<T, __half>::value) {
+        return w;
+    } else {
+        const float2 f = Elem<T>::pair(w);
+        return Elem<__half>::pack(f.x, f.y);
+    }
 }
 
 template <typename T>
@@ -181,11 +207,12 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
     }
 }
 
-template <int D, int G, typename T, int NS>
+template <int D, int G, typename T, int NS, bool KV8 = false>
 __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
-    using Gm = MmaGeo<D, G>;
+    using Gm = MmaGeo<D, G, KV8>;
+    using MT = typename std::conditional<KV8, __half, T>::type;  // MMA operand type
     extern __shared__ uint8_t smem_raw[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -305,7 +332,7 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
     // Fused append: the unit that holds a sequence's last token writes the new
     // K/V row into the pool and uses it in place of the tile's old contents.
     constexpr int NVR = D / 8;  // 16-byte vectors per row
-    const bool append = p.k_new != nullptr;
+    const bool append = !KV8 && p.k_new != nullptr;  // the fp8 cache has no fused append
 
     for (;;) {
         uint32_t qb[Gm::KS][2];  // B fragments of Q^T: query head g8, 2 columns
@@ -334,9 +361,19 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 const uint8_t *qs = qbuf + cur.slot * Gm::Q_BYTES;
 #pragma unroll
                 for (int i = 0; i < Gm::KS; ++i) {
-                    const int d = 16 * i + 2 * t4;
-                    qb[i][0] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
-                    qb[i][1] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 8) * 2) : 0u;
+                    if constexpr (KV8) {
+                        // Slice i pairs K elements 16i + 4*t4 + {0,1} and + {2,3}
+                        // (the order the byte-wise fragments arrive in); the
+                        // query fragment follows the same order.
+                        const int d = 16 * i + 4 * t4;
+                        qb[i][0] = g8 < G ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2)) : 0u;
+                        qb[i][1] = g8 < G ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 2) * 2))
+                                          : 0u;
+                    } else {
+                        const int d = 16 * i + 2 * t4;
+                        qb[i][0] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
+                        qb[i][1] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 8) * 2) : 0u;
+                    }
                 }
             }
             const int valid = min(16, cur.ntok - 16 * k);
@@ -361,7 +398,24 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
 
             // ---------------- S^T = K . Q^T ------------------------------------
             float s[4] = {0.f, 0.f, 0.f, 0.f};
-            {
+            if constexpr (KV8) {
+                // A 16-byte chunk holds 16 codes of a row; ldmatrix on byte pairs
+                // gives each thread codes 4*t4 .. 4*t4+3 of rows g8 and g8+8.
+                const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+                const int csel = lane >> 4;
+#pragma unroll
+                for (int i = 0; i < Gm::KS; i += 2) {
+                    uint32_t r[4];
+                    ldsm_x4(r, ks_s + swz(row, i + csel));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
+                        const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi), e4m3x2_to_f16x2(lo >> 16),
+                                               e4m3x2_to_f16x2(hi >> 16)};
+                        MmaType<__half>::mma(s, a, qb[i + h][0], qb[i + h][1]);
+                    }
+                }
+            } else {
                 const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
                 const int csel = lane >> 4;
 #pragma unroll
@@ -401,9 +455,9 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             // Padding heads (>= G) carry zero scores; give them weight 0.
             const float p0 = hv0 ? exp2f(x0 - M0) : 0.f, p1 = hv1 ? exp2f(x1 - M1) : 0.f;
             const float p2 = hv0 ? exp2f(x2 - M0) : 0.f, p3 = hv1 ? exp2f(x3 - M1) : 0.f;
-            const uint32_t w_lo = Elem<T>::pack(p0, p1), w_hi = Elem<T>::pack(p2, p3);
+            const uint32_t w_lo = Elem<MT>::pack(p0, p1), w_hi = Elem<MT>::pack(p2, p3);
             {
-                const float2 r_lo = Elem<T>::pair(w_lo), r_hi = Elem<T>::pair(w_hi);
+                const float2 r_lo = Elem<MT>::pair(w_lo), r_hi = Elem<MT>::pair(w_hi);
                 l0 += r_lo.x + r_hi.x;
                 l1 += r_lo.y + r_hi.y;
             }
@@ -423,7 +477,27 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
                 __syncwarp();
             }
-            {
+            if constexpr (KV8) {
+                // Transposed ldmatrix on byte pairs gives each thread, for tokens
+                // 2*t4 and 2*t4+1, the codes of elements 2*g8 and 2*g8+1 of a
+                // 16-element slice; a byte permute regroups them by element, so
+                // accumulator rows g8 / g8+8 hold elements 16i + 2*g8 / + 1.
+                const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+                const int csel = lane >> 4;
+#pragma unroll
+                for (int i = 0; i < Gm::KS; i += 2) {
+                    uint32_t r[4];
+                    ldsm_x4_trans(r, vs_s + swz(row, i + csel));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t x = __byte_perm(r[2 * h], 0, 0x3120);      // tokens 0-7
+                        const uint32_t y = __byte_perm(r[2 * h + 1], 0, 0x3120);  // tokens 8-15
+                        const uint32_t a[4] = {e4m3x2_to_f16x2(x), e4m3x2_to_f16x2(x >> 16), e4m3x2_to_f16x2(y),
+                                               e4m3x2_to_f16x2(y >> 16)};
+                        MmaType<__half>::mma(o[i + h], a, pb0, pb1);
+                    }
+                }
+            } else {
                 const int row = (lane & 7) + 8 * (lane >> 4);
                 const int csel = (lane >> 3) & 1;
 #pragma unroll
@@ -445,7 +519,18 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             l1 += __shfl_xor_sync(FULL_MASK, l1, off);
         }
         const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;
-        if (cur.nparts == 1) {
+        if (KV8 && cur.nparts == 1) {
+            // Accumulator rows g8 / g8+8 of slice i are elements 16i + 2*g8 / + 1:
+            // pairs of adjacent elements per head, stored directly.
+            const float i0 = hv0 ? p.v_scale / l0 : 0.f, i1 = hv1 ? p.v_scale / l1 : 0.f;
+            T *out = static_cast<T *>(p.out) + head0 * D;
+#pragma unroll
+            for (int i = 0; i < Gm::KS; ++i) {
+                const int d = 16 * i + 2 * g8;
+                if (hv0) *reinterpret_cast<uint32_t *>(out + h0 * D + d) = Elem<T>::pack(o[i][0] * i0, o[i][2] * i0);
+                if (hv1) *reinterpret_cast<uint32_t *>(out + h1 * D + d) = Elem<T>::pack(o[i][1] * i1, o[i][3] * i1);
+            }
+        } else if (cur.nparts == 1) {
             const float i0 = hv0 ? 1.f / l0 : 0.f, i1 = hv1 ? 1.f / l1 : 0.f;
             T *out = static_cast<T *>(p.out) + head0 * D;
 #pragma unroll
@@ -462,17 +547,21 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             const size_t group = (size_t)cur.s * Hkv + cur.kvh;
             const size_t row = group * p.max_parts + cur.part;
             float *acc = p.part_acc + row * (size_t)(D * G);
+            // Rows g8 / g8+8 of slice i: elements 16i + g8 / + 8 (16-bit cache)
+            // or 16i + 2*g8 / + 1 (fp8 cache, values scaled by v_scale).
+            const float vs = KV8 ? p.v_scale : 1.f;
 #pragma unroll
             for (int i = 0; i < Gm::KS; ++i) {
-                const int d = 16 * i + g8;
+                const int d = KV8 ? 16 * i + 2 * g8 : 16 * i + g8;
+                const int d2 = KV8 ? d + 1 : d + 8;
                 if constexpr (G == 1) {
                     if (hv0) {
-                        acc[d] = o[i][0];
-                        acc[d + 8] = o[i][2];
+                        acc[d] = o[i][0] * vs;
+                        acc[d2] = o[i][2] * vs;
                     }
                 } else if (hv1) {
-                    *reinterpret_cast<float2 *>(acc + d * G + h0) = make_float2(o[i][0], o[i][1]);
-                    *reinterpret_cast<float2 *>(acc + (d + 8) * G + h0) = make_float2(o[i][2], o[i][3]);
+                    *reinterpret_cast<float2 *>(acc + d * G + h0) = make_float2(o[i][0] * vs, o[i][1] * vs);
+                    *reinterpret_cast<float2 *>(acc + d2 * G + h0) = make_float2(o[i][2] * vs, o[i][3] * vs);
                 }
             }
             if (g8 == 0 && hv0) p.ml[row * G + h0] = make_float2(M0, l0);

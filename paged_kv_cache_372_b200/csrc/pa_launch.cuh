@@ -101,25 +101,24 @@ pa_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled *out) {
 }
 
 // A pool [num_blocks][num_kv_heads][block_size][D] as a 2-D tensor of
-// rows x D elements, read in boxes of 16 rows x 64 columns (128 bytes) with
-// the 128-byte shared-memory swizzle.
-template <typename T>
-pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, int D) {
+// rows x D elements, read in boxes of 16 rows x 128 bytes (64 16-bit or 128
+// 8-bit elements) with the 128-byte shared-memory swizzle.
+pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, int D, int elem_bytes,
+                          CUtensorMapDataType type) {
     PFN_cuTensorMapEncodeTiled enc;
     pa_status st = tensor_map_encoder(&enc);
     if (st != PA_OK) return st;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, 16};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * elem_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), 16};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, pa::MmaType<T>::tma_type, 2, const_cast<void *>(pool), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(map, type, 2, const_cast<void *>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return PA_OK;
 }
 
-template <int D, int G, typename T>
+template <int D, int G, typename T, bool KV8 = false>
 pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     constexpr int NS = pa::DECODE_MMA_STAGES;
     DeviceInfo info;
@@ -128,13 +127,14 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
     if (rows >= (1ll << 31)) return fail(PA_ERR_UNSUPPORTED, "pool has %lld rows, above 2^31", rows);
     CUtensorMap tmk, tmv;
-    if ((st = encode_pool_map<T>(&tmk, p.k_pool, rows, D)) != PA_OK) return st;
-    if ((st = encode_pool_map<T>(&tmv, p.v_pool, rows, D)) != PA_OK) return st;
-    int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS>();
+    const CUtensorMapDataType type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : pa::MmaType<T>::tma_type;
+    if ((st = encode_pool_map(&tmk, p.k_pool, rows, D, KV8 ? 1 : 2, type)) != PA_OK) return st;
+    if ((st = encode_pool_map(&tmv, p.v_pool, rows, D, KV8 ? 1 : 2, type)) != PA_OK) return st;
+    int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS, KV8>();
     if (warps > pa::DECODE_MAX_WARPS) warps = pa::DECODE_MAX_WARPS;
     if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "not enough shared memory for one warp");
-    const int smem = pa::mma_smem_bytes<D, G, NS>(warps);
-    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS>;
+    const int smem = pa::mma_smem_bytes<D, G, NS, KV8>(warps);
+    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS, KV8>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
@@ -154,6 +154,18 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
     return PA_OK;
+}
+
+// fp8 (E4M3) cache: tensor-core kernel, head_dim 128.
+template <typename T>
+pa_status dispatch_group_fp8(pa::DecodeParams &p, int group, cudaStream_t stream) {
+    switch (group) {
+        case 1: return launch_decode_mma<128, 1, T, true>(p, stream);
+        case 2: return launch_decode_mma<128, 2, T, true>(p, stream);
+        case 4: return launch_decode_mma<128, 4, T, true>(p, stream);
+        case 8: return launch_decode_mma<128, 8, T, true>(p, stream);
+    }
+    return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }
 
 template <int D, typename T>
