@@ -120,7 +120,7 @@ pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, in
 
 template <int D, int G, typename T, bool KV8 = false>
 pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
-    constexpr int NS = pa::DECODE_MMA_STAGES;
+    constexpr int NS = KV8 ? pa::DECODE_MMA_STAGES_FP8 : pa::DECODE_MMA_STAGES;
     DeviceInfo info;
     pa_status st = device_info(&info);
     if (st != PA_OK) return st;
