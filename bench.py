@@ -52,9 +52,24 @@ def parse():
                     help="fp8: E4M3 KV cache (pa_reshape_and_cache_fp8 + pa_decode_fp8)")
     ap.add_argument("--unfused", action="store_true",
                     help="separate cache-write launch instead of pa_decode_append")
+    ap.add_argument("--block-size", type=int, default=None,
+                    help="llama7b / llama3_8b at another block size (16, 32 or 64)")
+    ap.add_argument("--head-dim", type=int, default=None,
+                    help="llama7b / llama3_8b at another head size (64 or 128)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
+
+
+def shape_args(args) -> dict:
+    kw = {}
+    if args.block_size is not None:
+        kw["block_size"] = args.block_size
+    if args.head_dim is not None:
+        kw["head_dim"] = args.head_dim
+    if kw and args.workload not in ("llama7b", "llama3_8b"):
+        raise SystemExit("--block-size / --head-dim apply to llama7b and llama3_8b")
+    return kw
 
 
 def describe(wl) -> dict:
@@ -211,7 +226,7 @@ def run_ours(args, world, rank, local):
     from paged_kv_cache_372_b200 import build, workloads
     build.build()
     dev = torch.device("cuda", local if world > 1 else 0)
-    wl = workloads.build(args.workload, args.seed + rank)
+    wl = workloads.build(args.workload, args.seed + rank, **shape_args(args))
     st0 = wl.steps[0]
     B = int(len(st0.context_lens))
     kp, vp = wl.k_pool.to(dev), wl.v_pool.to(dev)
@@ -305,7 +320,17 @@ def run_ours(args, world, rank, local):
     barrier(world)
     clk = clocks.stop() if clocks else None
     total_ms = (sum(a.elapsed_time(b) for a, b in step_evs) if flush else start.elapsed_time(stop))
-    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    dec = np.array([a.elapsed_time(b) for a, b in evs])
+    decode_ms = float(dec.mean())
+    unflushed = None
+    if flush:
+        # The same steps with the blocks of the previous step left in L2.
+        m = min(args.steps, 200)
+        for i in range(m):
+            step(i, evs[i])
+        torch.cuda.synchronize(dev)
+        u = float(np.mean([a.elapsed_time(b) for a, b in evs[:m]]))
+        unflushed = {"steps": m, "decode_ms": u}
     total_ms = max_over_ranks(total_ms, world)
     decode_ms_max = max_over_ranks(decode_ms, world)
     ms_per_step = total_ms / args.steps
@@ -326,6 +351,7 @@ def run_ours(args, world, rank, local):
         "config": describe(wl),
         "kv_gbs": kv_unique * world / (ms_per_step * 1e-3) / 1e9,
         "decode_ms": decode_ms_max,
+        "decode_ms_p10_p50_p90": [float(x) for x in np.percentile(dec, [10, 50, 90])],
         "decode_kv_gbs": achieved,
         "decode_kv_gbs_logical": kv_bytes / (decode_ms * 1e-3) / 1e9,
         "hbm_frac_of_%s" % peak_kind: achieved / peak,
@@ -337,14 +363,18 @@ def run_ours(args, world, rank, local):
                                 "merge fused)" if fused else
                                 "pa_decode call (plan + attention launches; split merge fused)"),
                      "bytes": "unique K+V bytes of valid tokens per call",
-                     "traffic": profiled_traffic(wl.name if args.partition is None
-                                                 else f"{wl.name}@P{args.partition}")},
+                     "traffic": profiled_traffic(wl.name + ("@fp8" if kv8 else "")
+                                                 + ("" if args.partition is None else f"@P{args.partition}"))},
         "gpu_launches": launches,
         "step": ("pa_copy_blocks (if any), pa_reshape_and_cache_fp8, pa_decode_fp8" if kv8 else
                  "pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_append"
                  if fused else "pa_copy_blocks (if any), pa_reshape_and_cache, pa_decode"),
         "clocks": clk,
     }
+    if unflushed is not None:
+        unflushed["decode_kv_gbs"] = kv_unique / (unflushed["decode_ms"] * 1e-3) / 1e9
+        unflushed["decode_kv_gbs_logical"] = kv_bytes / (unflushed["decode_ms"] * 1e-3) / 1e9
+        result["unflushed"] = unflushed
     if kv8:
         result["config"]["kv_cache"] = f"E4M3 codes, k_scale = v_scale = {FP8_SCALE}"
         result["config"]["kv_bytes_per_step"] = int(kv_bytes)
@@ -501,7 +531,7 @@ def run_reference(args, world, rank):
     (8 sequences) of the same workload."""
     import oracle
     from paged_kv_cache_372_b200 import workloads
-    wl = workloads.build(args.workload, args.seed)
+    wl = workloads.build(args.workload, args.seed, **shape_args(args))
     B = int(len(wl.steps[0].context_lens))
     n = min(B, 8)
     s = oracle_sample(wl, n)

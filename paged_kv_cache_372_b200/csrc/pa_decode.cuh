@@ -248,12 +248,17 @@ __host__ __device__ constexpr int warp_smem_bytes() {
 #endif
 // Stages of the fp8-cache ring (its stages are half the bytes of a 16-bit one).
 #ifndef PA_DECODE_MMA_STAGES_FP8
-#define PA_DECODE_MMA_STAGES_FP8 4
+#define PA_DECODE_MMA_STAGES_FP8 2
+#endif
+// Warps per CTA of the fp8-cache kernel for small head groups.
+#ifndef PA_DECODE_MAX_WARPS_FP8
+#define PA_DECODE_MAX_WARPS_FP8 16
 #endif
 constexpr int DECODE_STAGES = PA_DECODE_STAGES;
 constexpr int DECODE_MAX_WARPS = PA_DECODE_MAX_WARPS;
 constexpr int DECODE_MMA_STAGES = PA_DECODE_MMA_STAGES;
 constexpr int DECODE_MMA_STAGES_FP8 = PA_DECODE_MMA_STAGES_FP8;
+constexpr int DECODE_MAX_WARPS_FP8 = PA_DECODE_MAX_WARPS_FP8;
 constexpr int DECODE_TENSOR_MIN_GROUP = PA_DECODE_TENSOR_MIN_GROUP;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
 // The running maximum of a head is only raised when a score exceeds it by more

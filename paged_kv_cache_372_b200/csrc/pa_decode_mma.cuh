@@ -52,10 +52,31 @@ __host__ __device__ constexpr int mma_warp_bytes() {
     return NS * MmaGeo<D, G, KV8>::STAGE_BYTES + 2 * MmaGeo<D, G, KV8>::Q_BYTES + NS * 8;
 }
 
-// Two E4M3 codes (low byte first) -> two f16 (exact: every E4M3 value is an f16).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Warps per CTA: the fp8 kernel runs DECODE_MAX_WARPS_FP8 warps for small head
+// groups (up to 4 query heads per KV head, where it fits 128 registers a
+// thread), DECODE_MAX_WARPS otherwise.
+#ifndef PA_FP8_WIDE_MAX_GROUP
+#define PA_FP8_WIDE_MAX_GROUP 4
+#endif
+template <int G, bool KV8>
+__host__ __device__ constexpr int mma_max_warps() {
+    return KV8 && G <= PA_FP8_WIDE_MAX_GROUP ? DECODE_MAX_WARPS_FP8 : DECODE_MAX_WARPS;
+}
+
+// E4M3 -> f16 widening: every E4M3 value is exactly an f16. One cvt converts
+// the two codes of one 16-bit half of a register; taking the half through a
+// register split (rather than a shift) keeps it to one instruction.
+// Codes in bytes 0 and 1 (low byte first) -> two f16.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes) {
+    uint32_t r;
+    asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}" : "=r"(r) : "r"(codes));
+    return r;
+}
+// Codes in bytes 2 and 3 -> two f16.
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t codes) {
+    uint32_t r;
+    asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.rn.f16x2.e4m3x2 %0, hi;\n}" : "=r"(r) : "r"(codes));
+    return r;
 }
 
 // Two 16-bit query elements of type T -> f16x2 (bf16 -> f16 is exact in f16's
@@ -208,7 +229,7 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
 }
 
 template <int D, int G, typename T, int NS, bool KV8 = false>
-__global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
+__global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
     using Gm = MmaGeo<D, G, KV8>;
@@ -397,7 +418,8 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
             }
 
             // ---------------- S^T = K . Q^T ------------------------------------
-            float s[4] = {0.f, 0.f, 0.f, 0.f};
+            // Two accumulators (even / odd slices) halve the chain of dependent MMAs.
+            float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
             if constexpr (KV8) {
                 // A 16-byte chunk holds 16 codes of a row; ldmatrix on byte pairs
                 // gives each thread codes 4*t4 .. 4*t4+3 of rows g8 and g8+8.
@@ -410,9 +432,9 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
-                        const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi), e4m3x2_to_f16x2(lo >> 16),
-                                               e4m3x2_to_f16x2(hi >> 16)};
-                        MmaType<__half>::mma(s, a, qb[i + h][0], qb[i + h][1]);
+                        const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi), e4m3x2_hi_to_f16x2(lo),
+                                               e4m3x2_hi_to_f16x2(hi)};
+                        MmaType<__half>::mma(h ? s2 : s, a, qb[i + h][0], qb[i + h][1]);
                     }
                 }
             } else {
@@ -422,9 +444,11 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                 for (int i = 0; i < Gm::KS; ++i) {
                     uint32_t a[4];
                     ldsm_x4(a, ks_s + swz(row, 2 * i + csel));
-                    MmaType<T>::mma(s, a, qb[i][0], qb[i][1]);
+                    MmaType<T>::mma((i & 1) ? s2 : s, a, qb[i][0], qb[i][1]);
                 }
             }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s[j] += s2[j];
             // s[0], s[1]: token g8, heads h0, h1; s[2], s[3]: token g8 + 8.
             const bool v_lo = g8 < valid, v_hi = g8 + 8 < valid;
             float x0 = v_lo ? s[0] * p.qscale : -INFINITY;
@@ -492,8 +516,8 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1)
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t x = __byte_perm(r[2 * h], 0, 0x3120);      // tokens 0-7
                         const uint32_t y = __byte_perm(r[2 * h + 1], 0, 0x3120);  // tokens 8-15
-                        const uint32_t a[4] = {e4m3x2_to_f16x2(x), e4m3x2_to_f16x2(x >> 16), e4m3x2_to_f16x2(y),
-                                               e4m3x2_to_f16x2(y >> 16)};
+                        const uint32_t a[4] = {e4m3x2_to_f16x2(x), e4m3x2_hi_to_f16x2(x), e4m3x2_to_f16x2(y),
+                                               e4m3x2_hi_to_f16x2(y)};
                         MmaType<__half>::mma(o[i + h], a, pb0, pb1);
                     }
                 }

@@ -167,19 +167,24 @@ def tiny(seed: int = 0) -> Workload:
     return wl
 
 
-def llama7b(seed: int = 0, num_seqs: int = 64) -> Workload:
+def _shape_name(base: str, block_size: int, head_dim: int) -> str:
+    """Name of a workload run at a block size / head size other than its own."""
+    return base if (block_size, head_dim) == (16, 128) else f"{base}_bs{block_size}_d{head_dim}"
+
+
+def llama7b(seed: int = 0, num_seqs: int = 64, block_size: int = 16, head_dim: int = 128) -> Workload:
     gen = inputs.generator(seed + 2000)
     ctx = inputs.uniform_int(128, 2048, num_seqs, gen)
-    wl, _ = _decode_batch("llama7b", ctx, heads=32, kv_heads=32, head_dim=128, block_size=16,
-                          dtype="f16", seed=seed + 2001)
+    wl, _ = _decode_batch(_shape_name("llama7b", block_size, head_dim), ctx, heads=32, kv_heads=32,
+                          head_dim=head_dim, block_size=block_size, dtype="f16", seed=seed + 2001)
     return wl
 
 
-def llama3_8b(seed: int = 0, num_seqs: int = 256) -> Workload:
+def llama3_8b(seed: int = 0, num_seqs: int = 256, block_size: int = 16, head_dim: int = 128) -> Workload:
     gen = inputs.generator(seed + 3000)
     ctx = inputs.lognormal_int(512.0, 1.0, 16, 8192, num_seqs, gen)
-    wl, _ = _decode_batch("llama3_8b", ctx, heads=32, kv_heads=8, head_dim=128, block_size=16,
-                          dtype="bf16", seed=seed + 3001)
+    wl, _ = _decode_batch(_shape_name("llama3_8b", block_size, head_dim), ctx, heads=32, kv_heads=8,
+                          head_dim=head_dim, block_size=block_size, dtype="bf16", seed=seed + 3001)
     return wl
 
 
