@@ -52,6 +52,9 @@ def parse():
                     help="fp8: E4M3 KV cache (pa_reshape_and_cache_fp8 + pa_decode_fp8)")
     ap.add_argument("--unfused", action="store_true",
                     help="separate cache-write launch instead of pa_decode_append")
+    ap.add_argument("--share", default="auto", choices=["auto", "on", "off"],
+                    help="pa_decode_shared (blocks shared by several sequences streamed once per group); "
+                         "auto: on when the workload's tables share blocks")
     ap.add_argument("--block-size", type=int, default=None,
                     help="llama7b / llama3_8b at another block size (16, 32 or 64)")
     ap.add_argument("--head-dim", type=int, default=None,
@@ -248,6 +251,10 @@ def run_ours(args, world, rank, local):
 
     kv8 = args.kv == "fp8"
     fused = not args.unfused and not kv8 and appends_at_last_positions(wl)
+    share = not kv8 and (args.share == "on" or (args.share == "auto" and wl.kv_bytes_unique() < wl.kv_bytes()))
+    if share:
+        ws = pa.alloc_workspace(B, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, max_ctx, P, dev,
+                                shared=True)
     if kv8:
         # The whole cache quantised once by the library's own E4M3 cache write.
         NB, Hkv, bs, D = kp.shape
@@ -284,6 +291,9 @@ def run_ours(args, world, rank, local):
         if kv8:
             pa.pa_decode_fp8(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, FP8_SCALE,
                              FP8_SCALE, P, ws)
+        elif share:
+            kw = dict(k_new=d["k_dec"], v_new=d["v_dec"]) if fused else {}
+            pa.pa_decode_shared(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws, **kw)
         elif fused:
             pa.pa_decode_append(d["out"], d["q"], d["k_dec"], d["v_dec"], kp, vp, d["tables"], d["ctx"], wl.scale,
                                 max_ctx, P, ws)
@@ -359,6 +369,10 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "kernel": ("pa_decode_fp8 call (plan + attention launches; split merge fused)" if kv8 else
+                                "pa_decode_shared call (grouping plan + attention launches; cache write and "
+                                "split merge fused)" if share and fused else
+                                "pa_decode_shared call (grouping plan + attention launches; split merge fused)"
+                                if share else
                                 "pa_decode_append call (plan + attention launches; cache write and split "
                                 "merge fused)" if fused else
                                 "pa_decode call (plan + attention launches; split merge fused)"),
@@ -367,10 +381,14 @@ def run_ours(args, world, rank, local):
                                                  + ("" if args.partition is None else f"@P{args.partition}"))},
         "gpu_launches": launches,
         "step": ("pa_copy_blocks (if any), pa_reshape_and_cache_fp8, pa_decode_fp8" if kv8 else
+                 "pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_shared with "
+                 "the new tokens" if share and fused else
+                 "pa_copy_blocks (if any), pa_reshape_and_cache, pa_decode_shared" if share else
                  "pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_append"
                  if fused else "pa_copy_blocks (if any), pa_reshape_and_cache, pa_decode"),
         "clocks": clk,
     }
+    result["config"]["shared_prefix_units"] = bool(share)
     if unflushed is not None:
         unflushed["decode_kv_gbs"] = kv_unique / (unflushed["decode_ms"] * 1e-3) / 1e9
         unflushed["decode_kv_gbs_logical"] = kv_bytes / (unflushed["decode_ms"] * 1e-3) / 1e9
@@ -379,7 +397,7 @@ def run_ours(args, world, rank, local):
         result["config"]["kv_cache"] = f"E4M3 codes, k_scale = v_scale = {FP8_SCALE}"
         result["config"]["kv_bytes_per_step"] = int(kv_bytes)
     if not args.no_e2e and not kv8:
-        e2e = run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused)
+        e2e = run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused, share)
         if rank == 0:
             result["e2e"] = e2e
     pa.pa_device_errors()
@@ -388,7 +406,7 @@ def run_ours(args, world, rank, local):
     return result
 
 
-def run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused):
+def run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused, share=False):
     """Same metric through the public API with host buffers: every step copies its
     inputs from pinned host memory and reads the output back."""
     nsteps = len(wl.steps)
@@ -411,7 +429,16 @@ def run_e2e(args, wl, pa, kp, vp, ws, P, max_ctx, dev, world, fused):
         if d["pairs"].shape[0]:
             pa.pa_copy_blocks([kp, vp], d["pairs"])
         out = torch.empty_like(d["q"])
-        if fused:
+        if share:
+            kw = {}
+            if fused:
+                if d["slots"].shape[0] > B:
+                    pa.pa_reshape_and_cache(d["k"][B:], d["v"][B:], kp, vp, d["slots"][B:])
+                kw = dict(k_new=d["k"][:B], v_new=d["v"][:B])
+            else:
+                pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
+            pa.pa_decode_shared(out, d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws, **kw)
+        elif fused:
             if d["slots"].shape[0] > B:
                 pa.pa_reshape_and_cache(d["k"][B:], d["v"][B:], kp, vp, d["slots"][B:])
             pa.pa_decode_append(out, d["q"], d["k"][:B], d["v"][:B], kp, vp, d["tables"], d["ctx"], wl.scale,

@@ -150,6 +150,48 @@ PA_API pa_status pa_decode_append(void *out, const void *q, const void *k_new, c
                                   size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * Paged decode attention that computes over shared blocks once per group of
+ * sequences. Same result as pa_decode (k_new = v_new = NULL) or
+ * pa_decode_append (both set) up to the order of fp32 rounding: the
+ * arithmetic is the definition of pa_decode, with the sum over tokens
+ * regrouped by partition.
+ *
+ * Sequences forked from one another (beam search, parallel sampling) hold
+ * the same physical blocks at the start of their block tables ("vLLM架构深度
+ * 解析：PagedAttention如何实现高吞吐LLM推理", section KV Cache内存共享; "别再让
+ * GPU内存拖后腿了", section 2.2). The library finds them on the device: it
+ * sorts the sequences by their first block and, within a run of sequences
+ * with the same first block, forms groups of up to 8 / (num_heads /
+ * num_kv_heads) consecutive ones. A group's shared part is the leading full
+ * blocks that all members have in common with its first member (with k_new,
+ * only blocks below the one holding each member's last position). That part
+ * is streamed once per KV head for the whole group, with the group's queries
+ * side by side in one tensor-core tile. Each member's remaining tokens run
+ * as ordinary partitions, and the partitions merge by the log-sum-exp
+ * identity. Without shared blocks, the result and the work are those of
+ * pa_decode.
+ *
+ * Requirements beyond pa_decode's: num_seqs <= 1024, fp16/bf16 cache
+ * (the tensor-core kernel). workspace: at least
+ * pa_decode_shared_workspace_size(...) bytes (one more partition per
+ * sequence than pa_decode, plus the grouping). Errors: PA_ERR_UNSUPPORTED
+ * for num_seqs > 1024 or a build without the tensor-core kernel for this
+ * head group; otherwise as pa_decode / pa_decode_append.
+ */
+PA_API pa_status pa_decode_shared(void *out, const void *q, const void *k_new, const void *v_new,
+                                  void *k_pool, void *v_pool, const int32_t *block_tables,
+                                  const int32_t *context_lens, int num_seqs, int num_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int num_blocks, int max_context_len,
+                                  float scale, int dtype, int partition_size, void *workspace,
+                                  size_t workspace_bytes, pa_stream_t stream);
+
+/* Workspace bytes pa_decode_shared needs (0 for unsupported shapes). */
+PA_API size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                              int head_dim, int block_size, int max_context_len,
+                                              int partition_size);
+
+/*
  * Paged decode attention over an 8-bit E4M3 ("fp8 e4m3fn") KV cache with
  * per-tensor scales: key element = k_scale * E4M3 code, value element =
  * v_scale * E4M3 code; otherwise exactly pa_decode (q and out stay fp16/bf16

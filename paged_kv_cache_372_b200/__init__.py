@@ -54,6 +54,11 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_append.restype = _I
         L.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                        _I, _P, _SZ, _P]
+        L.pa_decode_shared.restype = _I
+        L.pa_decode_shared.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                                       _I, _P, _SZ, _P]
+        L.pa_decode_shared_workspace_size.restype = _SZ
+        L.pa_decode_shared_workspace_size.argtypes = [_I] * 7
         L.pa_decode_fp8.restype = _I
         L.pa_decode_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _F, _F, _I,
                                     _P, _SZ, _P]
@@ -128,10 +133,21 @@ def pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_
     return n
 
 
+def pa_decode_shared_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                                    partition_size=0) -> int:
+    n = int(lib().pa_decode_shared_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                  max_context_len, partition_size))
+    if n == 0:
+        raise PagedAttentionError(PA_ERR_INVALID, "unsupported shape or partition size")
+    return n
+
+
 def alloc_workspace(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
-                    partition_size=0, device=None) -> torch.Tensor:
-    n = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                                 max_context_len, partition_size)
+                    partition_size=0, device=None, shared=False) -> torch.Tensor:
+    """Workspace for pa_decode / pa_decode_append / pa_decode_fp8, or with
+    shared=True for pa_decode_shared."""
+    size = pa_decode_shared_workspace_size if shared else pa_decode_workspace_size
+    n = size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size)
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
@@ -180,6 +196,37 @@ def pa_decode_append(out, q, k_new, v_new, k_pool, v_pool, block_tables, context
         _cuda(context_lens, "context_lens", torch.int32), B, H, Hkv, D, bs, block_tables.shape[1], NB,
         int(max_context_len), float(scale), _DTYPES[q.dtype], int(partition_size), _cuda(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def pa_decode_shared(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len,
+                     partition_size=0, workspace=None, stream=None, k_new=None, v_new=None) -> torch.Tensor:
+    """pa_decode (or, with k_new/v_new, pa_decode_append) that streams blocks
+    shared by the leading parts of several sequences' tables once per group."""
+    B, H, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch between q, out and the pools")
+    if q.dtype not in _DTYPES or k_pool.dtype != q.dtype or v_pool.dtype != q.dtype or out.dtype != q.dtype:
+        raise ValueError("q, out and the pools must share one dtype, fp16 or bf16")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None:
+        if tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D):
+            raise ValueError("k_new and v_new must be [B][Hkv][D]")
+        if k_new.dtype != q.dtype or v_new.dtype != q.dtype:
+            raise ValueError("k_new and v_new must have q's dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("block_tables must be [B][W] and context_lens [B]")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device, shared=True)
+    _check(lib().pa_decode_shared(
+        _cuda(out, "out"), _cuda(q, "q"), None if k_new is None else _cuda(k_new, "k_new"),
+        None if v_new is None else _cuda(v_new, "v_new"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
+        B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
+        int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
     return out
 
 

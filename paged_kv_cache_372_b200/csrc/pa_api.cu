@@ -119,6 +119,15 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
     return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts).total;
 }
 
+size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                       int max_context_len, int partition_size) {
+    const int P = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                           max_context_len, partition_size);
+    if (P == 0) return 0;
+    const int max_parts = (max_context_len > 0 ? ceil_div(max_context_len, P) : 1) + 1;
+    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts, true).total;
+}
+
 }  // extern "C"
 
 namespace {
@@ -128,8 +137,11 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
                       int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
                       int num_blocks, int max_context_len, float scale, int dtype, int partition_size,
                       void *workspace, size_t workspace_bytes, pa_stream_t stream, bool kv8 = false,
-                      float k_scale = 1.f, float v_scale = 1.f) {
+                      float k_scale = 1.f, float v_scale = 1.f, bool shared = false) {
     g_last_error.clear();
+    if (shared && num_seqs > pa::SHARE_MAX_SEQS)
+        return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode takes at most %d sequences, got %d", pa::SHARE_MAX_SEQS,
+                    num_seqs);
     if (kv8 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "fp8 cache supports head_dim 128, got %d", head_dim);
     if (kv8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || k_scale == INFINITY || v_scale == INFINITY))
         return fail(PA_ERR_INVALID, "k_scale and v_scale must be positive and finite");
@@ -152,10 +164,12 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
                     partition_size, partition_cap(block_size));
     const long long table_tokens = (long long)max_blocks_per_seq * block_size;
     const int ctx_limit = (int)(table_tokens < max_context_len ? table_tokens : max_context_len);
-    const int max_parts = max_context_len > 0 ? ceil_div(max_context_len, P) : 1;
+    // With shared prefixes a sequence's partitions are cut at the end of its
+    // shared blocks too, so it can have one more.
+    const int max_parts = (max_context_len > 0 ? ceil_div(max_context_len, P) : 1) + (shared ? 1 : 0);
     if ((long long)num_seqs * max_parts * num_kv_heads >= (1ll << 31))
         return fail(PA_ERR_UNSUPPORTED, "too many work units");
-    const pa::WsLayout L = pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts);
+    const pa::WsLayout L = pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts, shared);
     if (workspace_bytes < L.total)
         return fail(PA_ERR_INVALID, "workspace %zu bytes < %zu needed", workspace_bytes, L.total);
 
@@ -190,11 +204,22 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     p.ml = reinterpret_cast<float2 *>(ws + L.ml);
     p.part_acc = reinterpret_cast<float *>(ws + L.acc);
     p.merge_count = reinterpret_cast<int *>(ws + L.count);
+    p.entries_b = shared ? reinterpret_cast<int4 *>(ws + L.entries_b) : nullptr;
+    p.members = shared ? reinterpret_cast<int *>(ws + L.members) : nullptr;
+    p.member_nparts = shared ? reinterpret_cast<int *>(ws + L.member_nparts) : nullptr;
+    p.append_guard = k_new != nullptr;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int group = num_heads / num_kv_heads;
     if (kv8)
         return dtype == PA_F16 ? dispatch_group_fp8<__half>(p, group, s) : dispatch_group_fp8<__nv_bfloat16>(p, group, s);
+    if (shared) {
+        if (head_dim == 128)
+            return dtype == PA_F16 ? dispatch_group_shared<128, __half>(p, group, s)
+                                   : dispatch_group_shared<128, __nv_bfloat16>(p, group, s);
+        return dtype == PA_F16 ? dispatch_group_shared<64, __half>(p, group, s)
+                               : dispatch_group_shared<64, __nv_bfloat16>(p, group, s);
+    }
     if (head_dim == 128)
         return dtype == PA_F16 ? dispatch_group<128, __half>(p, group, s)
                                : dispatch_group<128, __nv_bfloat16>(p, group, s);
@@ -236,6 +261,20 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
     return decode_impl(out, q, k_new, v_new, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
                        num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
                        dtype, partition_size, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_shared(void *out, const void *q, const void *k_new, const void *v_new, void *k_pool,
+                           void *v_pool, const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                           int num_blocks, int max_context_len, float scale, int dtype, int partition_size,
+                           void *workspace, size_t workspace_bytes, pa_stream_t stream) {
+    if ((k_new == nullptr) != (v_new == nullptr)) {
+        g_last_error = "k_new and v_new must both be null or both be set";
+        return PA_ERR_INVALID;
+    }
+    return decode_impl(out, q, k_new, v_new, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream, false, 1.f, 1.f, true);
 }
 
 pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void *v_pool, const int64_t *slot_mapping,

@@ -12,6 +12,31 @@
 
 namespace pa {
 
+// Release / acquire fence at GPU scope (cheaper than a sequentially
+// consistent one).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Counts one finished partition of a partitioned result and reports whether
+// it was the last of `total`. The warp's lanes have stored their partial
+// results; the warp barrier orders those stores before the counting lane's
+// release fence (fences are cumulative), whose relaxed atomic then publishes
+// them at GPU scope. The lane that completes the count takes the acquire
+// fence after its atomic, and the second warp barrier extends that to the
+// other lanes, which then read every partition's partials. This is the
+// fence + relaxed atomic release / acquire pattern of the PTX memory model.
+__device__ __forceinline__ bool count_partition(int *counter, int total, bool counting_lane) {
+    __syncwarp();
+    bool last = false;
+    if (counting_lane) {
+        fence_acq_rel_gpu();
+        last = atomicAdd(counter, 1) == total - 1;
+        if (last) fence_acq_rel_gpu();
+    }
+    __syncwarp();
+    return last;
+}
+
+
 constexpr unsigned FULL_MASK = 0xffffffffu;
 
 // Per-device error word. Kernels OR PA_DEVERR_* bits into it instead of

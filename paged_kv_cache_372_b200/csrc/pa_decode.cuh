@@ -52,22 +52,37 @@ struct DecodeParams {
     float2 *ml;      // [seq][head][part] (max in log2 units, sum of weights)
     float *part_acc; // [seq][head][part][D] unnormalised outputs
     int *merge_count;// [seq][kv head] finished partitions
+    // Shared-prefix units (pa_decode_shared): a unit may serve several
+    // sequences whose block tables begin with the same blocks.
+    int4 *entries_b; // {first token, member offset, member count (0: one sequence), 0}
+    int *members;    // sequences in grouping order
+    int *member_nparts;  // partitions of members[i]
+    int append_guard;    // 1: a sequence's last position never lies in a shared block
 };
 
 // Workspace layout: header (counter, entry count), work list, partials.
 struct WsLayout {
-    size_t entries, ml, acc, count, total;
+    size_t entries, ml, acc, count, entries_b, members, member_nparts, total;
 };
 
 inline __host__ __device__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline __host__ __device__ WsLayout ws_layout(int B, int H, int Hkv, int D, int max_parts) {
+inline __host__ __device__ WsLayout ws_layout(int B, int H, int Hkv, int D, int max_parts, bool shared = false) {
     WsLayout L;
     size_t off = 256;
     L.entries = off;
     off = align256(off + sizeof(int4) * (size_t)B * max_parts);
     L.count = off;
     off = align256(off + sizeof(int) * (size_t)B * Hkv);
+    L.entries_b = L.members = L.member_nparts = 0;
+    if (shared) {
+        L.entries_b = off;
+        off = align256(off + sizeof(int4) * (size_t)B * max_parts);
+        L.members = off;
+        off = align256(off + sizeof(int) * (size_t)B);
+        L.member_nparts = off;
+        off = align256(off + sizeof(int) * (size_t)B);
+    }
     const size_t parts = max_parts > 1 ? (size_t)max_parts : 0;  // no partials without a split
     L.ml = off;
     off = align256(off + sizeof(float2) * (size_t)B * H * parts);
@@ -158,6 +173,237 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
             const int nvec = p.num_heads * p.head_dim / 8;
             uint4 *row = static_cast<uint4 *>(p.out) + (size_t)s * nvec;
             for (int i = 0; i < nvec; ++i) row[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+// ---- 1b. work list with shared-prefix units ------------------------------------
+// Sequences forked from one another (beam search, parallel sampling) hold the
+// same physical blocks at the start of their tables ("vLLM架构深度解析：
+// PagedAttention如何实现高吞吐LLM推理", section KV Cache内存共享). Their
+// attention over those blocks is the same product with different queries, so
+// one unit can stream the shared tiles once for up to 8 / G sequences: their
+// G query rows each fill the 8 columns of the MMA tile. Each member's own
+// blocks run as ordinary units, and the partitions merge by the usual
+// log-sum-exp identity (the definition's sum over all tokens, regrouped).
+//
+// Grouping: sequences are sorted by their first block; within a run of equal
+// first blocks, consecutive members form sub-groups of up to 8 / G. A
+// sub-group shares the leading full blocks that every member has in common
+// with its first member (a block is shared only below each member's context;
+// with append_guard, only below the block of the member's last position, so
+// the row a fused append writes is never in a shared unit). The shared tokens
+// are cut into partitions 0 .. pp-1 written for every member, the rest of each
+// member into pp, pp+1, ...
+constexpr int SHARE_MAX_SEQS = PLAN_THREADS;  // one sequence per plan thread
+constexpr int NO_SHARE = 0x7fffffff;
+
+__device__ __forceinline__ int shared_full_blocks(const DecodeParams &p, int ctx) {
+    const int pos = p.append_guard ? ctx - 1 : ctx;
+    return pos > 0 ? pos / p.block_size : 0;
+}
+
+__global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const DecodeParams p) {
+    __shared__ unsigned long long s_key[SHARE_MAX_SEQS];  // (first block << 32) | sequence, sorted
+    __shared__ int s_ctx[SHARE_MAX_SEQS];                 // clamped context of each sequence
+    __shared__ int s_grp[SHARE_MAX_SEQS];                 // sub-group of a position: first | count << 16
+    __shared__ int s_lcp[SHARE_MAX_SEQS];                 // leading blocks shared with the sub-group's first
+    __shared__ int s_bin_count[PLAN_MAX_BINS];
+    __shared__ int s_bin_next[PLAN_MAX_BINS];
+    __shared__ int s_warp[32];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int B = p.num_seqs, P = p.partition, tiles = P / 16, bs = p.block_size, W = p.max_blocks_per_seq;
+    const int cap = 8 / (p.num_heads / p.num_kv_heads);  // sequences per shared unit
+    int n = 1;
+    while (n < B) n <<= 1;
+    for (int i = tid; i < PLAN_MAX_BINS; i += PLAN_THREADS) s_bin_count[i] = 0;
+    for (int i = tid; i < B * p.num_kv_heads; i += PLAN_THREADS) p.merge_count[i] = 0;
+
+    // Key of this thread's sequence; padding keys sort last.
+    unsigned long long key = ~0ull;
+    if (tid < B) {
+        const int first = p.block_tables[(size_t)tid * W];  // loaded alongside the context
+        const int ctx = clamped_context(p, tid, true);
+        s_ctx[tid] = ctx;
+        const int b0 = shared_full_blocks(p, ctx) > 0 && first >= 0 && first < p.num_blocks ? first : NO_SHARE;
+        key = ((unsigned long long)(unsigned)b0 << 32) | (unsigned)tid;
+    }
+    // Bitonic sort, one key per thread: strides below 32 by shuffles within
+    // the warp, larger ones through shared memory.
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            unsigned long long other;
+            if (j >= 32) {
+                __syncthreads();
+                if (tid < n) s_key[tid] = key;
+                __syncthreads();
+                other = tid < n ? s_key[tid ^ j] : key;
+            } else {
+                other = __shfl_xor_sync(FULL_MASK, key, j);
+            }
+            const bool up = (tid & k) == 0, lower = (tid & j) == 0;
+            if (tid < n) key = (lower == up) ? (key < other ? key : other) : (key < other ? other : key);
+        }
+    }
+    __syncthreads();
+    if (tid < n) s_key[tid] = key;
+    __syncthreads();
+    // Run of equal first blocks around this position, and its sub-group.
+    if (tid < B) {
+        const unsigned b0 = (unsigned)(key >> 32);
+        int lead = tid, cnt = 1;
+        if (b0 != (unsigned)NO_SHARE) {
+            int lo = 0, hi = tid;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if ((unsigned)(s_key[mid] >> 32) < b0) lo = mid + 1; else hi = mid;
+            }
+            const int start = lo;
+            lo = tid + 1;
+            hi = B;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if ((unsigned)(s_key[mid] >> 32) <= b0) lo = mid + 1; else hi = mid;
+            }
+            lead = start + (tid - start) / cap * cap;
+            cnt = min(cap, lo - lead);
+        }
+        s_grp[tid] = lead | (cnt << 16);
+    }
+    __syncthreads();
+    // Leading blocks each position shares with its sub-group's first member:
+    // one warp per position, two positions per round (positions i and i + 32
+    // of a warp's stripe), 2 x 32 table entries of each row per load batch,
+    // so that B <= 64 costs one dependent round trip.
+    for (int i0 = warp; i0 < B; i0 += 2 * (PLAN_THREADS / 32)) {
+        int lcp[2], lim[2];
+        const int *tm[2], *tl[2];
+        bool todo[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int i = i0 + h * (PLAN_THREADS / 32);
+            const int ii = i < B ? i : i0;
+            const int lead = s_grp[ii] & 0xffff;
+            const int m = (int)(s_key[ii] & 0xffffffffu), l = (int)(s_key[lead] & 0xffffffffu);
+            const int nm = shared_full_blocks(p, s_ctx[m]);
+            todo[h] = i < B && ii != lead;
+            lim[h] = todo[h] ? min(nm, shared_full_blocks(p, s_ctx[l])) : 0;
+            lcp[h] = todo[h] ? lim[h] : nm;
+            tm[h] = p.block_tables + (size_t)m * W;
+            tl[h] = p.block_tables + (size_t)l * W;
+        }
+        for (int j0 = 0; j0 < max(lim[0], lim[1]); j0 += 64) {
+            int a[2][2], b[2][2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int j = j0 + 32 * r + lane;
+                    const bool in = j < lim[h] && lcp[h] == lim[h];
+                    a[h][r] = in ? tm[h][j] : 0;
+                    b[h][r] = in ? tl[h][j] : 0;
+                }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (lcp[h] != lim[h] || !todo[h]) continue;  // decided (uniform across the warp)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const unsigned d = __ballot_sync(FULL_MASK, a[h][r] != b[h][r]);
+                    if (d && lcp[h] == lim[h]) lcp[h] = j0 + 32 * r + __ffs(d) - 1;
+                }
+            }
+            if ((lcp[0] != lim[0] || !todo[0]) && (lcp[1] != lim[1] || !todo[1])) break;
+        }
+        if (lane == 0) {
+            s_lcp[i0] = lcp[0];
+            if (i0 + PLAN_THREADS / 32 < B) s_lcp[i0 + PLAN_THREADS / 32] = lcp[1];
+        }
+    }
+    __syncthreads();
+
+    // Per position: shared tokens S of its sub-group, its partitions, and
+    // (at a sub-group's first position) the shared partitions.
+    int m = 0, ctx = 0, S = 0, pp = 0, sfull = 0, stail = 0, nparts = 0, pfull = 0, ptail = 0, cnt = 1;
+    if (tid < B) {
+        const int lead = s_grp[tid] & 0xffff;
+        cnt = s_grp[tid] >> 16;
+        int sh = 0;
+        if (cnt >= 2) {
+            sh = s_lcp[lead];
+            for (int j = 1; j < cnt; ++j) sh = min(sh, s_lcp[lead + j]);
+        }
+        m = (int)(key & 0xffffffffu);
+        ctx = s_ctx[m];
+        S = sh * bs;
+        pp = (S + P - 1) / P;
+        sfull = (ctx - S) / P;
+        stail = (ctx - S) - sfull * P;
+        nparts = pp + sfull + (stail > 0);
+        if (S > 0 && lead == tid) {
+            pfull = S / P;
+            ptail = S - pfull * P;
+        }
+        p.members[tid] = m;
+        p.member_nparts[tid] = nparts;
+        if (stail > 0) atomicAdd(&s_bin_count[(stail + 15) >> 4], 1);
+        if (ptail > 0) atomicAdd(&s_bin_count[(ptail + 15) >> 4], 1);
+    }
+    // Pass 1: full partitions at offsets from a block-wide scan.
+    const int full = pfull + sfull;
+    int incl = full;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(FULL_MASK, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int w = s_warp[lane];
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(FULL_MASK, wi, o);
+            if (lane >= o) wi += v;
+        }
+        s_warp[lane] = wi - w;
+        if (lane == 31) {  // tails after all full partitions, longest first
+            int pos = wi;
+            for (int b = tiles; b >= 1; --b) {
+                s_bin_next[b] = pos;
+                pos += s_bin_count[b];
+            }
+            *p.num_entries = pos;
+            *p.counter = 0;
+        }
+    }
+    __syncthreads();
+    int off = s_warp[warp] + incl - full;
+    for (int j = 0; j < pfull; ++j, ++off) {
+        p.entries[off] = make_int4(m, j, P, 0);
+        p.entries_b[off] = make_int4(j * P, tid, cnt, 0);
+    }
+    for (int j = 0; j < sfull; ++j, ++off) {
+        p.entries[off] = make_int4(m, pp + j, P, nparts);
+        p.entries_b[off] = make_int4(S + j * P, 0, 0, 0);
+    }
+    // Pass 2: tails; empty sequences get zero output rows.
+    if (tid < B) {
+        if (stail > 0) {
+            const int pos = atomicAdd(&s_bin_next[(stail + 15) >> 4], 1);
+            p.entries[pos] = make_int4(m, pp + sfull, stail, nparts);
+            p.entries_b[pos] = make_int4(S + sfull * P, 0, 0, 0);
+        }
+        if (ptail > 0) {
+            const int pos = atomicAdd(&s_bin_next[(ptail + 15) >> 4], 1);
+            p.entries[pos] = make_int4(m, pfull, ptail, 0);
+            p.entries_b[pos] = make_int4(pfull * P, tid, cnt, 0);
+        }
+        if (ctx == 0) {
+            const int nvec = p.num_heads * p.head_dim / 8;
+            uint4 *row = static_cast<uint4 *>(p.out) + (size_t)m * nvec;
+            for (int v = 0; v < nvec; ++v) row[v] = make_uint4(0, 0, 0, 0);
         }
     }
 }
@@ -269,6 +515,9 @@ constexpr float LAZY_MAX_LOG2 = 8.0f;
 
 struct Unit {
     int s, kvh, part, ntok, nparts, ntiles, tbl, slot;
+    int tok0;       // first token of the unit
+    int mcnt;       // shared-prefix unit: member sequences (0: sequence s alone)
+    int mseq, mnp;  // lane j < mcnt: member j's sequence and its partition count
     bool valid;
 };
 
@@ -280,21 +529,24 @@ struct Unit {
 struct UnitSource {
     const DecodeParams *p;
     int lane, total_units, Hkv, bs, blocks_per_part;
-    int state;  // 0 idle, 1 cursor claimed, 2 entry loaded, 3 table loaded, 4 list exhausted
-    int u, tbl;
-    int4 ent;
+    bool shared;  // entries carry a second int4 (first token, members)
+    int state;    // 0 idle, 1 cursor claimed, 2 entry loaded, 3 table loaded, 4 list exhausted
+    int u, tbl, mseq, mnp;
+    int4 ent, entb;
 
-    __device__ void init(const DecodeParams &params, int lane_id, int total) {
+    __device__ void init(const DecodeParams &params, int lane_id, int total, bool shared_units = false) {
         p = &params;
         lane = lane_id;
         total_units = total;
         Hkv = params.num_kv_heads;
         bs = params.block_size;
         blocks_per_part = params.partition / params.block_size;
+        shared = shared_units;
         state = 0;
         u = 0;
         tbl = 0;
-        ent = make_int4(0, 0, 0, 0);
+        mseq = mnp = 0;
+        ent = entb = make_int4(0, 0, 0, 0);
     }
 
     __device__ __forceinline__ void step() {
@@ -310,11 +562,16 @@ struct UnitSource {
                 return;
             }
             ent = p->entries[u / Hkv];
+            if (shared) entb = p->entries_b[u / Hkv];
             state = 2;
         } else if (state == 2) {
             const int nblk = (ent.z + bs - 1) / bs;
-            tbl = lane < nblk ? p->block_tables[(size_t)ent.x * p->max_blocks_per_seq + ent.y * blocks_per_part + lane]
-                              : 0;
+            const int blk0 = shared ? entb.x / bs : ent.y * blocks_per_part;
+            tbl = lane < nblk ? p->block_tables[(size_t)ent.x * p->max_blocks_per_seq + blk0 + lane] : 0;
+            if (shared && lane < entb.z) {
+                mseq = p->members[entb.y + lane];
+                mnp = p->member_nparts[entb.y + lane];
+            }
             state = 3;
         }
     }
@@ -332,6 +589,10 @@ struct UnitSource {
         x.nparts = ent.w;
         x.ntiles = (ent.z + 15) >> 4;
         x.tbl = tbl;
+        x.tok0 = shared ? entb.x : ent.y * p->partition;
+        x.mcnt = shared ? entb.z : 0;
+        x.mseq = mseq;
+        x.mnp = mnp;
         state = 0;
     }
 };
@@ -776,15 +1037,8 @@ __global__ void __launch_bounds__(DECODE_MAX_WARPS * 32, 1) pa_decode_kernel(con
                 if (lane == g) p.ml[row] = f2(Mg[g], Lg[g]);
             }
             // The last partition of this (sequence, KV head) to finish merges all.
-            __threadfence();
-            __syncwarp();
-            int done = 0;
-            if (lane == 0) done = atomicAdd(&p.merge_count[(size_t)cur.s * Hkv + cur.kvh], 1);
-            done = __shfl_sync(FULL_MASK, done, 0);
-            if (done == cur.nparts - 1) {
-                __threadfence();
-                merge_partitions<D, G, T>(p, head0, cur.nparts, lane);
-            }
+            const bool last = count_partition(&p.merge_count[(size_t)cur.s * Hkv + cur.kvh], cur.nparts, lane == 0);
+            if (__shfl_sync(FULL_MASK, last, 0)) merge_partitions<D, G, T>(p, head0, cur.nparts, lane);
         }
 
         // ---------------- next unit -------------------------------------------

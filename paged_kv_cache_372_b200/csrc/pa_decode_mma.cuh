@@ -38,18 +38,30 @@ struct MmaGeo {
     static constexpr int NBOX = D * EB / 128;             // 128-byte TMA boxes per row
     static constexpr int HALF_BYTES = 16 * D * EB;        // one K (or V) tile
     static constexpr int STAGE_BYTES = 2 * HALF_BYTES;    // K then V of one tile
-    static constexpr int Q_BYTES = G * D * 2;
 };
 
-template <int D, int G, int NS, bool KV8 = false>
-__host__ __device__ constexpr int mma_smem_bytes(int warps) {
-    // 1024 bytes of slack re-align the base for the 128-byte swizzle pattern.
-    return 1024 + warps * (NS * MmaGeo<D, G, KV8>::STAGE_BYTES + 2 * MmaGeo<D, G, KV8>::Q_BYTES) + warps * NS * 8;
+// Query slots of a warp: the G rows of one sequence, double-buffered (the
+// next unit's rows arrive while the current unit runs), or for units shared
+// by several sequences one slot of 8 rows (the MMA's N) that the next unit's
+// rows may fill once the current unit has read its own.
+template <int D, int G, bool SHARED>
+__host__ __device__ constexpr int mma_q_slot_bytes() {
+    return (SHARED ? 8 : G) * D * 2;
+}
+template <bool SHARED>
+__host__ __device__ constexpr int mma_q_slots() {
+    return SHARED ? 1 : 2;
 }
 
-template <int D, int G, int NS, bool KV8 = false>
+template <int D, int G, int NS, bool KV8 = false, bool SHARED = false>
 __host__ __device__ constexpr int mma_warp_bytes() {
-    return NS * MmaGeo<D, G, KV8>::STAGE_BYTES + 2 * MmaGeo<D, G, KV8>::Q_BYTES + NS * 8;
+    return NS * MmaGeo<D, G, KV8>::STAGE_BYTES + mma_q_slots<SHARED>() * mma_q_slot_bytes<D, G, SHARED>() + NS * 8;
+}
+
+template <int D, int G, int NS, bool KV8 = false, bool SHARED = false>
+__host__ __device__ constexpr int mma_smem_bytes(int warps) {
+    // 1024 bytes of slack re-align the base for the 128-byte swizzle pattern.
+    return 1024 + warps * mma_warp_bytes<D, G, NS, KV8, SHARED>();
 }
 
 // Warps per CTA: the fp8 kernel runs DECODE_MAX_WARPS_FP8 warps for small head
@@ -228,11 +240,14 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
     }
 }
 
-template <int D, int G, typename T, int NS, bool KV8 = false>
+template <int D, int G, typename T, int NS, bool KV8 = false, bool SHARED = false>
 __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
     using Gm = MmaGeo<D, G, KV8>;
+    constexpr int QB = mma_q_slot_bytes<D, G, SHARED>();  // bytes of one query slot
+    constexpr int QS = mma_q_slots<SHARED>();              // query slots per warp
+    constexpr int QG = G * D * 2;                          // query rows of one sequence
     using MT = typename std::conditional<KV8, __half, T>::type;  // MMA operand type
     extern __shared__ uint8_t smem_raw[];
     const int lane = threadIdx.x & 31;
@@ -247,9 +262,9 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     uint8_t *base = smem_raw + (base_s - raw_s);
     const uint32_t ring_s = base_s + warp * NS * Gm::STAGE_BYTES;
     uint8_t *ring = base + warp * NS * Gm::STAGE_BYTES;
-    const uint32_t qbuf_s = base_s + warps * NS * Gm::STAGE_BYTES + warp * 2 * Gm::Q_BYTES;
-    const uint8_t *qbuf = base + warps * NS * Gm::STAGE_BYTES + warp * 2 * Gm::Q_BYTES;
-    const uint32_t bar_s = base_s + warps * (NS * Gm::STAGE_BYTES + 2 * Gm::Q_BYTES) + warp * NS * 8;
+    const uint32_t qbuf_s = base_s + warps * NS * Gm::STAGE_BYTES + warp * QS * QB;
+    const uint8_t *qbuf = base + warps * NS * Gm::STAGE_BYTES + warp * QS * QB;
+    const uint32_t bar_s = base_s + warps * (NS * Gm::STAGE_BYTES + QS * QB) + warp * NS * 8;
 
     if (lane == 0) {
         for (int i = 0; i < NS; ++i) mbar_init(bar_s + 8 * i, 1);
@@ -265,20 +280,28 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     const int total_units = *p.num_entries * Hkv;
 
     UnitSource src;
-    src.init(p, lane, total_units);
+    src.init(p, lane, total_units, SHARED);
     auto fetch = [&](Unit &x) { src.take(x); };
 
     // Item `it` of a unit is its tile `it`: the K and V rows of 16 tokens;
-    // item 0 also brings the unit's G query rows.
-    auto issue = [&](int s, int kvh, int tbl, int qslot, int it, uint32_t stage) {
+    // item 0 also brings the unit's query rows (G per member sequence; mseq
+    // is lane j's member sequence for a unit of mcnt > 0 members).
+    auto issue = [&](int s, int kvh, int tbl, int qslot, int mcnt, int mseq, int it, uint32_t stage) {
         const int tok = 16 * it;
         const int bi = tok / bs;
         const int pb = __shfl_sync(FULL_MASK, tbl, bi);
+        // Member sequences of a shared unit reach the issuing lane by shuffle.
+        int mid[SHARED ? 8 : 1];
+        if constexpr (SHARED) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mid[j] = __shfl_sync(FULL_MASK, mseq, j);
+        }
         if (lane == 0) {
             const uint32_t bar = bar_s + 8 * stage;
             const bool ok = (unsigned)pb < (unsigned)p.num_blocks;
             if (!ok) raise_error(PA_DEVERR_BLOCK_ID);
-            const uint32_t bytes = (ok ? Gm::STAGE_BYTES : 0) + (it == 0 ? Gm::Q_BYTES : 0);
+            const int qrows_bytes = it != 0 ? 0 : (SHARED && mcnt > 0 ? mcnt * QG : QG);
+            const uint32_t bytes = (ok ? Gm::STAGE_BYTES : 0) + qrows_bytes;
             fence_proxy_async_smem();
             if (bytes) {
                 mbar_arrive_expect_tx(bar, bytes);
@@ -291,9 +314,21 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                         tma_load_2d(dst + Gm::HALF_BYTES + b * 2048, &tm_v, 64 * b, row, bar, policy);
                     }
                 }
-                if (it == 0)
-                    bulk_load(qbuf_s + qslot * Gm::Q_BYTES, qg + ((size_t)s * H + kvh * G) * D, Gm::Q_BYTES, bar,
-                              policy);
+                if (it == 0) {
+                    if constexpr (SHARED) {
+                        if (mcnt > 0) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                if (j < mcnt)
+                                    bulk_load(qbuf_s + qslot * QB + j * QG,
+                                              qg + ((size_t)mid[j] * H + kvh * G) * D, QG, bar, policy);
+                        } else {
+                            bulk_load(qbuf_s + qslot * QB, qg + ((size_t)s * H + kvh * G) * D, QG, bar, policy);
+                        }
+                    } else {
+                        bulk_load(qbuf_s + qslot * QB, qg + ((size_t)s * H + kvh * G) * D, QG, bar, policy);
+                    }
+                }
             } else {
                 mbar_arrive(bar);
             }
@@ -309,28 +344,45 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     bool prod_on_nxt = false, exhausted = false;
     int pitem = 0;
     uint32_t issued = 0, consumed = 0;
+    uint32_t cur_q_item = 0, nxt_q_item = 0;  // issue index of a unit's item 0 (its query rows)
 
-    auto produce = [&]() {
-        if (exhausted) return;
+    // Issues the next item if it may go now; returns whether it did.
+    auto produce = [&]() -> bool {
+        if (exhausted) return false;
         if (pitem >= (prod_on_nxt ? nxt.ntiles : cur.ntiles)) {
-            if (prod_on_nxt) return;
+            if (prod_on_nxt) return false;
             fetch(nxt);
             if (!nxt.valid) {
                 exhausted = true;
-                return;
+                return false;
             }
-            nxt.slot = next_slot;
+            nxt.slot = QS == 1 ? 0 : next_slot;
             next_slot ^= 1;
             prod_on_nxt = true;
             pitem = 0;
         }
+        // One query slot: the next unit's rows wait until the current unit
+        // has read its own (at its first tile).
+        if (QS == 1 && prod_on_nxt && pitem == 0 && consumed <= cur_q_item) return false;
+        if (pitem == 0) {
+            if (prod_on_nxt)
+                nxt_q_item = issued;
+            else
+                cur_q_item = issued;
+        }
         if (prod_on_nxt)
-            issue(nxt.s, nxt.kvh, nxt.tbl, nxt.slot, pitem, issued % NS);
+            issue(nxt.s, nxt.kvh, nxt.tbl, nxt.slot, nxt.mcnt, nxt.mseq, pitem, issued % NS);
         else
-            issue(cur.s, cur.kvh, cur.tbl, cur.slot, pitem, issued % NS);
+            issue(cur.s, cur.kvh, cur.tbl, cur.slot, cur.mcnt, cur.mseq, pitem, issued % NS);
         ++pitem;
         ++issued;
         src.step();  // one link of the next unit's claim per issued item
+        return true;
+    };
+    // Keeps NS items in flight while there is work that may be issued.
+    auto fill = [&]() {
+        while (issued - consumed < (uint32_t)NS && produce()) {
+        }
     };
 
     auto wait_item = [&]() -> bool {
@@ -345,18 +397,26 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
         return ok;
     };
 
-    for (int i = 0; i < NS; ++i) produce();
+    // With two query slots nothing is ever held back: NS items now, then one
+    // per freed stage keeps the ring full. With one slot, refill to NS.
+    if constexpr (QS == 1)
+        fill();
+    else
+        for (int i = 0; i < NS; ++i) produce();
 
-    // Heads this lane's accumulator columns belong to, and whether they exist.
+    // Query rows (MMA columns) of this lane's accumulators.
     const int h0 = 2 * t4, h1 = 2 * t4 + 1;
-    const bool hv0 = h0 < G, hv1 = h1 < G;
     // Fused append: the unit that holds a sequence's last token writes the new
     // K/V row into the pool and uses it in place of the tile's old contents.
     constexpr int NVR = D / 8;  // 16-byte vectors per row
     const bool append = !KV8 && p.k_new != nullptr;  // the fp8 cache has no fused append
 
     for (;;) {
-        uint32_t qb[Gm::KS][2];  // B fragments of Q^T: query head g8, 2 columns
+        // Query rows of the unit (G per member sequence) and whether this
+        // lane's two accumulator columns are among them.
+        const int nrows = SHARED && cur.mcnt > 0 ? cur.mcnt * G : G;
+        const bool hv0 = h0 < nrows, hv1 = h1 < nrows;
+        uint32_t qb[Gm::KS][2];  // B fragments of Q^T: query row g8, 2 columns
         float o[Gm::KS][4];      // O^T fragments: rows d = 16*i + g8 (+8), heads h0, h1
         float M0 = -INFINITY, M1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 #pragma unroll
@@ -379,7 +439,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             const uint32_t ks_s = ring_s + stage * Gm::STAGE_BYTES;
             const uint32_t vs_s = ks_s + Gm::HALF_BYTES;
             if (k == 0) {
-                const uint8_t *qs = qbuf + cur.slot * Gm::Q_BYTES;
+                const uint8_t *qs = qbuf + cur.slot * QB;
 #pragma unroll
                 for (int i = 0; i < Gm::KS; ++i) {
                     if constexpr (KV8) {
@@ -387,13 +447,15 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                         // (the order the byte-wise fragments arrive in); the
                         // query fragment follows the same order.
                         const int d = 16 * i + 4 * t4;
-                        qb[i][0] = g8 < G ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2)) : 0u;
-                        qb[i][1] = g8 < G ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 2) * 2))
-                                          : 0u;
+                        qb[i][0] = g8 < nrows ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2))
+                                              : 0u;
+                        qb[i][1] = g8 < nrows
+                                       ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 2) * 2))
+                                       : 0u;
                     } else {
                         const int d = 16 * i + 2 * t4;
-                        qb[i][0] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
-                        qb[i][1] = g8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 8) * 2) : 0u;
+                        qb[i][0] = g8 < nrows ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
+                        qb[i][1] = g8 < nrows ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 8) * 2) : 0u;
                     }
                 }
             }
@@ -533,7 +595,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             }
             ++consumed;
             __syncwarp();
-            produce();
+            if constexpr (QS == 1)
+                fill();
+            else
+                produce();
         }
 
         // ---------------- totals and store -------------------------------------
@@ -543,7 +608,49 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             l1 += __shfl_xor_sync(FULL_MASK, l1, off);
         }
         const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;
-        if (KV8 && cur.nparts == 1) {
+        if (SHARED && cur.mcnt > 0) {
+            // Partials of every member: column h of the accumulators is query
+            // row h, i.e. head h % G of member h / G.
+            const int seq0 = __shfl_sync(FULL_MASK, cur.mseq, (h0 / G) & 7);
+            const int seq1 = __shfl_sync(FULL_MASK, cur.mseq, (h1 / G) & 7);
+            const size_t row0 = ((size_t)seq0 * Hkv + cur.kvh) * p.max_parts + cur.part;
+            const size_t row1 = ((size_t)seq1 * Hkv + cur.kvh) * p.max_parts + cur.part;
+            float *acc0 = p.part_acc + row0 * (size_t)(D * G);
+            float *acc1 = p.part_acc + row1 * (size_t)(D * G);
+            const int g0 = h0 % G, g1 = h1 % G;
+            const float vs = KV8 ? p.v_scale : 1.f;
+#pragma unroll
+            for (int i = 0; i < Gm::KS; ++i) {
+                const int d = KV8 ? 16 * i + 2 * g8 : 16 * i + g8;
+                const int d2 = KV8 ? d + 1 : d + 8;
+                if constexpr (G == 1) {
+                    if (hv0) {
+                        acc0[d] = o[i][0] * vs;
+                        acc0[d2] = o[i][2] * vs;
+                    }
+                    if (hv1) {
+                        acc1[d] = o[i][1] * vs;
+                        acc1[d2] = o[i][3] * vs;
+                    }
+                } else if (hv1) {  // G even: columns h0, h1 are heads g0, g0 + 1 of one member
+                    *reinterpret_cast<float2 *>(acc0 + d * G + g0) = make_float2(o[i][0] * vs, o[i][1] * vs);
+                    *reinterpret_cast<float2 *>(acc0 + d2 * G + g0) = make_float2(o[i][2] * vs, o[i][3] * vs);
+                }
+            }
+            if (g8 == 0 && hv0) p.ml[row0 * G + g0] = make_float2(M0, l0);
+            if (g8 == 0 && hv1) p.ml[row1 * G + g1] = make_float2(M1, l1);
+            // Lane j counts member j's partition.
+            const bool last = count_partition(&p.merge_count[(size_t)cur.mseq * Hkv + cur.kvh], cur.mnp,
+                                              lane < cur.mcnt);
+            unsigned lm = __ballot_sync(FULL_MASK, last);
+            while (lm) {
+                const int j = __ffs(lm) - 1;
+                lm &= lm - 1;
+                const int sj = __shfl_sync(FULL_MASK, cur.mseq, j);
+                const int nj = __shfl_sync(FULL_MASK, cur.mnp, j);
+                mma_merge<D, G, T>(p, (size_t)sj * Hkv + cur.kvh, (size_t)sj * H + (size_t)cur.kvh * G, nj, lane);
+            }
+        } else if (KV8 && cur.nparts == 1) {
             // Accumulator rows g8 / g8+8 of slice i are elements 16i + 2*g8 / + 1:
             // pairs of adjacent elements per head, stored directly.
             const float i0 = hv0 ? p.v_scale / l0 : 0.f, i1 = hv1 ? p.v_scale / l1 : 0.f;
@@ -590,21 +697,16 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             }
             if (g8 == 0 && hv0) p.ml[row * G + h0] = make_float2(M0, l0);
             if (g8 == 0 && hv1) p.ml[row * G + h1] = make_float2(M1, l1);
-            __threadfence();
-            __syncwarp();
-            int done = 0;
-            if (lane == 0) done = atomicAdd(&p.merge_count[group], 1);
-            done = __shfl_sync(FULL_MASK, done, 0);
-            if (done == cur.nparts - 1) {
-                __threadfence();
-                mma_merge<D, G, T>(p, group, head0, cur.nparts, lane);
-            }
+            const bool last = count_partition(&p.merge_count[group], cur.nparts, lane == 0);
+            if (__shfl_sync(FULL_MASK, last, 0)) mma_merge<D, G, T>(p, group, head0, cur.nparts, lane);
         }
 
         while (!prod_on_nxt && !exhausted) produce();
         if (!prod_on_nxt) break;
         cur = nxt;
+        cur_q_item = nxt_q_item;
         prod_on_nxt = false;
+        if constexpr (QS == 1) fill();
     }
 }
 

@@ -118,7 +118,7 @@ pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, in
     return PA_OK;
 }
 
-template <int D, int G, typename T, bool KV8 = false>
+template <int D, int G, typename T, bool KV8 = false, bool SHARED = false>
 pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     constexpr int NS = KV8 ? pa::DECODE_MMA_STAGES_FP8 : pa::DECODE_MMA_STAGES;
     DeviceInfo info;
@@ -131,15 +131,18 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     if ((st = encode_pool_map(&tmk, p.k_pool, rows, D, KV8 ? 1 : 2, type)) != PA_OK) return st;
     if ((st = encode_pool_map(&tmv, p.v_pool, rows, D, KV8 ? 1 : 2, type)) != PA_OK) return st;
     constexpr int max_warps = pa::mma_max_warps<G, KV8>();
-    int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS, KV8>();
+    int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS, KV8, SHARED>();
     if (warps > max_warps) warps = max_warps;
     if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "not enough shared memory for one warp");
-    const int smem = pa::mma_smem_bytes<D, G, NS, KV8>(warps);
-    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS, KV8>;
+    const int smem = pa::mma_smem_bytes<D, G, NS, KV8, SHARED>(warps);
+    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS, KV8, SHARED>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
-    pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
+    if constexpr (SHARED)
+        pa::pa_plan_shared_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
+    else
+        pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sms);
     cfg.blockDim = dim3(warps * 32);
@@ -165,6 +168,24 @@ pa_status dispatch_group_fp8(pa::DecodeParams &p, int group, cudaStream_t stream
         case 2: return launch_decode_mma<128, 2, T, true>(p, stream);
         case 4: return launch_decode_mma<128, 4, T, true>(p, stream);
         case 8: return launch_decode_mma<128, 8, T, true>(p, stream);
+    }
+    return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
+}
+
+// Shared-prefix units (pa_decode_shared): tensor-core kernel, 16-bit cache.
+template <int D, typename T>
+pa_status dispatch_group_shared(pa::DecodeParams &p, int group, cudaStream_t stream) {
+    if (group < pa::DECODE_TENSOR_MIN_GROUP)
+        return fail(PA_ERR_UNSUPPORTED, "shared-prefix units need the tensor-core kernel (group %d)", group);
+    switch (group) {
+        case 1: return launch_decode_mma<D, 1, T, false, true>(p, stream);
+        case 2: return launch_decode_mma<D, 2, T, false, true>(p, stream);
+        case 4: return launch_decode_mma<D, 4, T, false, true>(p, stream);
+        case 8: {
+            // Eight query heads fill a unit's 8 query rows: nothing to share.
+            p.entries_b = nullptr;
+            return launch_decode_mma<D, 8, T>(p, stream);
+        }
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }

@@ -83,3 +83,28 @@ def gpu_step_fused(wl, step, kp, vp, partition_size=None, workspace=None):
                         torch.from_numpy(st.block_tables).to(dev), torch.from_numpy(st.context_lens).to(dev),
                         wl.scale, int(st.context_lens.max()), P, workspace)
     return out
+
+
+def gpu_step_shared(wl, step, kp, vp, partition_size=None, workspace=None, fused=True):
+    """The same step through pa_decode_shared: copies, extra tokens, then the
+    shared-prefix decode, appending each sequence's new token (fused) or with
+    every new token written by pa_reshape_and_cache first."""
+    st = wl.steps[step]
+    dev = kp.device
+    B = st.q.shape[0]
+    if len(st.copy_pairs):
+        pa.pa_copy_blocks([kp, vp], torch.from_numpy(st.copy_pairs).to(dev))
+    first = B if fused else 0
+    if len(st.slot_mapping) > first:
+        pa.pa_reshape_and_cache(st.k_new[first:].to(dev), st.v_new[first:].to(dev), kp, vp,
+                                torch.from_numpy(st.slot_mapping[first:]).to(dev))
+    q = st.q.to(dev)
+    out = torch.empty_like(q)
+    P = wl.partition_size if partition_size is None else partition_size
+    kw = {}
+    if fused:
+        kw = dict(k_new=st.k_new[:B].contiguous().to(dev), v_new=st.v_new[:B].contiguous().to(dev))
+    pa.pa_decode_shared(out, q, kp, vp, torch.from_numpy(st.block_tables).to(dev),
+                        torch.from_numpy(st.context_lens).to(dev), wl.scale, int(st.context_lens.max()), P,
+                        workspace, **kw)
+    return out

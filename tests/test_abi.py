@@ -42,3 +42,21 @@ def test_reshape_rejects_bad_arguments_without_a_device():
     ptrs = (ctypes.c_void_p * 1)(None)
     assert lib.pa_copy_blocks(ptrs, 1, None, 1, 100, 32, None) == pa.PA_ERR_INVALID
     assert lib.pa_last_error() != b""
+
+
+def test_shared_decode_host_checks_without_a_device():
+    lib = pa.lib()
+    plain = pa.pa_decode_workspace_size(64, 32, 8, 128, 16, 2048, 0)
+    shared = pa.pa_decode_shared_workspace_size(64, 32, 8, 128, 16, 2048, 0)
+    # one more partition of partials per sequence, the second entry words and the member lists
+    parts = 2048 // 512
+    assert shared >= plain + 64 * 32 * (8 + 128 * 4) + 64 * (parts + 1) * 16 + 2 * 64 * 4
+    assert lib.pa_decode_shared_workspace_size(4, 2, 2, 96, 16, 33, 0) == 0
+    dummy = ctypes.c_void_p(256)
+    args = [dummy, dummy, None, None, dummy, dummy, dummy, dummy]
+    rest = [32, 8, 128, 16, 64, 4096, 1024, ctypes.c_float(0.1), 0, 0, dummy, 1 << 30, None]
+    # k_new without v_new
+    assert lib.pa_decode_shared(dummy, dummy, dummy, None, *args[4:], 8, *rest) == pa.PA_ERR_INVALID
+    # more sequences than the grouping takes
+    assert lib.pa_decode_shared(*args, 1025, *rest) == pa.PA_ERR_UNSUPPORTED
+    assert b"1024" in lib.pa_last_error()
