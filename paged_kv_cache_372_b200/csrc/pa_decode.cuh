@@ -507,6 +507,9 @@ constexpr int DECODE_MMA_STAGES_FP8 = PA_DECODE_MMA_STAGES_FP8;
 constexpr int DECODE_MAX_WARPS_FP8 = PA_DECODE_MAX_WARPS_FP8;
 constexpr int DECODE_TENSOR_MIN_GROUP = PA_DECODE_TENSOR_MIN_GROUP;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
+// Items of a unit over which the tensor-core kernel claims the next unit
+// (the claim is three dependent global accesses, one per issued item).
+constexpr int CLAIM_AHEAD = 3;
 // The running maximum of a head is only raised when a score exceeds it by more
 // than this many log2 units, so exponentials stay <= 2^8 and rescaling of the
 // accumulators is rare. The final normalisation uses the same reference, so the
@@ -526,18 +529,28 @@ struct Unit {
 // block-table slice, one entry per lane); step() advances the chain for the
 // next unit by one link, so that called once per issued tile it has the next
 // unit ready before the warp needs it, and take() only finishes what is left.
+// The first claims of a launch arrive about in CTA order, all at once, so
+// in a longest-first list the first CTAs would take only long units and the
+// last ones only short ones. Claims below `wave1` (a multiple of the warps
+// per CTA, at most the number of warps) are therefore spread: claim c takes
+// unit (c % K) * (wave1 / K) + c / K, K warps per CTA, so each CTA's first
+// units come from every part of the list; later claims go in list order.
 struct UnitSource {
     const DecodeParams *p;
     int lane, total_units, Hkv, bs, blocks_per_part;
-    bool shared;  // entries carry a second int4 (first token, members)
+    int k, wave1;  // warps per CTA; claims spread over the first wave
+    bool shared;   // entries carry a second int4 (first token, members)
     int state;    // 0 idle, 1 cursor claimed, 2 entry loaded, 3 table loaded, 4 list exhausted
     int u, tbl, mseq, mnp;
     int4 ent, entb;
 
-    __device__ void init(const DecodeParams &params, int lane_id, int total, bool shared_units = false) {
+    __device__ void init(const DecodeParams &params, int lane_id, int total, bool shared_units = false,
+                         int warps_per_cta = 1, int warps_total = 0) {
         p = &params;
         lane = lane_id;
         total_units = total;
+        k = warps_per_cta;
+        wave1 = min(warps_total, total) / warps_per_cta * warps_per_cta;
         Hkv = params.num_kv_heads;
         bs = params.block_size;
         blocks_per_part = params.partition / params.block_size;
@@ -557,6 +570,7 @@ struct UnitSource {
             state = 1;
         } else if (state == 1) {
             u = __shfl_sync(FULL_MASK, u, 0);
+            if (u < wave1) u = (u % k) * (wave1 / k) + u / k;
             if (u >= total_units) {
                 state = 4;
                 return;

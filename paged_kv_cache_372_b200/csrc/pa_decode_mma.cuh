@@ -169,60 +169,96 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 // j computes partition j's G weights (32 partitions per round), the weights
 // reach the other lanes by shuffle, and each lane reads its EPL x G contiguous
 // floats of every partition with vector loads.
-template <int D, int G, typename T>
+// LEAN (kernels under a 128-register cap) keeps fewer values live: the
+// (max, sum) pairs are read twice and no partials are loaded ahead.
+template <int D, int G, typename T, bool LEAN = false>
 __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, size_t head0, int nparts, int lane) {
     constexpr int EPL = D / 32;
-    constexpr int VW = EPL * G >= 4 ? 4 : EPL * G;  // floats per vector load (4 or 2)
-    constexpr int NV4 = EPL * G / VW;               // vector loads per partition per lane
+    constexpr int F = EPL * G;                             // floats of one partition per lane
+    constexpr int VW = F >= 4 ? 4 : F;                     // floats per vector load (4 or 2)
+    constexpr int NV4 = F / VW;                            // vector loads per partition per lane
+    // partitions whose partials load up front
+    constexpr int PF = LEAN ? 0 : (F <= 8 ? 4 : (F <= 16 ? 1 : 0));
     const float2 *ml = p.ml + group * p.max_parts * G;
     const float *acc = p.part_acc + group * p.max_parts * (size_t)(D * G);
-    float M[G], L[G], o[EPL * G];
+    auto load = [&](int j, float (&f)[F]) {
+        const float *a = acc + (size_t)j * D * G + lane * F;
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) {
+            if constexpr (VW == 4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(a) + i);
+                f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
+            } else {
+                const float2 v = __ldcg(reinterpret_cast<const float2 *>(a) + i);
+                f[2 * i] = v.x; f[2 * i + 1] = v.y;
+            }
+        }
+    };
+    // The first partitions' partials are requested together with the (max,
+    // sum) pairs, which each lane reads once (lane j: partition j), so the
+    // usual few-partition merge waits on one round of loads.
+    float pre[PF > 0 ? PF : 1][F];
+#pragma unroll
+    for (int q = 0; q < PF; ++q) {
+        if (q < nparts) {
+            load(q, pre[q]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < F; ++c) pre[q][c] = 0.f;
+        }
+    }
+    float2 mine[LEAN ? 1 : G];
+    float M[G], L[G], o[F];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        M[g] = -INFINITY;
+        const float2 v = lane < nparts ? __ldcg(&ml[lane * G + g]) : make_float2(-INFINITY, 0.f);
+        if constexpr (!LEAN) mine[g] = v;
+        M[g] = v.x;
         L[g] = 0.f;
     }
-#pragma unroll
-    for (int i = 0; i < EPL * G; ++i) o[i] = 0.f;
-    for (int j = lane; j < nparts; j += 32)
+    for (int j = lane + 32; j < nparts; j += 32)
 #pragma unroll
         for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __ldcg(&ml[j * G + g].x));
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1)
 #pragma unroll
         for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], __shfl_xor_sync(FULL_MASK, M[g], off));
+#pragma unroll
+    for (int c = 0; c < F; ++c) o[c] = 0.f;
     for (int base = 0; base < nparts; base += 32) {
         float w[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) w[g] = 0.f;
-        if (base + lane < nparts) {
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float2 v = __ldcg(&ml[(base + lane) * G + g]);
-                w[g] = exp2f(v.x - M[g]);
-                L[g] = fmaf(w[g], v.y, L[g]);
-            }
+        for (int g = 0; g < G; ++g) {
+            float2 v;
+            if (!LEAN && base == 0)
+                v = mine[LEAN ? 0 : g];
+            else
+                v = base + lane < nparts ? __ldcg(&ml[(base + lane) * G + g]) : make_float2(-INFINITY, 0.f);
+            w[g] = base + lane < nparts ? exp2f(v.x - M[g]) : 0.f;
+            L[g] = fmaf(w[g], v.y, L[g]);
         }
         const int n = min(32, nparts - base);
-#pragma unroll 4
-        for (int jj = 0; jj < n; ++jj) {
-            const float *a = acc + (size_t)(base + jj) * D * G + lane * EPL * G;
-            float f[EPL * G];
+        int jj = 0;
+        if (PF > 0 && base == 0) {
 #pragma unroll
-            for (int i = 0; i < NV4; ++i) {
-                if constexpr (VW == 4) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(a) + i);
-                    f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
-                } else {
-                    const float2 v = __ldcg(reinterpret_cast<const float2 *>(a) + i);
-                    f[2 * i] = v.x; f[2 * i + 1] = v.y;
-                }
+            for (int q = 0; q < PF; ++q) {
+                float wj[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) wj[g] = __shfl_sync(FULL_MASK, w[g], q);  // 0 past nparts
+#pragma unroll
+                for (int c = 0; c < F; ++c) o[c] = fmaf(wj[c % G], pre[q][c], o[c]);
             }
+            jj = PF;
+        }
+#pragma unroll 4
+        for (; jj < n; ++jj) {
+            float f[F];
+            load(base + jj, f);
             float wj[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) wj[g] = __shfl_sync(FULL_MASK, w[g], jj);
 #pragma unroll
-            for (int c = 0; c < EPL * G; ++c) o[c] = fmaf(wj[c % G], f[c], o[c]);
+            for (int c = 0; c < F; ++c) o[c] = fmaf(wj[c % G], f[c], o[c]);
         }
     }
 #pragma unroll
@@ -280,7 +316,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     const int total_units = *p.num_entries * Hkv;
 
     UnitSource src;
-    src.init(p, lane, total_units, SHARED);
+    src.init(p, lane, total_units, SHARED, warps, warps * (int)gridDim.x);
     auto fetch = [&](Unit &x) { src.take(x); };
 
     // Item `it` of a unit is its tile `it`: the K and V rows of 16 tokens;
@@ -376,7 +412,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             issue(cur.s, cur.kvh, cur.tbl, cur.slot, cur.mcnt, cur.mseq, pitem, issued % NS);
         ++pitem;
         ++issued;
-        src.step();  // one link of the next unit's claim per issued item
+        // One link of the next unit's claim per issued item, over the unit's
+        // last CLAIM_AHEAD items only: claimed earlier, a unit would wait on
+        // a busy warp while others that finish sooner could start it.
+        if ((prod_on_nxt ? nxt.ntiles : cur.ntiles) - pitem < CLAIM_AHEAD) src.step();
         return true;
     };
     // Keeps NS items in flight while there is work that may be issued.
@@ -648,7 +687,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                 lm &= lm - 1;
                 const int sj = __shfl_sync(FULL_MASK, cur.mseq, j);
                 const int nj = __shfl_sync(FULL_MASK, cur.mnp, j);
-                mma_merge<D, G, T>(p, (size_t)sj * Hkv + cur.kvh, (size_t)sj * H + (size_t)cur.kvh * G, nj, lane);
+                mma_merge<D, G, T, KV8>(p, (size_t)sj * Hkv + cur.kvh, (size_t)sj * H + (size_t)cur.kvh * G, nj, lane);
             }
         } else if (KV8 && cur.nparts == 1) {
             // Accumulator rows g8 / g8+8 of slice i are elements 16i + 2*g8 / + 1:
@@ -698,7 +737,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             if (g8 == 0 && hv0) p.ml[row * G + h0] = make_float2(M0, l0);
             if (g8 == 0 && hv1) p.ml[row * G + h1] = make_float2(M1, l1);
             const bool last = count_partition(&p.merge_count[group], cur.nparts, lane == 0);
-            if (__shfl_sync(FULL_MASK, last, 0)) mma_merge<D, G, T>(p, group, head0, cur.nparts, lane);
+            if (__shfl_sync(FULL_MASK, last, 0)) mma_merge<D, G, T, KV8>(p, group, head0, cur.nparts, lane);
         }
 
         while (!prod_on_nxt && !exhausted) produce();
