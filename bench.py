@@ -377,7 +377,7 @@ def run_ours(args, world, rank, local):
                                 "merge fused)" if fused else
                                 "pa_decode call (plan + attention launches; split merge fused)"),
                      "bytes": "unique K+V bytes of valid tokens per call",
-                     "traffic": profiled_traffic(wl.name + ("@fp8" if kv8 else "")
+                     "traffic": profiled_traffic(wl.name + ("@fp8" if kv8 else "") + ("@shared" if share else "")
                                                  + ("" if args.partition is None else f"@P{args.partition}"))},
         "gpu_launches": launches,
         "step": ("pa_copy_blocks (if any), pa_reshape_and_cache_fp8, pa_decode_fp8" if kv8 else

@@ -171,6 +171,10 @@ PA_API pa_status pa_decode_append(void *out, const void *q, const void *k_new, c
  * identity. Without shared blocks, the result and the work are those of
  * pa_decode.
  *
+ * partition_size 0 picks 16 blocks for grouped heads (group >= 2; smaller
+ * units balance better once the shared tiles are streamed once per group),
+ * otherwise as pa_decode.
+ *
  * Requirements beyond pa_decode's: num_seqs <= 1024, fp16/bf16 cache
  * (the tensor-core kernel). workspace: at least
  * pa_decode_shared_workspace_size(...) bytes (one more partition per
@@ -185,6 +189,10 @@ PA_API pa_status pa_decode_shared(void *out, const void *q, const void *k_new, c
                                   int max_blocks_per_seq, int num_blocks, int max_context_len,
                                   float scale, int dtype, int partition_size, void *workspace,
                                   size_t workspace_bytes, pa_stream_t stream);
+
+/* Partition pa_decode_shared uses for these arguments (0 if invalid). */
+PA_API int pa_decode_shared_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                           int block_size, int max_context_len, int partition_size);
 
 /* Workspace bytes pa_decode_shared needs (0 for unsupported shapes). */
 PA_API size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int num_kv_heads,

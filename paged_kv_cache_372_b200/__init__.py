@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_shared.restype = _I
         L.pa_decode_shared.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                        _I, _P, _SZ, _P]
+        L.pa_decode_shared_partition_size.restype = _I
+        L.pa_decode_shared_partition_size.argtypes = [_I] * 7
         L.pa_decode_shared_workspace_size.restype = _SZ
         L.pa_decode_shared_workspace_size.argtypes = [_I] * 7
         L.pa_decode_fp8.restype = _I
@@ -131,6 +133,12 @@ def pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_
     if n == 0:
         raise PagedAttentionError(PA_ERR_INVALID, "unsupported shape or partition size")
     return n
+
+
+def pa_decode_shared_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                                    partition_size=0) -> int:
+    return int(lib().pa_decode_shared_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                     max_context_len, partition_size))
 
 
 def pa_decode_shared_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,

@@ -52,6 +52,11 @@ def test_shared_decode_host_checks_without_a_device():
     parts = 2048 // 512
     assert shared >= plain + 64 * 32 * (8 + 128 * 4) + 64 * (parts + 1) * 16 + 2 * 64 * 4
     assert lib.pa_decode_shared_workspace_size(4, 2, 2, 96, 16, 33, 0) == 0
+    # shared-prefix units: 16 blocks for grouped heads, as pa_decode otherwise
+    assert pa.pa_decode_shared_partition_size(4, 32, 8, 128, 16, 8192, 0) == 256
+    assert pa.pa_decode_shared_partition_size(4, 32, 32, 128, 16, 8192, 0) == 256
+    assert pa.pa_decode_shared_partition_size(4, 32, 8, 128, 16, 100, 0) == 112
+    assert pa.pa_decode_shared_partition_size(4, 32, 8, 128, 16, 8192, 512) == 512
     dummy = ctypes.c_void_p(256)
     args = [dummy, dummy, None, None, dummy, dummy, dummy, dummy]
     rest = [32, 8, 128, 16, 64, 4096, 1024, ctypes.c_float(0.1), 0, 0, dummy, 1 << 30, None]

@@ -213,7 +213,7 @@ def test_sharing_patterns_match_oracle(shape, append):
         if append:
             assert H.pools_equal(kp, vp, okp, ovp)
         # The plan grouped the sequences as described (units per KV head).
-        Pr = pa.pa_decode_partition_size(len(case["ctx"]), heads, kv_heads, D, bs, int(case["ctx"].max()), P)
+        Pr = pa.pa_decode_shared_partition_size(len(case["ctx"]), heads, kv_heads, D, bs, int(case["ctx"].max()), P)
         n_expect, n_shared = expected_entries(case, Pr, append)
         assert int(ws[4:8].view(torch.int32).item()) == n_expect
         assert n_shared >= 10 or heads // kv_heads == 8  # 8 query heads fill a unit alone
