@@ -250,6 +250,9 @@ def run_ours(args, world, rank, local):
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
 
     kv8 = args.kv == "fp8"
+    if kv8:
+        ws = pa.alloc_workspace(B, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, max_ctx, P, dev,
+                                fp8=True)
     fused = not args.unfused and not kv8 and appends_at_last_positions(wl)
     share = not kv8 and (args.share == "on" or (args.share == "auto" and wl.kv_bytes_unique() < wl.kv_bytes()))
     if share:

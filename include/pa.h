@@ -190,6 +190,13 @@ PA_API pa_status pa_decode_shared(void *out, const void *q, const void *k_new, c
                                   float scale, int dtype, int partition_size, void *workspace,
                                   size_t workspace_bytes, pa_stream_t stream);
 
+/* Partition and workspace bytes pa_decode_fp8 uses for these arguments
+ * (0 if invalid, e.g. head_dim other than 128). */
+PA_API int pa_decode_fp8_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                        int block_size, int max_context_len, int partition_size);
+PA_API size_t pa_decode_fp8_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                           int block_size, int max_context_len, int partition_size);
+
 /* Partition pa_decode_shared uses for these arguments (0 if invalid). */
 PA_API int pa_decode_shared_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                            int block_size, int max_context_len, int partition_size);
@@ -206,8 +213,10 @@ PA_API size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int n
  * by `dtype`). k_pool, v_pool: uint8 codes [num_blocks][num_kv_heads]
  * [block_size][head_dim], written by pa_reshape_and_cache_fp8. head_dim 128.
  * The products run on tensor cores with the codes widened to fp16 (exact) and
- * the queries converted to fp16 (exact for |q| in fp16's normal range); the
- * workspace is sized by pa_decode_workspace_size as for pa_decode.
+ * the queries converted to fp16 (exact for |q| in fp16's normal range). The
+ * workspace is sized by pa_decode_fp8_workspace_size: partition_size 0 picks
+ * 512 tokens for one query head per KV head and max(256 tokens, 8 blocks)
+ * otherwise (pa_decode_fp8_partition_size).
  *
  * Defined by: "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
  * section 3.2 (内存压缩技术) — keep the KV cache in fewer bits to cut its

@@ -57,6 +57,10 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_shared.restype = _I
         L.pa_decode_shared.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                        _I, _P, _SZ, _P]
+        L.pa_decode_fp8_partition_size.restype = _I
+        L.pa_decode_fp8_partition_size.argtypes = [_I] * 7
+        L.pa_decode_fp8_workspace_size.restype = _SZ
+        L.pa_decode_fp8_workspace_size.argtypes = [_I] * 7
         L.pa_decode_shared_partition_size.restype = _I
         L.pa_decode_shared_partition_size.argtypes = [_I] * 7
         L.pa_decode_shared_workspace_size.restype = _SZ
@@ -135,6 +139,21 @@ def pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_
     return n
 
 
+def pa_decode_fp8_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                                 partition_size=0) -> int:
+    return int(lib().pa_decode_fp8_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                  max_context_len, partition_size))
+
+
+def pa_decode_fp8_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                                 partition_size=0) -> int:
+    n = int(lib().pa_decode_fp8_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                               max_context_len, partition_size))
+    if n == 0:
+        raise PagedAttentionError(PA_ERR_INVALID, "unsupported shape or partition size")
+    return n
+
+
 def pa_decode_shared_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
                                     partition_size=0) -> int:
     return int(lib().pa_decode_shared_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
@@ -151,10 +170,11 @@ def pa_decode_shared_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
 
 
 def alloc_workspace(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
-                    partition_size=0, device=None, shared=False) -> torch.Tensor:
-    """Workspace for pa_decode / pa_decode_append / pa_decode_fp8, or with
-    shared=True for pa_decode_shared."""
-    size = pa_decode_shared_workspace_size if shared else pa_decode_workspace_size
+                    partition_size=0, device=None, shared=False, fp8=False) -> torch.Tensor:
+    """Workspace for pa_decode / pa_decode_append, or with shared=True for
+    pa_decode_shared, or with fp8=True for pa_decode_fp8."""
+    size = (pa_decode_shared_workspace_size if shared else pa_decode_fp8_workspace_size if fp8
+            else pa_decode_workspace_size)
     n = size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size)
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
@@ -251,7 +271,7 @@ def pa_decode_fp8(out, q, k_pool, v_pool, block_tables, context_lens, scale, max
     if q.dtype not in _DTYPES or out.dtype != q.dtype:
         raise ValueError("q and out must share one dtype, fp16 or bf16")
     if workspace is None:
-        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device)
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device, fp8=True)
     _check(lib().pa_decode_fp8(
         _cuda(out, "out"), _cuda(q, "q"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
         _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),

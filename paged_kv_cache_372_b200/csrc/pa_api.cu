@@ -123,7 +123,24 @@ int pa_decode_shared_partition_size(int num_seqs, int num_heads, int num_kv_head
                                     int max_context_len, int partition_size) {
     if (num_seqs < 0 || max_context_len < 0 || partition_size < 0) return 0;
     if (!shape_supported(num_heads, num_kv_heads, head_dim, block_size)) return 0;
-    return resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size, true);
+    return resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size,
+                             PartMode::shared);
+}
+
+int pa_decode_fp8_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                 int max_context_len, int partition_size) {
+    if (num_seqs < 0 || max_context_len < 0 || partition_size < 0 || head_dim != 128) return 0;
+    if (!shape_supported(num_heads, num_kv_heads, head_dim, block_size)) return 0;
+    return resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size, PartMode::fp8);
+}
+
+size_t pa_decode_fp8_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                    int max_context_len, int partition_size) {
+    const int P = pa_decode_fp8_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                               max_context_len, partition_size);
+    if (P == 0) return 0;
+    const int max_parts = max_context_len > 0 ? ceil_div(max_context_len, P) : 1;
+    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts).total;
 }
 
 size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
@@ -165,7 +182,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
         return fail(PA_ERR_INVALID, "misaligned pointer (16 B tensors, 4 B int arrays, 256 B workspace)");
-    const int P = resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size, shared);
+    const int P = resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size,
+                                    shared ? PartMode::shared : kv8 ? PartMode::fp8 : PartMode::plain);
     if (P == 0)
         return fail(PA_ERR_INVALID, "partition_size %d (multiple of 16 and of block_size, at most %d)",
                     partition_size, partition_cap(block_size));

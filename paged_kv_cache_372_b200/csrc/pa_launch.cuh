@@ -17,12 +17,20 @@ int partition_cap(int block_size) { return 32 * block_size; }
 // Partition used when the caller passes 0 (a whole sequence when every
 // context fits in it): 32 blocks for grouped heads, 256 tokens for one query
 // head per KV head (measured best on the benchmark workloads).
+// Which entry point a partition is chosen for.
+enum class PartMode { plain, shared, fp8 };
+
 // With shared-prefix units (which always merge) 16 blocks for grouped heads:
 // the shared tiles are streamed once per group, so the remaining work is
-// spread better over the warps in smaller units.
-int auto_partition(int group, int block_size, bool shared = false) {
-    if (group >= 2) return (shared ? 16 : 32) * block_size;
-    return 256;
+// spread better over the warps in smaller units. The fp8 kernel is
+// issue-bound rather than memory-bound and was measured best at 512 tokens
+// for one query head per KV head and at max(256 tokens, 8 blocks) otherwise.
+int auto_partition(int group, int block_size, PartMode mode = PartMode::plain) {
+    switch (mode) {
+        case PartMode::shared: return group >= 2 ? 16 * block_size : 256;
+        case PartMode::fp8: return group >= 2 ? (8 * block_size > 256 ? 8 * block_size : 256) : 512;
+        default: return group >= 2 ? 32 * block_size : 256;
+    }
 }
 
 bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_size) {
@@ -34,12 +42,13 @@ bool shape_supported(int num_heads, int num_kv_heads, int head_dim, int block_si
 }
 
 // Resolves partition_size (0 = auto). Returns 0 for an invalid request.
-int resolve_partition(int group, int block_size, int max_context_len, int requested, bool shared = false) {
+int resolve_partition(int group, int block_size, int max_context_len, int requested,
+                      PartMode mode = PartMode::plain) {
     if (requested > 0) {
         if (requested % 16 || requested % block_size || requested > partition_cap(block_size)) return 0;
         return requested;
     }
-    const int auto_p = auto_partition(group, block_size, shared);
+    const int auto_p = auto_partition(group, block_size, mode);
     if (max_context_len <= auto_p) {
         const int need = max_context_len > 0 ? max_context_len : 1;
         return ((need + block_size - 1) / block_size) * block_size;
