@@ -108,9 +108,7 @@ PA_API const char *pa_last_error(void);
  *
  * max_context_len bounds every context_lens entry (larger ones are clamped and
  * flagged) and sizes the workspace. scale multiplies q.k (1/sqrt(head_dim) for
- * standard attention). context_len 0 gives a zero output row. The work list
- * encodes up to 4095 partitions of a sequence and contexts below 2^24 tokens;
- * beyond either, the call returns PA_ERR_UNSUPPORTED.
+ * standard attention). context_len 0 gives a zero output row.
  *
  * workspace: device memory of at least pa_decode_workspace_size(...) bytes,
  * 256-byte aligned, owned by the caller, contents need no initialisation.

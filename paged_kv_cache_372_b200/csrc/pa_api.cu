@@ -115,9 +115,8 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
     const int P = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                            max_context_len, partition_size);
     if (P == 0) return 0;
-    const int F = fine_partition(P, block_size, PartMode::plain);
-    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim,
-                         parts_per_sequence(max_context_len, P, F, false)).total;
+    const int max_parts = max_context_len > 0 ? ceil_div(max_context_len, P) : 1;
+    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts).total;
 }
 
 int pa_decode_shared_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
@@ -140,9 +139,8 @@ size_t pa_decode_fp8_workspace_size(int num_seqs, int num_heads, int num_kv_head
     const int P = pa_decode_fp8_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                                max_context_len, partition_size);
     if (P == 0) return 0;
-    const int F = fine_partition(P, block_size, PartMode::fp8);
-    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim,
-                         parts_per_sequence(max_context_len, P, F, false)).total;
+    const int max_parts = max_context_len > 0 ? ceil_div(max_context_len, P) : 1;
+    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts).total;
 }
 
 size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
@@ -150,8 +148,8 @@ size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int num_kv_h
     const int P = pa_decode_shared_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                                   max_context_len, partition_size);
     if (P == 0) return 0;
-    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim,
-                         parts_per_sequence(max_context_len, P, P, true), true).total;
+    const int max_parts = (max_context_len > 0 ? ceil_div(max_context_len, P) : 1) + 1;
+    return pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts, true).total;
 }
 
 }  // extern "C"
@@ -191,14 +189,11 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
                     partition_size, partition_cap(block_size));
     const long long table_tokens = (long long)max_blocks_per_seq * block_size;
     const int ctx_limit = (int)(table_tokens < max_context_len ? table_tokens : max_context_len);
-    const PartMode mode = shared ? PartMode::shared : kv8 ? PartMode::fp8 : PartMode::plain;
-    const int F = fine_partition(P, block_size, mode);
-    const int max_parts = parts_per_sequence(max_context_len, P, F, shared);
+    // With shared prefixes a sequence's partitions are cut at the end of its
+    // shared blocks too, so it can have one more.
+    const int max_parts = (max_context_len > 0 ? ceil_div(max_context_len, P) : 1) + (shared ? 1 : 0);
     if ((long long)num_seqs * max_parts * num_kv_heads >= (1ll << 31))
         return fail(PA_ERR_UNSUPPORTED, "too many work units");
-    if (max_parts >= pa::MAX_PARTS_LIMIT || max_context_len >= pa::MAX_TOKENS_LIMIT)
-        return fail(PA_ERR_UNSUPPORTED, "%d partitions of a sequence or %d tokens: above the work-list encoding",
-                    max_parts, max_context_len);
     const pa::WsLayout L = pa::ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_parts, shared);
     if (workspace_bytes < L.total)
         return fail(PA_ERR_INVALID, "workspace %zu bytes < %zu needed", workspace_bytes, L.total);
@@ -224,7 +219,6 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     p.num_blocks = num_blocks;
     p.ctx_limit = ctx_limit;
     p.partition = P;
-    p.fine = F;
     p.max_parts = max_parts;
     p.qscale = scale * 1.4426950408889634f * k_scale;
     p.v_scale = v_scale;

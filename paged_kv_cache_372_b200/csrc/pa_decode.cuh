@@ -43,13 +43,12 @@ struct DecodeParams {
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks;
     int ctx_limit;   // context lengths are clamped to [0, ctx_limit]
     int partition;   // P, tokens per partition
-    int fine;        // tokens of the units that end each sequence (P when not finer; divides P)
-    int max_parts;   // partitions of the longest sequence (partial slots per sequence)
+    int max_parts;   // ceil(ctx_limit / P)
     float qscale;    // scale * log2(e) (times k_scale for an fp8 cache)
     float v_scale;   // fp8 cache: dequantisation scale of V (1 otherwise)
     int *counter;    // work-list cursor (reset by the plan kernel)
     int *num_entries;
-    int4 *entries;   // {seq, unit_pos(partition, first token), tokens, partitions of seq}
+    int4 *entries;   // {seq, partition, tokens, partitions of seq}
     float2 *ml;      // [seq][head][part] (max in log2 units, sum of weights)
     float *part_acc; // [seq][head][part][D] unnormalised outputs
     int *merge_count;// [seq][kv head] finished partitions
@@ -102,31 +101,6 @@ __device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, boo
     return c;
 }
 
-// A work-list entry's second word: the partition index (partial slot) in the
-// top 12 bits and the unit's first token / 16 in the low 20.
-__host__ __device__ __forceinline__ int unit_pos(int part, int tok0) {
-    return (int)(((unsigned)part << 20) | ((unsigned)tok0 >> 4));
-}
-__device__ __forceinline__ int unit_part(int pos) { return (int)((unsigned)pos >> 20); }
-__device__ __forceinline__ int unit_tok0(int pos) { return (int)(((unsigned)pos & 0xfffffu) << 4); }
-constexpr int MAX_PARTS_LIMIT = 1 << 12;   // partitions per sequence the entry encodes
-constexpr int MAX_TOKENS_LIMIT = 1 << 24;  // first tokens the entry encodes
-
-// How a sequence of ctx tokens is cut: `coarse` units of P tokens, then the
-// remaining 1..P tokens as `nf` units of `fine` tokens, the last of `last`.
-struct Cut {
-    int coarse, nf, last;
-};
-__device__ __forceinline__ Cut cut_sequence(int ctx, int P, int fine) {
-    Cut c{0, 0, 0};
-    if (ctx <= 0) return c;
-    c.coarse = (ctx - 1) / P;
-    const int r = ctx - c.coarse * P;
-    c.nf = (r + fine - 1) / fine;
-    c.last = r - (c.nf - 1) * fine;
-    return c;
-}
-
 // ---- 1. work list -----------------------------------------------------------
 constexpr int PLAN_THREADS = 1024;
 constexpr int PLAN_MAX_BINS = 129;  // tiles per partition <= 128
@@ -139,23 +113,19 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
     // Let the attention kernel launch now; it waits for this grid's results.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int P = p.partition, F = p.fine, tiles = P / 16;
+    const int P = p.partition, tiles = P / 16;
     for (int i = tid; i < PLAN_MAX_BINS; i += PLAN_THREADS) s_bin_count[i] = 0;
     for (int i = tid; i < p.num_seqs * p.num_kv_heads; i += PLAN_THREADS) p.merge_count[i] = 0;
     if (tid == 0) s_carry = 0;
     __syncthreads();
 
-    // Pass 1: each sequence's coarse units (all of P tokens) in sequence
-    // order; histogram of the units that end sequences (F tokens, or fewer).
-    int my_ctx = 0;  // the context of sequence tid, kept for pass 2
+    // Pass 1: full partitions in sequence order; histogram of the tails.
     for (int base = 0; base < p.num_seqs; base += PLAN_THREADS) {
         const int s = base + tid;
         const int ctx = s < p.num_seqs ? clamped_context(p, s, true) : 0;
-        if (base == 0) my_ctx = ctx;
-        const Cut c = cut_sequence(ctx, P, F);
-        if (c.nf > 1) atomicAdd(&s_bin_count[F >> 4], c.nf - 1);
-        if (c.nf > 0) atomicAdd(&s_bin_count[(c.last + 15) >> 4], 1);
-        int incl = c.coarse;
+        const int full = ctx / P, tail = ctx - full * P;
+        if (tail > 0) atomicAdd(&s_bin_count[(tail + 15) >> 4], 1);
+        int incl = full;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(FULL_MASK, incl, o);
@@ -174,11 +144,11 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
             s_warp[lane] = wi - w;
         }
         __syncthreads();
-        const int off = s_carry + s_warp[warp] + incl - c.coarse;
-        const int nparts = c.coarse + c.nf;
-        for (int j = 0; j < c.coarse; ++j) p.entries[off + j] = make_int4(s, unit_pos(j, j * P), P, nparts);
+        const int off = s_carry + s_warp[warp] + incl - full;
+        const int nparts = full + (tail > 0);
+        for (int j = 0; j < full; ++j) p.entries[off + j] = make_int4(s, j, P, nparts);
         __syncthreads();
-        if (tid == PLAN_THREADS - 1) s_carry = off + c.coarse;
+        if (tid == PLAN_THREADS - 1) s_carry = off + full;
         __syncthreads();
     }
     if (tid == 0) {
@@ -191,21 +161,15 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
         *p.counter = 0;
     }
     __syncthreads();
-    // Pass 2: the units that end each sequence, longest first. An empty
-    // sequence gets no work; its output rows are zeroed here.
+    // Pass 2: each sequence's last, partial partition, longest first. An
+    // empty sequence gets no work; its output rows are zeroed here.
     for (int s = tid; s < p.num_seqs; s += PLAN_THREADS) {
-        const int ctx = s < PLAN_THREADS ? my_ctx : clamped_context(p, s, false);
-        const Cut c = cut_sequence(ctx, P, F);
-        const int nparts = c.coarse + c.nf, tok = c.coarse * P;
-        if (c.nf > 1) {
-            const int pos = atomicAdd(&s_bin_next[F >> 4], c.nf - 1);
-            for (int k = 0; k < c.nf - 1; ++k)
-                p.entries[pos + k] = make_int4(s, unit_pos(c.coarse + k, tok + k * F), F, nparts);
-        }
-        if (c.nf > 0) {
-            const int pos = atomicAdd(&s_bin_next[(c.last + 15) >> 4], 1);
-            p.entries[pos] = make_int4(s, unit_pos(nparts - 1, tok + (c.nf - 1) * F), c.last, nparts);
-        } else {
+        const int ctx = clamped_context(p, s, false);
+        const int full = ctx / P, tail = ctx - full * P;
+        if (tail > 0) {
+            const int pos = atomicAdd(&s_bin_next[(tail + 15) >> 4], 1);
+            p.entries[pos] = make_int4(s, full, tail, full + 1);
+        } else if (ctx == 0) {
             const int nvec = p.num_heads * p.head_dim / 8;
             uint4 *row = static_cast<uint4 *>(p.out) + (size_t)s * nvec;
             for (int i = 0; i < nvec; ++i) row[i] = make_uint4(0, 0, 0, 0);
@@ -417,23 +381,23 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
     __syncthreads();
     int off = s_warp[warp] + incl - full;
     for (int j = 0; j < pfull; ++j, ++off) {
-        p.entries[off] = make_int4(m, unit_pos(j, j * P), P, 0);
+        p.entries[off] = make_int4(m, j, P, 0);
         p.entries_b[off] = make_int4(j * P, tid, cnt, 0);
     }
     for (int j = 0; j < sfull; ++j, ++off) {
-        p.entries[off] = make_int4(m, unit_pos(pp + j, S + j * P), P, nparts);
+        p.entries[off] = make_int4(m, pp + j, P, nparts);
         p.entries_b[off] = make_int4(S + j * P, 0, 0, 0);
     }
     // Pass 2: tails; empty sequences get zero output rows.
     if (tid < B) {
         if (stail > 0) {
             const int pos = atomicAdd(&s_bin_next[(stail + 15) >> 4], 1);
-            p.entries[pos] = make_int4(m, unit_pos(pp + sfull, S + sfull * P), stail, nparts);
+            p.entries[pos] = make_int4(m, pp + sfull, stail, nparts);
             p.entries_b[pos] = make_int4(S + sfull * P, 0, 0, 0);
         }
         if (ptail > 0) {
             const int pos = atomicAdd(&s_bin_next[(ptail + 15) >> 4], 1);
-            p.entries[pos] = make_int4(m, unit_pos(pfull, pfull * P), ptail, 0);
+            p.entries[pos] = make_int4(m, pfull, ptail, 0);
             p.entries_b[pos] = make_int4(pfull * P, tid, cnt, 0);
         }
         if (ctx == 0) {
@@ -616,7 +580,7 @@ struct UnitSource {
             state = 2;
         } else if (state == 2) {
             const int nblk = (ent.z + bs - 1) / bs;
-            const int blk0 = unit_tok0(ent.y) / bs;
+            const int blk0 = shared ? entb.x / bs : ent.y * blocks_per_part;
             tbl = lane < nblk ? p->block_tables[(size_t)ent.x * p->max_blocks_per_seq + blk0 + lane] : 0;
             if (shared && lane < entb.z) {
                 mseq = p->members[entb.y + lane];
@@ -634,12 +598,12 @@ struct UnitSource {
         const int e = u / Hkv;
         x.kvh = u - e * Hkv;
         x.s = ent.x;
-        x.part = unit_part(ent.y);
+        x.part = ent.y;
         x.ntok = ent.z;
         x.nparts = ent.w;
         x.ntiles = (ent.z + 15) >> 4;
         x.tbl = tbl;
-        x.tok0 = unit_tok0(ent.y);
+        x.tok0 = shared ? entb.x : ent.y * p->partition;
         x.mcnt = shared ? entb.z : 0;
         x.mseq = mseq;
         x.mnp = mnp;

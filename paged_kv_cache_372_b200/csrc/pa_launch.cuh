@@ -56,19 +56,6 @@ int resolve_partition(int group, int block_size, int max_context_len, int reques
     return auto_p;
 }
 
-// Tokens of the units that end each sequence. The plans can cut a
-// sequence's last up to P tokens into finer units (the work list then ends
-// in small units); measured on the benchmark workloads (P/2, P/4) the extra
-// merges cost as much as the finer balance gains, so the end units are P.
-int fine_partition(int P, int /*block_size*/, PartMode /*mode*/) { return P; }
-
-// Partial slots per sequence: its coarse units plus up to P / F end units,
-// plus one where shared-prefix units cut at the end of the shared blocks.
-int parts_per_sequence(int max_context_len, int P, int F, bool shared) {
-    const int base = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
-    return base + (P / F - 1) + (shared ? 1 : 0);
-}
-
 template <int D, int G, typename T>
 pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
     constexpr int NS = pa::DECODE_STAGES;

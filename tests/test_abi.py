@@ -72,13 +72,3 @@ def test_shared_decode_host_checks_without_a_device():
     # more sequences than the grouping takes
     assert lib.pa_decode_shared(*args, 1025, *rest) == pa.PA_ERR_UNSUPPORTED
     assert b"1024" in lib.pa_last_error()
-
-
-def test_decode_rejects_sizes_beyond_the_work_list_encoding():
-    lib = pa.lib()
-    dummy = ctypes.c_void_p(256)
-    # 2^24 tokens of context in 512-token partitions: 32768 partitions of a sequence
-    st = lib.pa_decode(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 8, 128, 16, 1 << 20, 1 << 20, 1 << 24,
-                       ctypes.c_float(0.1), 0, 512, dummy, 1 << 40, None)
-    assert st == pa.PA_ERR_UNSUPPORTED
-    assert b"encoding" in lib.pa_last_error()
