@@ -72,3 +72,47 @@ def test_shared_decode_host_checks_without_a_device():
     # more sequences than the grouping takes
     assert lib.pa_decode_shared(*args, 1025, *rest) == pa.PA_ERR_UNSUPPORTED
     assert b"1024" in lib.pa_last_error()
+
+
+def _header_declarations():
+    import re
+    with open(pa.HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    decls = {}
+    for m in re.finditer(r"PA_API\s+([\w\s\*]+?)\s*\b(pa_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = [x.strip() for x in m.group(3).split(",") if x.strip() and x.strip() != "void"]
+        decls[m.group(2)] = (m.group(1).strip(), params)
+    return decls
+
+
+def _ctypes_kind(c_type: str):
+    t = c_type.replace("const", "").strip()
+    if "*" in t or t.startswith("pa_stream_t"):
+        return "pointer"
+    t = t.split()[:-1] if len(t.split()) > 1 else t.split()
+    base = " ".join(t)
+    return {"int": "int", "pa_dtype": "int", "pa_status": "int", "float": "float", "size_t": "u64",
+            "unsigned long long": "u64", "unsigned int": "uint"}[base]
+
+
+def test_binding_signatures_match_header():
+    """Every function the header declares is set up in the binding with the
+    same number and kinds of arguments (a mismatch would pass garbage)."""
+    lib = pa.lib()
+    # size_t and unsigned long long are both 64-bit unsigned here (one ctypes class)
+    kinds = {ctypes.c_int: "int", ctypes.c_float: "float", ctypes.c_size_t: "u64",
+             ctypes.c_ulonglong: "u64", ctypes.c_uint: "uint", ctypes.c_void_p: "pointer",
+             ctypes.c_char_p: "pointer"}
+    decls = _header_declarations()
+    assert set(decls) == set(pa.header_functions())
+    for name, (ret, params) in decls.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, f"{name}: argtypes not set in the binding"
+        assert len(fn.argtypes) == len(params), f"{name}: {len(fn.argtypes)} argtypes, header has {len(params)}"
+        for i, (a, p) in enumerate(zip(fn.argtypes, params)):
+            got = "pointer" if hasattr(a, "_type_") and a not in kinds else kinds.get(a)
+            if a not in kinds and isinstance(a, type) and issubclass(a, ctypes._Pointer):
+                got = "pointer"
+            assert got == _ctypes_kind(p), f"{name} argument {i} ({p}): binding has {a}"
