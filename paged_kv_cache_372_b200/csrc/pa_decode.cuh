@@ -103,6 +103,7 @@ __device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, boo
 
 // ---- 1. work list -----------------------------------------------------------
 constexpr int PLAN_THREADS = 1024;
+static_assert(PLAN_THREADS % 32 == 0 && PLAN_THREADS <= 1024, "plan block: whole warps, at most 32");
 constexpr int PLAN_MAX_BINS = 129;  // tiles per partition <= 128
 
 __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParams p) {
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParam
         if (lane == 31) s_warp[warp] = incl;
         __syncthreads();
         if (warp == 0) {
-            const int w = s_warp[lane];
+            const int w = lane < PLAN_THREADS / 32 ? s_warp[lane] : 0;  // warps of the block only
             int wi = w;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
     if (lane == 31) s_warp[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const int w = s_warp[lane];
+        const int w = lane < PLAN_THREADS / 32 ? s_warp[lane] : 0;  // warps of the block only
         int wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
