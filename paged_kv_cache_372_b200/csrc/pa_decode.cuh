@@ -231,16 +231,18 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
         key = ((unsigned long long)(unsigned)b0 << 32) | (unsigned)tid;
     }
     // Bitonic sort, one key per thread: strides below 32 by shuffles within
-    // the warp, larger ones through shared memory.
+    // the warp (only the warps that hold keys), larger ones through shared
+    // memory (every thread takes the block barriers).
+    const bool keyed_warp = warp * 32 < n;
     for (int k = 2; k <= n; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
-            unsigned long long other;
+            unsigned long long other = key;
             if (j >= 32) {
                 __syncthreads();
                 if (tid < n) s_key[tid] = key;
                 __syncthreads();
-                other = tid < n ? s_key[tid ^ j] : key;
-            } else {
+                if (tid < n) other = s_key[tid ^ j];
+            } else if (keyed_warp) {
                 other = __shfl_xor_sync(FULL_MASK, key, j);
             }
             const bool up = (tid & k) == 0, lower = (tid & j) == 0;
@@ -275,8 +277,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
     __syncthreads();
     // Leading blocks each position shares with its sub-group's first member:
     // one warp per position, two positions per round (positions i and i + 32
-    // of a warp's stripe), 2 x 32 table entries of each row per load batch,
-    // so that B <= 64 costs one dependent round trip.
+    // of a warp's stripe), 4 x 32 table entries of each row per load batch,
+    // so that B <= 64 with shared prefixes up to 128 blocks costs one
+    // dependent round trip.
     for (int i0 = warp; i0 < B; i0 += 2 * (PLAN_THREADS / 32)) {
         int lcp[2], lim[2];
         const int *tm[2], *tl[2];
@@ -294,12 +297,12 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
             tm[h] = p.block_tables + (size_t)m * W;
             tl[h] = p.block_tables + (size_t)l * W;
         }
-        for (int j0 = 0; j0 < max(lim[0], lim[1]); j0 += 64) {
-            int a[2][2], b[2][2];
+        for (int j0 = 0; j0 < max(lim[0], lim[1]); j0 += 128) {
+            int a[2][4], b[2][4];
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
+                for (int r = 0; r < 4; ++r) {
                     const int j = j0 + 32 * r + lane;
                     const bool in = j < lim[h] && lcp[h] == lim[h];
                     a[h][r] = in ? tm[h][j] : 0;
@@ -309,7 +312,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
             for (int h = 0; h < 2; ++h) {
                 if (lcp[h] != lim[h] || !todo[h]) continue;  // decided (uniform across the warp)
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
+                for (int r = 0; r < 4; ++r) {
                     const unsigned d = __ballot_sync(FULL_MASK, a[h][r] != b[h][r]);
                     if (d && lcp[h] == lim[h]) lcp[h] = j0 + 32 * r + __ffs(d) - 1;
                 }
