@@ -4,19 +4,26 @@
 //     and writes the work list, longest partitions first, so that the
 //     persistent attention kernel finishes with the short ones. It also
 //     zeroes the per-(sequence, KV head) merge counters.
-//  2. pa_decode_kernel (one persistent CTA per SM, launched with programmatic
-//     dependent launch so its set-up overlaps the plan) — every warp is an
-//     independent worker. It takes (sequence, KV head, partition) units from
-//     the work list with an atomic counter and streams the unit's 16-token K
-//     and V tiles, each one contiguous chunk of the pool, through a private
-//     ring of shared-memory stages filled by 1-D bulk copies (TMA) that
-//     complete on mbarriers; K and V tiles alternate. The block-table entries
-//     of a unit are loaded once into lane registers and handed to the
-//     copy-issuing lane by a shuffle. Per tile: scores of the G query heads
-//     of the KV head, online softmax, weighted sum of the values. A unit that
-//     is a whole sequence writes the normalised output; otherwise it writes
-//     (max, sum, unnormalised output) partials, and the last warp to finish a
-//     (sequence, KV head) merges its partitions by the log-sum-exp identity.
+//     pa_plan_shared_kernel does the same for pa_decode_shared, after
+//     grouping sequences whose tables begin with the same blocks.
+//  2. The attention kernel (one persistent CTA per SM, launched with
+//     programmatic dependent launch so its set-up overlaps the plan) — every
+//     warp is an independent worker. It takes (sequence, KV head, partition)
+//     units from the work list with an atomic counter and streams the unit's
+//     16-token K and V tiles through a private ring of shared-memory stages
+//     filled by TMA copies that complete on mbarriers. The block-table
+//     entries of a unit are loaded once into lane registers and handed to
+//     the copy-issuing lane by a shuffle. Per tile: scores of the G query
+//     heads of the KV head, online softmax, weighted sum of the values. A
+//     unit that is a whole sequence writes the normalised output; otherwise
+//     it writes (max, sum, unnormalised output) partials, and the last warp
+//     to finish a (sequence, KV head) merges its partitions by the
+//     log-sum-exp identity.
+//     The default attention kernel is the tensor-core one in
+//     pa_decode_mma.cuh. This file holds the CUDA-core kernel
+//     (pa_decode_kernel: 1-D bulk copies of each tile, FFMA2 dot products),
+//     selected with -DPA_DECODE_TENSOR_MIN_GROUP, plus what both share: the
+//     plans, the unit source and the merges.
 
 // The arithmetic is the definition in "别再让GPU内存拖后腿了：vLLM的PagedAttention
 // 如何像操作系统一样管理KV Cache", section 3.1: scores of the query against every
@@ -531,8 +538,9 @@ struct Unit {
 // Hands out work-list units to one warp. Claiming a unit is a chain of three
 // dependent global accesses (atomic cursor -> work-list entry -> the unit's
 // block-table slice, one entry per lane); step() advances the chain for the
-// next unit by one link, so that called once per issued tile it has the next
-// unit ready before the warp needs it, and take() only finishes what is left.
+// next unit by one link, so that called once per issued tile (the CUDA-core
+// kernel) or over a unit's last tiles (the tensor-core kernel) it has the
+// next unit ready before the warp needs it; take() only finishes what is left.
 // The first claims of a launch arrive about in CTA order, all at once, so
 // in a longest-first list the first CTAs would take only long units and the
 // last ones only short ones. Claims below `wave1` (a multiple of the warps

@@ -15,6 +15,11 @@
 // (movmatrix). Scores, softmax state and O^T stay in fp32; P is rounded to the
 // input type for the second product and the softmax denominator sums the
 // same rounded values.
+//
+// Variants (template flags): KV8 reads an E4M3 cache (byte tiles widened to
+// f16 in registers, 16 warps per CTA for head groups up to 4); SHARED lets a
+// unit serve up to 8 / G sequences that share the unit's blocks, their G
+// query rows each filling the MMA's 8 columns (pa_decode_shared).
 #pragma once
 
 #include <cuda.h>
