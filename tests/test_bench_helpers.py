@@ -1,0 +1,51 @@
+"""Host-side helpers of bench.py (CPU only): the kernel-source digest that
+keys the committed traffic figures, the L2-flush rule and the shape options."""
+import os
+import sys
+import types
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+
+
+def test_code_only_drops_comments_and_blank_space_but_keeps_code():
+    a = 'int a = 1; // note\n/* block\n comment */ int b = "s//t";\n'
+    b = 'int a = 1;\n\n  int b = "s//t"; // another note\n'
+    assert bench.code_only(a) == bench.code_only(b) == 'int a = 1; int b = "s//t";'
+    assert bench.code_only("int a = 1;") != bench.code_only("int a = 2;")
+    assert bench.code_only('x = "/* not a comment */";') == 'x = "/* not a comment */";'
+
+
+def test_source_digest_is_stable_and_covers_the_kernel_files():
+    d = bench.source_digest()
+    assert len(d) == 16 and d == bench.source_digest()
+    csrc = os.path.join(bench.ROOT, "paged_kv_cache_372_b200", "csrc")
+    for name in bench.KERNEL_SOURCES:
+        assert os.path.exists(os.path.join(csrc, name))
+
+
+def test_committed_traffic_matches_the_current_kernels():
+    # every committed entry names the digest of the sources it was captured on
+    import json
+    with open(bench.PROFILE_TRAFFIC) as f:
+        entries = {k: v for k, v in json.load(f).items() if isinstance(v, dict)}
+    assert entries
+    for key, e in entries.items():
+        assert e["dram_bytes_per_launch"] > 0
+        assert os.path.exists(os.path.join(os.path.dirname(bench.PROFILE_TRAFFIC), e["summary"]))
+        if e["source_digest"] == bench.source_digest():
+            assert bench.profiled_traffic(key) == e["dram_bytes_per_launch"]
+
+
+def test_shape_options_only_for_the_decode_batches():
+    args = types.SimpleNamespace(block_size=32, head_dim=None, workload="llama7b")
+    assert bench.shape_args(args) == {"block_size": 32}
+    args = types.SimpleNamespace(block_size=None, head_dim=64, workload="llama3_8b")
+    assert bench.shape_args(args) == {"head_dim": 64}
+    args = types.SimpleNamespace(block_size=32, head_dim=None, workload="beam")
+    try:
+        bench.shape_args(args)
+    except SystemExit:
+        pass
+    else:
+        raise AssertionError("beam takes no block-size option")
