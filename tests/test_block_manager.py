@@ -181,3 +181,57 @@ def test_beam256_workload_forks_every_beam():
         assert not (set(dst.tolist()) & set(st.copy_pairs[:, 0].tolist()))
     # first step: 8 parents per group, each forked 4 ways -> 3 copies per parent with a partial tail
     assert 0 < len(wl.steps[0].copy_pairs) <= 2 * 8 * 3
+
+
+def _check_decode_batch(wl, B, H, Hkv, D, bs, dtype, lo, hi):
+    st = wl.steps[0]
+    assert (wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, wl.dtype) == (H, Hkv, D, bs, dtype)
+    assert st.q.shape == (B, H, D) and st.k_new.shape[1:] == (Hkv, D)
+    ctx = st.context_lens
+    assert ctx.shape == (B,) and ctx.min() >= lo and ctx.max() <= hi
+    need = sum(-(-int(c) // bs) for c in ctx)
+    assert wl.num_blocks >= 1.25 * need - 1          # pool 1.25x what the tables hold
+    used = st.block_tables[st.block_tables >= 0]
+    assert len(set(used.tolist())) == len(used)      # no block is shared in a decode batch
+    for s in range(B):
+        n = int(ctx[s])
+        assert (st.block_tables[s, :-(-n // bs)] >= 0).all()
+        assert st.slot_mapping[s] == st.block_tables[s, (n - 1) // bs] * bs + (n - 1) % bs
+    return ctx
+
+
+def test_decode_batches_follow_the_recipe():
+    ctx = _check_decode_batch(workloads.llama7b(0), 64, 32, 32, 128, 16, "f16", 128, 2048)
+    assert 700 < ctx.mean() < 1400                   # uniform on [128, 2048]
+    ctx = _check_decode_batch(workloads.llama3_8b(0), 256, 32, 8, 128, 16, "bf16", 16, 8192)
+    assert 350 < np.median(ctx) < 750                # lognormal, median 512
+    # the same batches at another block size or head size (same contexts)
+    wl = workloads.llama7b(0, block_size=32, head_dim=64)
+    assert wl.name == "llama7b_bs32_d64"
+    _check_decode_batch(wl, 64, 32, 32, 64, 32, "f16", 128, 2048)
+    assert np.array_equal(wl.steps[0].context_lens, workloads.llama7b(0).steps[0].context_lens)
+
+
+def test_beam_groups_share_their_prefix():
+    """Every step of the beam workload: the sequences of a group hold the same
+    64 leading blocks (the 1024-token prefix), which is what shared-prefix
+    decode finds and streams once per group."""
+    wl = workloads.beam(0, groups=4, steps=2)
+    for st in wl.steps:
+        first = st.block_tables[:, 0]
+        groups = {}
+        for s, b in enumerate(first.tolist()):
+            groups.setdefault(b, []).append(s)
+        assert len(groups) == 4 and all(len(m) == 8 for m in groups.values())
+        for members in groups.values():
+            lead = st.block_tables[members[0]]
+            for s in members[1:]:
+                row = st.block_tables[s]
+                lcp = 0
+                while row[lcp] == lead[lcp]:
+                    lcp += 1
+                assert lcp >= 64
+                # the block holding the sequence's newest token is its own
+                n = int(st.context_lens[s])
+                others = st.block_tables[[m for m in range(len(first)) if m != s]]
+                assert row[(n - 1) // 16] not in set(others[others >= 0].tolist())
