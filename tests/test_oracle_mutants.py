@@ -53,6 +53,11 @@ MUTATIONS = {
                                 "o[d] += scores[t] * oracle_e4m3_to_double(val[d]);"),
     "fp8_write_scale_times": ("k_pool[dst + d] = oracle_e4m3_encode(kx / k_scale);",
                               "k_pool[dst + d] = oracle_e4m3_encode(kx * k_scale);"),
+    "negative_slot_stops_the_write": (
+        "int num_kv_heads, int head_dim, int block_size)\n{\n    for (int t = 0; t < num_tokens; t++) {\n"
+        "        const int64_t slot = slot_mapping[t];\n        if (slot < 0)\n            continue;",
+        "int num_kv_heads, int head_dim, int block_size)\n{\n    for (int t = 0; t < num_tokens; t++) {\n"
+        "        const int64_t slot = slot_mapping[t];\n        if (slot < 0)\n            break;"),
     "slot_offset": ("slots[i] = (int64_t)table[pos / block_size] * block_size + pos % block_size;",
                     "slots[i] = (int64_t)table[pos / block_size] * block_size + (pos + 1) % block_size;"),
 }
