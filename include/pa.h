@@ -75,6 +75,7 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_SLOT     4u   /* slot_mapping entry >= num_blocks*block_size */
 #define PA_DEVERR_PAIR     8u   /* copy pair id outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT 16u   /* a bounded device-side wait ran out */
+#define PA_DEVERR_QRANGE  32u   /* pa_decode_fp8: a bf16 query element above 65504 in magnitude */
 
 /* Opaque CUDA stream handle (cudaStream_t). */
 typedef void *pa_stream_t;
@@ -213,7 +214,9 @@ PA_API size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int n
  * by `dtype`). k_pool, v_pool: uint8 codes [num_blocks][num_kv_heads]
  * [block_size][head_dim], written by pa_reshape_and_cache_fp8. head_dim 128.
  * The products run on tensor cores with the codes widened to fp16 (exact) and
- * the queries converted to fp16 (exact for |q| in fp16's normal range). The
+ * the queries converted to fp16 (exact for |q| in fp16's normal range; a bf16
+ * query element above 65504 in magnitude has no fp16 value: the kernel sets
+ * PA_DEVERR_QRANGE and that head's output is undefined). The
  * workspace is sized by pa_decode_fp8_workspace_size: partition_size 0 picks
  * 512 tokens for one query head per KV head and max(256 tokens, 8 blocks)
  * otherwise (pa_decode_fp8_partition_size).
@@ -350,9 +353,11 @@ PA_API pa_status pa_selftest_bounded_wait(unsigned long long limit_ns, pa_stream
  * Sizes whose pa_decode_workspace_size() exceeds the array are rejected with
  * PA_ERR_UNSUPPORTED before anything is launched (pa_last_error() says why).
  *
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture. All calls share the one array: calls that overlap on the GPU
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress; nothing is cached, so the address stays valid after
+ * a device reset or a new primary context). The first call on a device may
+ * load the library's device code there: make it before any stream capture.
+ * All calls share the one array: calls that overlap on the GPU
  * (different streams, or different host threads without ordering) race and
  * give undefined results. Calls ordered on one stream are safe; each call
  * re-initialises the parts of the array that must start at zero.

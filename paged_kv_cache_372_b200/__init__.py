@@ -21,7 +21,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "pa.h")
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK = range(5)
 PA_F16, PA_BF16 = 0, 1
-DEVERR_BLOCK_ID, DEVERR_CONTEXT, DEVERR_SLOT, DEVERR_PAIR, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
+DEVERR_BLOCK_ID, DEVERR_CONTEXT, DEVERR_SLOT, DEVERR_PAIR, DEVERR_TIMEOUT, DEVERR_QRANGE = 1, 2, 4, 8, 16, 32
 
 _DTYPES = {torch.float16: PA_F16, torch.bfloat16: PA_BF16}
 

@@ -97,13 +97,15 @@ __device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t codes) {
 }
 
 // Two 16-bit query elements of type T -> f16x2 (bf16 -> f16 is exact in f16's
-// normal range, which decode queries stay within).
+// normal range). A bf16 element above f16's largest finite value (65504)
+// would become infinite: `big` is set so that the caller can flag it.
 template <typename T>
-__device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
+__device__ __forceinline__ uint32_t to_f16x2(uint32_t w, bool &big) {
     if constexpr (std::is_same<T, __half>::value) {
         return w;
     } else {
         const float2 f = Elem<T>::pair(w);
+        big |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
         return Elem<__half>::pack(f.x, f.y);
     }
 }
@@ -484,6 +486,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             const uint32_t vs_s = ks_s + Gm::HALF_BYTES;
             if (k == 0) {
                 const uint8_t *qs = qbuf + cur.slot * QB;
+                bool qbig = false;  // a bf16 query element outside f16's range (fp8 cache)
 #pragma unroll
                 for (int i = 0; i < Gm::KS; ++i) {
                     if constexpr (KV8) {
@@ -491,16 +494,20 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                         // (the order the byte-wise fragments arrive in); the
                         // query fragment follows the same order.
                         const int d = 16 * i + 4 * t4;
-                        qb[i][0] = g8 < nrows ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2))
-                                              : 0u;
-                        qb[i][1] = g8 < nrows
-                                       ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 2) * 2))
+                        qb[i][0] = g8 < nrows
+                                       ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2), qbig)
                                        : 0u;
+                        qb[i][1] = g8 < nrows ? to_f16x2<T>(
+                                                    *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 2) * 2), qbig)
+                                              : 0u;
                     } else {
                         const int d = 16 * i + 2 * t4;
                         qb[i][0] = g8 < nrows ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
                         qb[i][1] = g8 < nrows ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 8) * 2) : 0u;
                     }
+                }
+                if constexpr (KV8 && !std::is_same<T, __half>::value) {
+                    if (__any_sync(FULL_MASK, qbig) && lane == 0) raise_error(PA_DEVERR_QRANGE);
                 }
             }
             const int valid = min(16, cur.ntok - 16 * k);

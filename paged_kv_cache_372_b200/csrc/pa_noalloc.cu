@@ -12,7 +12,6 @@
 // The array is PA_NOALLOC_SCRATCH_BYTES (16 MiB). Every GPU that loads this
 // library holds it until the process exits.
 #include <cstdio>
-#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -25,10 +24,6 @@ namespace {
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void *g_scratch[kMaxDevices];  // device address of g_noalloc_scratch, per device
-
 }  // namespace
 
 extern "C" pa_status pa_decode_noalloc(void *out, const void *q, const void *k_pool, const void *v_pool,
@@ -36,34 +31,6 @@ extern "C" pa_status pa_decode_noalloc(void *out, const void *q, const void *k_p
                                        int num_heads, int num_kv_heads, int head_dim, int block_size,
                                        int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
                                        int dtype, int partition_size, pa_stream_t stream) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) {
-        pa_internal_set_last_error(cudaGetErrorString(e));
-        return PA_ERR_CUDA;
-    }
-    if (dev < 0 || dev >= kMaxDevices) {
-        pa_internal_set_last_error("device index out of range");
-        return PA_ERR_CUDA;
-    }
-    void *scratch = nullptr;
-    {
-        // First call on this device: look up the array's device address with
-        // the device current. Host code cannot use the array's name as an
-        // address; only this lookup gives one.
-        std::lock_guard<std::mutex> lock(g_mutex);
-        if (!g_scratch[dev]) {
-            void *ptr = nullptr;
-            e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-            if (e != cudaSuccess || !ptr) {
-                pa_internal_set_last_error(e != cudaSuccess ? cudaGetErrorString(e)
-                                                            : "cudaGetSymbolAddress returned null");
-                return PA_ERR_CUDA;
-            }
-            g_scratch[dev] = ptr;
-        }
-        scratch = g_scratch[dev];
-    }
     const size_t need = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                                  max_context_len, partition_size);
     if (need > (size_t)PA_NOALLOC_SCRATCH_BYTES) {
@@ -74,6 +41,17 @@ extern "C" pa_status pa_decode_noalloc(void *out, const void *q, const void *k_p
                  need, (size_t)PA_NOALLOC_SCRATCH_BYTES);
         pa_internal_set_last_error(msg);
         return PA_ERR_UNSUPPORTED;
+    }
+    // The array's device address on the current device. Host code cannot use
+    // the array's name as an address; only this lookup gives one. It runs on
+    // every call rather than being cached, so that the address stays right
+    // after a device reset or a new primary context (which reload the module
+    // at another address); once the module is loaded it is a host-side lookup.
+    void *scratch = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+    if (e != cudaSuccess || !scratch) {
+        pa_internal_set_last_error(e != cudaSuccess ? cudaGetErrorString(e) : "cudaGetSymbolAddress returned null");
+        return PA_ERR_CUDA;
     }
     // pa_decode's plan kernel re-initialises everything in the scratch that
     // must start from zero (work-list cursor, merge counters) on every call.

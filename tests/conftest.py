@@ -20,3 +20,12 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    from tests import margins
+    lines = margins.summary_lines()
+    if lines:
+        terminalreporter.write_sep("-", "attention max-abs error against the oracle / tolerance (worst per case)")
+        for line in lines:
+            terminalreporter.write_line(line)

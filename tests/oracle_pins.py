@@ -7,7 +7,8 @@ mistake each (at least one pin must fail for every copy).
 
 What pins what:
   * element decoding      all 65536 patterns vs numpy float16 / float32 types
-  * paged attention       numpy contiguous-cache brute force; torch SDPA (fp64);
+  * paged attention       numpy contiguous-cache brute force; torch SDPA (fp64),
+                          on fixed shapes and on seeded random tiny shapes;
                           closed forms (1 token -> its V row; equal keys or
                           scale 0 -> mean of V; a 2-token case with weights
                           1/(1+e) and e/(1+e)); invariants (physical block
@@ -106,6 +107,35 @@ def pin_sdpa(orc, seed=1):
         got = orc.paged_attention(q, kp, vp, tab, cl, scale, dt)
         ref = sdpa_attention(decode(q, dt), decode(kp, dt), decode(vp, dt), tab, cl, scale)
         assert np.abs(got - ref).max() <= ATOL
+
+
+def random_shapes(rng, n):
+    """n seeded random tiny shapes: 1-4 sequences with contexts in [0, 80)
+    (empty ones included), 1-3 KV heads with groups of 1-4 query heads, head
+    sizes 8-64, block sizes 1-32, fp16 or bf16."""
+    shapes = []
+    for _ in range(n):
+        B = int(rng.integers(1, 5))
+        Hkv = int(rng.integers(1, 4))
+        G = int(rng.choice([1, 2, 3, 4]))
+        D = int(rng.choice([8, 16, 24, 64]))
+        bs = int(rng.choice([1, 2, 4, 8, 16, 32]))
+        ctx = [int(c) for c in rng.integers(0, 80, B)]
+        shapes.append((B, G * Hkv, Hkv, D, bs, ctx, str(rng.choice(["f16", "bf16"]))))
+    return shapes
+
+
+def pin_random_shapes(orc, seed=15, n=24):
+    """The oracle against the numpy brute force and torch SDPA on seeded random
+    tiny shapes, each with its own random scale."""
+    rng = np.random.default_rng(seed)
+    for B, H, Hkv, D, bs, ctx, dt in random_shapes(rng, n):
+        q, kp, vp, tab, cl = _case(rng, B, H, Hkv, D, bs, ctx, dt)
+        scale = float(rng.uniform(0.1, 2.0)) / math.sqrt(D)
+        got = orc.paged_attention(q, kp, vp, tab, cl, scale, dt)
+        args = (decode(q, dt), decode(kp, dt), decode(vp, dt), tab, cl, scale)
+        for ref in (contiguous_attention(*args), sdpa_attention(*args)):
+            assert np.abs(got - ref).max() <= ATOL, (B, H, Hkv, D, bs, ctx, dt)
 
 
 def pin_single_token(orc, seed=2):
@@ -369,7 +399,7 @@ def pin_slot_mapping(orc, seed=10):
     assert np.array_equal(got, np.array(want, dtype=np.int64))
 
 
-ALL_PINS = [pin_decode_f16, pin_decode_bf16, pin_bruteforce, pin_sdpa, pin_single_token,
+ALL_PINS = [pin_decode_f16, pin_decode_bf16, pin_bruteforce, pin_sdpa, pin_random_shapes, pin_single_token,
             pin_equal_keys, pin_two_token_closed_form, pin_block_permutation,
             pin_shared_equals_duplicated, pin_tail_slots_ignored, pin_gqa_mapping,
             pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_swap_blocks, pin_slot_mapping,

@@ -49,3 +49,19 @@ def test_shape_options_only_for_the_decode_batches():
         pass
     else:
         raise AssertionError("beam takes no block-size option")
+
+
+def test_cpu_baseline_and_reference_arm_time_the_same_sample():
+    """Both arms run the oracle over the same bounded sample of the workload and
+    report the same config keys."""
+    from paged_kv_cache_372_b200 import workloads
+    wl = workloads.tiny(0)
+    cb = bench.cpu_baseline(wl, repeats=1)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["kv_gbs"] > 0
+    assert cb["cores_1"]["seqs_per_s"] > 0 and cb["cores_all"]["seqs_per_s"] == cb["value"]
+    args = types.SimpleNamespace(workload="tiny", seed=0, steps=2, warmup=1, gpus=1, block_size=None,
+                                 head_dim=None)
+    ref = bench.run_reference(args, 1, 0)
+    assert ref["impl"] == "reference" and ref["config"] == bench.describe(wl)
+    n = min(wl.num_seqs, bench.ORACLE_SAMPLE_SEQS)
+    assert cb["sample"].startswith(f"{n} of ") and ref["cpu_baseline"]["sample"].startswith(f"{n} of ")

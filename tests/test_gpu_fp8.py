@@ -11,6 +11,7 @@ import torch
 import oracle
 import paged_kv_cache_372_b200 as pa
 from paged_kv_cache_372_b200 import workloads
+from tests import margins
 from tests.bruteforce import bits_of
 
 pytestmark = pytest.mark.gpu
@@ -58,6 +59,7 @@ def test_fp8_decode_matches_oracle(name, kw):
     ref = oracle_decode(wl, k8, v8)
     err = float(np.abs(out.float().cpu().double().numpy() - ref).max())
     assert err <= TOL[wl.dtype], err
+    margins.record(f"fp8 {name} {wl.dtype} B={wl.num_seqs}", err, TOL[wl.dtype])
 
 
 @pytest.mark.parametrize("partition", [16, 64, 256])
@@ -131,3 +133,20 @@ def test_fp8_rejects_unsupported_head_dim():
         pa.pa_decode_fp8(torch.empty_like(st.q).cuda(), st.q.cuda(), k8, k8,
                          torch.as_tensor(st.block_tables).cuda(), torch.as_tensor(st.context_lens).cuda(),
                          wl.scale, 33, K_SCALE, V_SCALE)
+
+
+def test_fp8_flags_bf16_queries_outside_f16_range():
+    """The fp8 kernel multiplies in f16: a bf16 query element above 65504 in
+    magnitude has no f16 value, so the kernel flags it (DEVERR_QRANGE) instead
+    of returning NaN silently. In-range queries raise nothing."""
+    wl = workloads.llama3_8b(36, num_seqs=4)
+    k8, v8 = fp8_pools(wl)
+    st = wl.steps[0]
+    q = st.q.clone()
+    q[2, 5, 17] = 1.0e5                           # representable in bf16, not in f16
+    out = torch.empty_like(q).cuda()
+    pa.pa_decode_fp8(out, q.cuda(), k8.cuda(), v8.cuda(), torch.from_numpy(st.block_tables).cuda(),
+                     torch.from_numpy(st.context_lens).cuda(), wl.scale, int(st.context_lens.max()),
+                     K_SCALE, V_SCALE)
+    assert pa.pa_device_errors(clear=True) == pa.DEVERR_QRANGE
+    run_decode(wl, k8, v8)                         # the unmodified queries flag nothing

@@ -11,11 +11,12 @@ import torch
 import paged_kv_cache_372_b200 as pa
 from paged_kv_cache_372_b200 import workloads
 from tests import gpu_harness as H
+from tests import margins
 
 pytestmark = pytest.mark.gpu
 
 
-def run_and_compare(wl, partition_size=None, steps=None):
+def run_and_compare(wl, partition_size=None, steps=None, label=None):
     kp, vp = H.to_gpu(wl)
     okp, ovp = H.oracle_state(wl)
     errs = []
@@ -28,6 +29,8 @@ def run_and_compare(wl, partition_size=None, steps=None):
         err = H.max_err(out, ref)
         errs.append(err)
         assert err <= H.TOL[wl.dtype], (wl.name, i, err)
+    P = wl.partition_size if partition_size is None else partition_size
+    margins.record(label or f"{wl.name} {wl.dtype} B={wl.num_seqs} P={P or 'auto'}", max(errs), H.TOL[wl.dtype])
     return errs
 
 
@@ -100,7 +103,7 @@ def test_shapes(shape, block_size):
                                 inputs.normal((nb, hkv, block_size, D), dtype, gen),
                                 inputs.normal((nb, hkv, block_size, D), dtype, gen), [st])
         for P in (0, block_size * max(1, 64 // block_size)):
-            run_and_compare(wl, partition_size=P)
+            run_and_compare(wl, partition_size=P, label=f"shapes D={D} G={G} bs={block_size} {dtype} P={P or 'auto'}")
 
 
 @pytest.mark.parametrize("name,kw", [("tiny", {}), ("llama7b", {"num_seqs": 8}), ("llama3_8b", {"num_seqs": 16}),
@@ -122,4 +125,6 @@ def test_fused_append_matches_oracle_and_unfused_path(name, kw):
         assert torch.equal(kf, ku) and torch.equal(vf, vu), f"pools differ at step {i}"
         assert H.pools_equal(kf, vf, okp, ovp)
         assert torch.equal(fused, unfused), f"outputs differ at step {i}"
-        assert H.max_err(fused, ref) <= H.TOL[wl.dtype]
+        err = H.max_err(fused, ref)
+        assert err <= H.TOL[wl.dtype]
+        margins.record(f"fused append {name} {wl.dtype}", err, H.TOL[wl.dtype])

@@ -19,6 +19,7 @@ import oracle
 import paged_kv_cache_372_b200 as pa
 from paged_kv_cache_372_b200 import inputs, workloads
 from tests import gpu_harness as H
+from tests import margins
 from tests.bruteforce import bits_of
 
 pytestmark = pytest.mark.gpu
@@ -210,6 +211,8 @@ def test_sharing_patterns_match_oracle(shape, append):
         out, kp, vp, ws = run_shared(case, P, append)
         err = H.max_err(out, ref)
         assert err <= H.TOL[dtype], (shape, P, err)
+        margins.record(f"shared {heads}/{kv_heads} D={D} bs={bs} {dtype} P={P or 'auto'}"
+                       f"{' append' if append else ''}", err, H.TOL[dtype])
         if append:
             assert H.pools_equal(kp, vp, okp, ovp)
         # The plan grouped the sequences as described (units per KV head).
@@ -245,7 +248,9 @@ def test_beam_workloads(name, fused):
         torch.cuda.synchronize()
         assert pa.pa_device_errors() == 0
         assert H.pools_equal(kp, vp, okp, ovp), f"pools differ after step {i}"
-        assert H.max_err(out, ref) <= H.TOL[wl.dtype]
+        err = H.max_err(out, ref)
+        assert err <= H.TOL[wl.dtype]
+        margins.record(f"shared {name}{' fused' if fused else ''} {wl.dtype}", err, H.TOL[wl.dtype])
 
 
 def test_without_sharing_equals_plain_decode():
