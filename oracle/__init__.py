@@ -26,6 +26,7 @@ LIBRARY = os.path.join(HERE, "liboracle.so")
 
 F16 = 0
 BF16 = 1
+KV_FORMATS = {"e4m3": 0, "int8": 1}   # 8-bit cache formats of the *_kv8 functions
 _DTYPE_CODES = {"f16": F16, "fp16": F16, "float16": F16, "bf16": BF16, "bfloat16": BF16}
 
 
@@ -85,6 +86,15 @@ class Oracle:
         L.oracle_reshape_and_cache_fp8.restype = None
         L.oracle_reshape_and_cache_fp8.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
                                                    ctypes.c_float, ctypes.c_float]
+        L.oracle_int8_to_double.restype = ctypes.c_double
+        L.oracle_int8_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_int8_encode.restype = ctypes.c_uint8
+        L.oracle_int8_encode.argtypes = [ctypes.c_float]
+        L.oracle_paged_attention_kv8.restype = None
+        L.oracle_paged_attention_kv8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                                 ctypes.c_double, _I, _I, _P, _P, _I]
+        L.oracle_reshape_and_cache_kv8.restype = None
+        L.oracle_reshape_and_cache_kv8.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
         L.oracle_slot_mapping.restype = None
         L.oracle_slot_mapping.argtypes = [_P, _P, _I, _P, _P, _I, _I]
 
@@ -143,6 +153,64 @@ class Oracle:
         assert slot_mapping.max(initial=-1) < NB * bs
         self.lib.oracle_reshape_and_cache_fp8(_ptr(k), _ptr(v), _ptr(k_pool), _ptr(v_pool), _ptr(slot_mapping),
                                               T, Hkv, D, bs, dtype_code(dtype), float(k_scale), float(v_scale))
+
+    def int8_to_double(self, codes) -> np.ndarray:
+        flat = np.ascontiguousarray(codes, dtype=np.uint8).ravel()
+        f = self.lib.oracle_int8_to_double
+        return np.array([f(int(c)) for c in flat], dtype=np.float64).reshape(np.shape(codes))
+
+    def int8_encode(self, values) -> np.ndarray:
+        flat = np.ascontiguousarray(values, dtype=np.float32).ravel()
+        f = self.lib.oracle_int8_encode
+        return np.array([f(float(v)) for v in flat], dtype=np.uint8).reshape(np.shape(values))
+
+    def paged_attention_kv8(self, q, k_pool, v_pool, block_tables, context_lens, scale, q_dtype, kv_format,
+                            k_scales, v_scales, num_threads: int = 0) -> np.ndarray:
+        """out[s][h][:] in fp64 over an 8-bit cache (uint8 codes; kv_format "e4m3" or
+        "int8") with one scale per KV head (k_scales, v_scales: [num_kv_heads])."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        k_pool = np.ascontiguousarray(k_pool, dtype=np.uint8)
+        v_pool = np.ascontiguousarray(v_pool, dtype=np.uint8)
+        block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+        context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+        B, H, D = q.shape
+        NB, Hkv, bs, D2 = k_pool.shape
+        assert D2 == D and v_pool.shape == k_pool.shape and H % Hkv == 0
+        ks = np.ascontiguousarray(k_scales, dtype=np.float64)
+        vs = np.ascontiguousarray(v_scales, dtype=np.float64)
+        assert ks.shape == (Hkv,) and vs.shape == (Hkv,)
+        for s in range(B):
+            n = int(context_lens[s])
+            pages = -(-n // bs)
+            assert 0 <= n and pages <= block_tables.shape[1]
+            if pages:
+                used = block_tables[s, :pages]
+                assert used.min() >= 0 and used.max() < NB
+        out = np.zeros((B, H, D), dtype=np.float64)
+        self.lib.oracle_paged_attention_kv8(
+            _ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), _ptr(context_lens),
+            B, H, Hkv, D, bs, block_tables.shape[1], float(scale), dtype_code(q_dtype), KV_FORMATS[kv_format],
+            _ptr(ks), _ptr(vs), int(num_threads))
+        return out
+
+    def reshape_and_cache_kv8(self, k, v, k_pool, v_pool, slot_mapping, dtype, kv_format, k_scales,
+                              v_scales) -> None:
+        """In place on uint8 pools: code = encode(x / scale[h]) in fp32, per KV head h."""
+        for a in (k_pool, v_pool):
+            assert a.dtype == np.uint8 and a.flags.c_contiguous
+        k = np.ascontiguousarray(k, dtype=np.uint16)
+        v = np.ascontiguousarray(v, dtype=np.uint16)
+        slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        T, Hkv, D = k.shape
+        NB, Hkv2, bs, D2 = k_pool.shape
+        assert Hkv2 == Hkv and D2 == D and v.shape == k.shape and slot_mapping.shape == (T,)
+        assert slot_mapping.max(initial=-1) < NB * bs
+        ks = np.ascontiguousarray(k_scales, dtype=np.float32)
+        vs = np.ascontiguousarray(v_scales, dtype=np.float32)
+        assert ks.shape == (Hkv,) and vs.shape == (Hkv,)
+        self.lib.oracle_reshape_and_cache_kv8(_ptr(k), _ptr(v), _ptr(k_pool), _ptr(v_pool), _ptr(slot_mapping),
+                                              T, Hkv, D, bs, dtype_code(dtype), KV_FORMATS[kv_format], _ptr(ks),
+                                              _ptr(vs))
 
     def max_threads(self) -> int:
         return int(self.lib.oracle_max_threads())
@@ -263,6 +331,14 @@ def paged_attention_fp8(*args, **kwargs):
 
 def reshape_and_cache_fp8(*args, **kwargs):
     return get().reshape_and_cache_fp8(*args, **kwargs)
+
+
+def paged_attention_kv8(*args, **kwargs):
+    return get().paged_attention_kv8(*args, **kwargs)
+
+
+def reshape_and_cache_kv8(*args, **kwargs):
+    return get().reshape_and_cache_kv8(*args, **kwargs)
 
 
 def to_double(*args, **kwargs):

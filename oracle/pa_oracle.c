@@ -339,6 +339,151 @@ void oracle_reshape_and_cache_fp8(const uint16_t *k, const uint16_t *v,
 }
 
 /*
+ * 8-bit signed integer KV cache, the INT8 row of the compression table of
+ * "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
+ * section 3.2 (内存压缩技术; section 4.3 applies it to older pages). Stored
+ * excess-128: byte u holds the integer u - 128. An element x with scale s is
+ * stored as clamp(round(x / s), -127, 127) + 128, the rounding to nearest with
+ * ties to even, the division in fp32 (float operands, IEEE single). NaN stores
+ * 128 (zero); infinities clamp.
+ */
+double oracle_int8_to_double(uint8_t code)
+{
+    return (double)code - 128.0;
+}
+
+uint8_t oracle_int8_encode(float y)
+{
+    if (isnan(y))
+        return 128;
+    if (y >= 127.0f)
+        return 255;
+    if (y <= -127.0f)
+        return 1;
+    const double a = (double)y;
+    double r = floor(a);
+    const double f = a - r;                 /* exact: |a| < 127 */
+    if (f > 0.5 || (f == 0.5 && fmod(r, 2.0) != 0.0))
+        r += 1.0;
+    return (uint8_t)(int)(r + 128.0);
+}
+
+enum { ORACLE_KV_E4M3 = 0, ORACLE_KV_INT8 = 1 };
+
+static double kv8_to_double(uint8_t code, int format)
+{
+    return format == ORACLE_KV_INT8 ? oracle_int8_to_double(code) : oracle_e4m3_to_double(code);
+}
+
+/*
+ * Paged decode attention over an 8-bit KV cache (E4M3 or INT8 codes) with one
+ * scale per KV head: key element of KV head j = k_scales[j] * decode(code),
+ * value element = v_scales[j] * decode(code). Otherwise the computation of
+ * oracle_paged_attention, in fp64.
+ */
+void oracle_paged_attention_kv8(double *out, const uint16_t *q,
+                                const uint8_t *k_pool, const uint8_t *v_pool,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int num_heads, int num_kv_heads,
+                                int head_dim, int block_size, int max_blocks_per_seq,
+                                double scale, int q_dtype, int format,
+                                const double *k_scales, const double *v_scales, int num_threads)
+{
+    const int group = num_heads / num_kv_heads;
+    const long pairs = (long)num_seqs * num_heads;
+#ifdef _OPENMP
+    if (num_threads > 0)
+        omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long sh = 0; sh < pairs; sh++) {
+        const int s = (int)(sh / num_heads);
+        const int h = (int)(sh % num_heads);
+        const int kvh = h / group;
+        const int n = context_lens[s];
+        const double ks = k_scales[kvh], vs = v_scales[kvh];
+        double *o = out + (size_t)sh * head_dim;
+        for (int d = 0; d < head_dim; d++)
+            o[d] = 0.0;
+        if (n <= 0)
+            continue;
+        double *qd = (double *)malloc(sizeof(double) * head_dim);
+        double *scores = (double *)malloc(sizeof(double) * n);
+        for (int d = 0; d < head_dim; d++)
+            qd[d] = oracle_to_double(q[(size_t)sh * head_dim + d], q_dtype);
+        const int pages = (n + block_size - 1) / block_size;
+        const int32_t *table = block_tables + (size_t)s * max_blocks_per_seq;
+        for (int i = 0; i < pages; i++) {
+            const size_t page = (size_t)table[i];
+            for (int r = 0; r < block_size; r++) {
+                const int t = i * block_size + r;
+                if (t >= n)
+                    break;
+                const uint8_t *key = k_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;
+                double dot = 0.0;
+                for (int d = 0; d < head_dim; d++)
+                    dot += qd[d] * (ks * kv8_to_double(key[d], format));
+                scores[t] = dot;
+            }
+        }
+        double mx = -INFINITY;
+        for (int t = 0; t < n; t++)
+            if (scale * scores[t] > mx)
+                mx = scale * scores[t];
+        double total = 0.0;
+        for (int t = 0; t < n; t++) {
+            scores[t] = exp(scale * scores[t] - mx);
+            total += scores[t];
+        }
+        for (int t = 0; t < n; t++)
+            scores[t] /= total;
+        for (int i = 0; i < pages; i++) {
+            const size_t page = (size_t)table[i];
+            for (int r = 0; r < block_size; r++) {
+                const int t = i * block_size + r;
+                if (t >= n)
+                    break;
+                const uint8_t *val = v_pool + ((page * num_kv_heads + kvh) * block_size + r) * head_dim;
+                for (int d = 0; d < head_dim; d++)
+                    o[d] += scores[t] * (vs * kv8_to_double(val[d], format));
+            }
+        }
+        free(scores);
+        free(qd);
+    }
+}
+
+/*
+ * Quantising cache write with one scale per KV head: element x of head h is
+ * stored as encode(x / k_scales[h]) (keys) or encode(x / v_scales[h])
+ * (values), the division in fp32, encode being the E4M3 or the INT8 encoder.
+ */
+void oracle_reshape_and_cache_kv8(const uint16_t *k, const uint16_t *v,
+                                  uint8_t *k_pool, uint8_t *v_pool,
+                                  const int64_t *slot_mapping, int num_tokens,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int dtype, int format, const float *k_scales, const float *v_scales)
+{
+    for (int t = 0; t < num_tokens; t++) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; h++) {
+            const size_t src = ((size_t)t * num_kv_heads + h) * head_dim;
+            const size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) * head_dim;
+            for (int d = 0; d < head_dim; d++) {
+                const float kx = (float)oracle_to_double(k[src + d], dtype) / k_scales[h];
+                const float vx = (float)oracle_to_double(v[src + d], dtype) / v_scales[h];
+                k_pool[dst + d] = format == ORACLE_KV_INT8 ? oracle_int8_encode(kx) : oracle_e4m3_encode(kx);
+                v_pool[dst + d] = format == ORACLE_KV_INT8 ? oracle_int8_encode(vx) : oracle_e4m3_encode(vx);
+            }
+        }
+    }
+}
+
+/*
  * Write each new token's K and V rows into its pool slot. slot = block *
  * block_size + offset; a negative slot means "no write" for that token.
  * Pure bit copy of the 16-bit elements.

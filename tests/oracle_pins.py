@@ -21,6 +21,11 @@ What pins what:
                           closed forms, round trip of every finite code
   * fp8 attention / write brute force over the numpy-dequantised cache; numpy
                           float32 division + torch's cast
+  * INT8 codes            every byte decodes to byte - 128; encoding vs numpy's
+                          round-half-to-even clipped to [-127, 127]
+  * 8-bit cache with      E4M3 and INT8, per-KV-head scales spanning up to
+    per-head scales       100x: brute force over the numpy-dequantised cache;
+                          the write vs numpy / torch per head
 """
 from __future__ import annotations
 
@@ -384,6 +389,78 @@ def pin_fp8_cache_write(orc, seed=14):
         assert np.array_equal(kp, ek) and np.array_equal(vp, ev)
 
 
+def pin_int8_codes(orc, seed=16):
+    """INT8 (excess-128) codes: every byte decodes to byte - 128; the encoder is
+    numpy's round-half-to-even clipped to [-127, 127], with exact ties, the
+    saturation points, NaN (stored as zero) and infinities."""
+    codes = np.arange(256, dtype=np.uint8)
+    assert np.array_equal(orc.int8_to_double(codes), codes.astype(np.float64) - 128.0)
+    rng = np.random.default_rng(seed)
+    x = np.concatenate([rng.standard_normal(1500) * s for s in (0.3, 3.0, 40.0, 200.0)])
+    x = np.concatenate([x, np.arange(-130, 130) + 0.5, np.arange(-130, 131)]).astype(np.float32)
+    want = (np.clip(np.rint(x), -127, 127).astype(np.int64) + 128).astype(np.uint8)
+    assert np.array_equal(orc.int8_encode(x), want)
+    special = np.array([np.nan, np.inf, -np.inf, 127.49, -127.5, 1e30], dtype=np.float32)
+    assert list(orc.int8_encode(special)) == [128, 255, 1, 255, 1, 255]
+
+
+def _dequant_kv8(codes, kv_format, scales):
+    """Codes [NB][Hkv][bs][D] -> float64 values with one scale per KV head: E4M3
+    through torch's float8_e4m3fn, INT8 as byte - 128."""
+    if kv_format == "e4m3":
+        v = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    else:
+        v = codes.astype(np.float64) - 128.0
+    return v * np.asarray(scales, dtype=np.float64)[None, :, None, None]
+
+
+def _head_scales(rng, n, base):
+    """n per-head scales spanning up to 100x around `base`."""
+    return base * 10.0 ** rng.uniform(-1.0, 1.0, n)
+
+
+def pin_kv8_attention_bruteforce(orc, seed=17):
+    """Attention over an 8-bit cache with per-KV-head scales (E4M3 and INT8) =
+    the brute force over the numpy-dequantised cache."""
+    rng = np.random.default_rng(seed)
+    for fmt in ("e4m3", "int8"):
+        for B, H, Hkv, D, bs, ctx, dt in SHAPES:
+            q, k8, v8, tab, cl = _fp8_case(rng, B, H, Hkv, D, bs, ctx, dt)
+            ks, vs = _head_scales(rng, Hkv, 0.05), _head_scales(rng, Hkv, 0.05)
+            got = orc.paged_attention_kv8(q, k8, v8, tab, cl, 1.0 / math.sqrt(D), dt, fmt, ks, vs)
+            ref = contiguous_attention(decode(q, dt), _dequant_kv8(k8, fmt, ks), _dequant_kv8(v8, fmt, vs), tab, cl,
+                                       1.0 / math.sqrt(D))
+            assert np.abs(got - ref).max() <= ATOL * max(1.0, np.abs(ref).max()), (fmt, B, H, Hkv)
+
+
+def pin_kv8_cache_write(orc, seed=18):
+    """Quantising write with per-KV-head scales: code = encode(x / scale[h]) with
+    the division in float32; E4M3 through torch's cast, INT8 through numpy."""
+    rng = np.random.default_rng(seed)
+    NB, Hkv, bs, D, T = 5, 3, 16, 32, 12
+    for fmt in ("e4m3", "int8"):
+        for dt in ("f16", "bf16"):
+            k = _rand_bits(rng, (T, Hkv, D), dt)
+            v = _rand_bits(rng, (T, Hkv, D), dt)
+            kp = rng.integers(0, 256, (NB, Hkv, bs, D), dtype=np.uint8)
+            vp = rng.integers(0, 256, (NB, Hkv, bs, D), dtype=np.uint8)
+            slots = rng.choice(NB * bs, T, replace=False).astype(np.int64)
+            slots[2] = -1
+            ks = _head_scales(rng, Hkv, 0.02).astype(np.float32)
+            vs = _head_scales(rng, Hkv, 0.02).astype(np.float32)
+            ek, ev = kp.copy(), vp.copy()
+            keep = slots >= 0
+            for pool, x, sc in ((ek, k, ks), (ev, v, vs)):
+                y = (decode(x, dt).astype(np.float32) / sc[None, :, None]).astype(np.float32)
+                if fmt == "e4m3":
+                    codes = _torch_e4m3_codes(np.clip(y, -448, 448))
+                else:
+                    codes = (np.clip(np.rint(y), -127, 127).astype(np.int64) + 128).astype(np.uint8)
+                pool[slots[keep] // bs, :, slots[keep] % bs, :] = codes[keep]
+            orc.reshape_and_cache_kv8(k, v, kp, vp, slots, dt, fmt, ks, vs)
+            assert np.array_equal(kp, ek) and np.array_equal(vp, ev), (fmt, dt)
+
+
 def pin_slot_mapping(orc, seed=10):
     rng = np.random.default_rng(seed)
     bs, B, W = 16, 5, 6
@@ -403,4 +480,5 @@ ALL_PINS = [pin_decode_f16, pin_decode_bf16, pin_bruteforce, pin_sdpa, pin_rando
             pin_equal_keys, pin_two_token_closed_form, pin_block_permutation,
             pin_shared_equals_duplicated, pin_tail_slots_ignored, pin_gqa_mapping,
             pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_swap_blocks, pin_slot_mapping,
-            pin_e4m3_decode, pin_e4m3_encode, pin_fp8_attention_bruteforce, pin_fp8_cache_write]
+            pin_e4m3_decode, pin_e4m3_encode, pin_fp8_attention_bruteforce, pin_fp8_cache_write,
+            pin_int8_codes, pin_kv8_attention_bruteforce, pin_kv8_cache_write]

@@ -53,6 +53,17 @@ MUTATIONS = {
                                 "o[d] += scores[t] * oracle_e4m3_to_double(val[d]);"),
     "fp8_write_scale_times": ("k_pool[dst + d] = oracle_e4m3_encode(kx / k_scale);",
                               "k_pool[dst + d] = oracle_e4m3_encode(kx * k_scale);"),
+    "int8_excess_127": ("return (double)code - 128.0;", "return (double)code - 127.0;"),
+    "int8_ties_away": ("if (f > 0.5 || (f == 0.5 && fmod(r, 2.0) != 0.0))", "if (f >= 0.5)"),
+    "int8_clamps_at_minus_128": ("if (y <= -127.0f)\n        return 1;", "if (y <= -127.0f)\n        return 0;"),
+    "kv8_scale_of_query_head": ("const double ks = k_scales[kvh], vs = v_scales[kvh];",
+                                "const double ks = k_scales[h % num_kv_heads], vs = v_scales[h % num_kv_heads];"),
+    "kv8_scales_swapped": ("const double ks = k_scales[kvh], vs = v_scales[kvh];",
+                           "const double ks = v_scales[kvh], vs = k_scales[kvh];"),
+    "kv8_write_scale_of_head_0": ("/ k_scales[h];", "/ k_scales[0];"),
+    "kv8_format_ignored": (
+        "return format == ORACLE_KV_INT8 ? oracle_int8_to_double(code) : oracle_e4m3_to_double(code);",
+        "return oracle_e4m3_to_double(code);"),
     "negative_slot_stops_the_write": (
         "int num_kv_heads, int head_dim, int block_size)\n{\n    for (int t = 0; t < num_tokens; t++) {\n"
         "        const int64_t slot = slot_mapping[t];\n        if (slot < 0)\n            continue;",
