@@ -69,6 +69,12 @@ typedef enum {
 
 typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 
+/* Formats of an 8-bit KV cache (pa_reshape_and_cache_quant, pa_decode_quant). */
+typedef enum {
+    PA_KV_E4M3 = 0,  /* fp8 e4m3fn codes: value = scale * E4M3(code) */
+    PA_KV_INT8 = 1   /* signed 8-bit integers stored excess-128: value = scale * (code - 128) */
+} pa_kv_format;
+
 /* Bits of the per-device error word (pa_device_errors). */
 #define PA_DEVERR_BLOCK_ID 1u   /* block table entry outside [0, num_blocks) */
 #define PA_DEVERR_CONTEXT  2u   /* context_len < 0 or above the limit (clamped) */
@@ -246,6 +252,50 @@ PA_API pa_status pa_reshape_and_cache_fp8(const void *k, const void *v, void *k_
                                           int num_kv_heads, int head_dim, int block_size,
                                           int num_blocks, int dtype, float k_scale, float v_scale,
                                           pa_stream_t stream);
+
+/*
+ * Quantising cache write with one scale per KV head, in either 8-bit format:
+ * element x of KV head h (keys; values alike with v_scales) is stored as the
+ * code of y = x / k_scales[h], the division in fp32 rounded to nearest.
+ *   PA_KV_E4M3: the E4M3 code of y, rounded to nearest even, magnitudes past
+ *               448 saturated to 448 (as pa_reshape_and_cache_fp8).
+ *   PA_KV_INT8: clamp(round(y), -127, 127) + 128, rounding to nearest even;
+ *               NaN stores 128 (zero).
+ * k_scales, v_scales: DEVICE arrays [num_kv_heads] of positive finite floats,
+ * 4-byte aligned. Pools uint8 [num_blocks][num_kv_heads][block_size][head_dim],
+ * 8-byte aligned; other arguments, slot rules and error reporting as
+ * pa_reshape_and_cache.
+ *
+ * Defined by: "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
+ * section 3.2 (内存压缩技术) — the compression table's INT8 row (a quarter of
+ * the fp32 bytes) and, in section 4.3, INT8 for older pages; the per-head
+ * scale and the excess-128 storage are this library's choices.
+ */
+PA_API pa_status pa_reshape_and_cache_quant(const void *k, const void *v, void *k_pool, void *v_pool,
+                                            const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                                            int head_dim, int block_size, int num_blocks, int dtype, int kv_format,
+                                            const float *k_scales, const float *v_scales, pa_stream_t stream);
+
+/*
+ * Paged decode attention over an 8-bit cache with one scale per KV head: key
+ * element of KV head j = k_scales[j] * decode(code), value element =
+ * v_scales[j] * decode(code), decode being E4M3 (PA_KV_E4M3) or code - 128
+ * (PA_KV_INT8); otherwise exactly pa_decode (q and out fp16/bf16 by dtype).
+ * head_dim 128. The partition and the workspace are those of pa_decode_fp8
+ * (pa_decode_fp8_partition_size, pa_decode_fp8_workspace_size). INT8 codes
+ * enter the tensor-core products as the exact fp16 numbers 1152 + (code - 128);
+ * the constant is taken off the scores (per query row) and the outputs (times
+ * the softmax sum) in fp32. Queries are converted to fp16 as in pa_decode_fp8
+ * (PA_DEVERR_QRANGE for bf16 elements above 65504).
+ *
+ * Defined by: the same section 3.2; the attention is that of section 3.1.
+ */
+PA_API pa_status pa_decode_quant(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                 const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                 int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, int dtype,
+                                 int kv_format, const float *k_scales, const float *v_scales, int partition_size,
+                                 void *workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /* Workspace bytes pa_decode needs for these sizes (0 if the shape is invalid). */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,

@@ -21,6 +21,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "pa.h")
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK = range(5)
 PA_F16, PA_BF16 = 0, 1
+PA_KV_E4M3, PA_KV_INT8 = 0, 1
 DEVERR_BLOCK_ID, DEVERR_CONTEXT, DEVERR_SLOT, DEVERR_PAIR, DEVERR_TIMEOUT, DEVERR_QRANGE = 1, 2, 4, 8, 16, 32
 
 _DTYPES = {torch.float16: PA_F16, torch.bfloat16: PA_BF16}
@@ -86,6 +87,11 @@ def lib() -> ctypes.CDLL:
         L.pa_num_sms.argtypes = []
         L.pa_selftest_bounded_wait.restype = _I
         L.pa_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _P]
+        L.pa_reshape_and_cache_quant.restype = _I
+        L.pa_reshape_and_cache_quant.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.pa_decode_quant.restype = _I
+        L.pa_decode_quant.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P,
+                                      _I, _P, _SZ, _P]
         L.pa_decode_noalloc.restype = _I
         L.pa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]
         _lib = L
@@ -293,6 +299,56 @@ def pa_reshape_and_cache_fp8(k, v, k_pool, v_pool, slot_mapping, k_scale, v_scal
         _cuda(k, "k"), _cuda(v, "v"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
         _cuda(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, bs, NB, _DTYPES[k.dtype], float(k_scale),
         float(v_scale), _stream(stream)))
+
+
+KV_FORMATS = {"e4m3": PA_KV_E4M3, "int8": PA_KV_INT8}
+
+
+def _scales(t, name, n):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != (n,):
+        raise ValueError(f"{name} must be a float32 CUDA tensor of shape [num_kv_heads]")
+    return _cuda(t, name)
+
+
+def pa_reshape_and_cache_quant(k, v, k_pool, v_pool, slot_mapping, kv_format, k_scales, v_scales,
+                               stream=None) -> None:
+    """Quantising write into an 8-bit cache ("e4m3" or "int8" codes) with one
+    scale per KV head: k_pool[slot] = encode(k[t] / k_scales[h]) (and v)."""
+    T, Hkv, D = k.shape
+    NB, Hkv2, bs, D2 = k_pool.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(v.shape) != tuple(k.shape) or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("shape mismatch between k, v and the pools")
+    if k.dtype not in _DTYPES or v.dtype != k.dtype or k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("k, v fp16/bf16; pools uint8")
+    _check(lib().pa_reshape_and_cache_quant(
+        _cuda(k, "k"), _cuda(v, "v"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, bs, NB, _DTYPES[k.dtype],
+        KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv), _scales(v_scales, "v_scales", Hkv),
+        _stream(stream)))
+
+
+def pa_decode_quant(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len, kv_format,
+                    k_scales, v_scales, partition_size=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode over an 8-bit cache ("e4m3" or "int8" uint8 codes [NB][Hkv][bs][D])
+    with one scale per KV head (float32 CUDA tensors [Hkv])."""
+    B, H, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch between q, out and the pools")
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("8-bit pools must be uint8 tensors of codes")
+    if q.dtype not in _DTYPES or out.dtype != q.dtype:
+        raise ValueError("q and out must share one dtype, fp16 or bf16")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device, fp8=True)
+    _check(lib().pa_decode_quant(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
+        B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
+        KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv), _scales(v_scales, "v_scales", Hkv),
+        int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return out
 
 
 def pa_reshape_and_cache(k, v, k_pool, v_pool, slot_mapping, stream=None) -> None:

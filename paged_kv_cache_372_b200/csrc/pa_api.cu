@@ -3,7 +3,9 @@
 // stream. Nothing here allocates device memory or synchronises (except
 // pa_device_errors, which exists to do so).
 #include <cstdarg>
+#include <atomic>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <string>
 
@@ -34,6 +36,7 @@ pa_status cuda_fail(cudaError_t e, const char *what) {
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct DeviceInfo {
+    int dev = 0;
     int sms = 0;
     int smem_optin = 0;
 };
@@ -54,6 +57,7 @@ pa_status device_info(DeviceInfo *out) {
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
         e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(shared memory)");
+        cache[dev].dev = dev;
         cache[dev].sms = sms;
         cache[dev].smem_optin = smem;
     }
@@ -161,8 +165,11 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
                       int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
                       int num_blocks, int max_context_len, float scale, int dtype, int partition_size,
                       void *workspace, size_t workspace_bytes, pa_stream_t stream, bool kv8 = false,
-                      float k_scale = 1.f, float v_scale = 1.f, bool shared = false) {
+                      float k_scale = 1.f, float v_scale = 1.f, bool shared = false, bool int8 = false,
+                      const float *k_scales = nullptr, const float *v_scales = nullptr) {
     g_last_error.clear();
+    if ((k_scales == nullptr) != (v_scales == nullptr) || (k_scales && (!aligned(k_scales, 4) || !aligned(v_scales, 4))))
+        return fail(PA_ERR_INVALID, "k_scales and v_scales: both null or both 4-byte aligned device arrays");
     if (shared && num_seqs > pa::SHARE_MAX_SEQS)
         return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode takes at most %d sequences, got %d", pa::SHARE_MAX_SEQS,
                     num_seqs);
@@ -219,7 +226,9 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     p.num_blocks = num_blocks;
     p.ctx_limit = ctx_limit;
     p.partition = P;
-    p.max_parts = max_parts;
+    p.max_parts = L.slots;
+    p.l1_base = max_parts;
+    p.max_chunks = L.chunks;
     p.qscale = scale * 1.4426950408889634f * k_scale;
     p.v_scale = v_scale;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -229,13 +238,24 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     p.ml = reinterpret_cast<float2 *>(ws + L.ml);
     p.part_acc = reinterpret_cast<float *>(ws + L.acc);
     p.merge_count = reinterpret_cast<int *>(ws + L.count);
+    p.chunk_count = reinterpret_cast<int *>(ws + L.chunk_count);
     p.entries_b = shared ? reinterpret_cast<int4 *>(ws + L.entries_b) : nullptr;
     p.members = shared ? reinterpret_cast<int *>(ws + L.members) : nullptr;
     p.member_nparts = shared ? reinterpret_cast<int *>(ws + L.member_nparts) : nullptr;
     p.append_guard = k_new != nullptr;
+    p.early = 0;          // set by the launcher of the tensor-core kernels
+    p.reduce_launch = 0;  // likewise
+    p.k_scales = k_scales;
+    p.v_scales = v_scales;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int group = num_heads / num_kv_heads;
+    if (kv8 && int8)
+        return dtype == PA_F16 ? dispatch_group_fp8<__half, true, true>(p, group, s)
+                               : dispatch_group_fp8<__nv_bfloat16, true, true>(p, group, s);
+    if (kv8 && k_scales)
+        return dtype == PA_F16 ? dispatch_group_fp8<__half, false, true>(p, group, s)
+                               : dispatch_group_fp8<__nv_bfloat16, false, true>(p, group, s);
     if (kv8)
         return dtype == PA_F16 ? dispatch_group_fp8<__half>(p, group, s) : dispatch_group_fp8<__nv_bfloat16>(p, group, s);
     if (shared) {
@@ -333,6 +353,45 @@ pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void 
     return PA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The 8-bit cache write: E4M3 or INT8 codes, one scale per tensor (k_scale,
+// v_scale) or one per KV head (k_scales, v_scales, device arrays).
+pa_status reshape_kv8_impl(const void *k, const void *v, void *k_pool, void *v_pool, const int64_t *slot_mapping,
+                           int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                           bool int8, float k_scale, float v_scale, const float *k_scales, const float *v_scales,
+                           pa_stream_t stream) {
+    DeviceInfo info;
+    pa_status st = device_info(&info);
+    if (st != PA_OK) return st;
+    const int vec_per_row = head_dim / 8;
+    const long long total = (long long)num_tokens * num_kv_heads * vec_per_row;
+    long long blocks = (total + 255) / 256;
+    if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto launch = [&](auto kernel) {
+        kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+                                                 static_cast<uint2 *>(k_pool), static_cast<uint2 *>(v_pool),
+                                                 slot_mapping, total, vec_per_row, num_kv_heads, block_size,
+                                                 (long long)num_blocks * block_size, k_scale, v_scale, k_scales,
+                                                 v_scales);
+    };
+    if (dtype == PA_F16)
+        int8 ? launch(pa::pa_reshape_kv8_kernel<__half, true>) : launch(pa::pa_reshape_kv8_kernel<__half, false>);
+    else
+        int8 ? launch(pa::pa_reshape_kv8_kernel<__nv_bfloat16, true>)
+             : launch(pa::pa_reshape_kv8_kernel<__nv_bfloat16, false>);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "8-bit cache write launch");
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 pa_status pa_reshape_and_cache_fp8(const void *k, const void *v, void *k_pool, void *v_pool,
                                    const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
                                    int block_size, int num_blocks, int dtype, float k_scale, float v_scale,
@@ -349,27 +408,44 @@ pa_status pa_reshape_and_cache_fp8(const void *k, const void *v, void *k_pool, v
     if (!k || !v || !k_pool || !v_pool || !slot_mapping) return fail(PA_ERR_INVALID, "null pointer");
     if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_pool, 8) || !aligned(v_pool, 8) || !aligned(slot_mapping, 8))
         return fail(PA_ERR_INVALID, "misaligned pointer");
-    DeviceInfo info;
-    pa_status st = device_info(&info);
-    if (st != PA_OK) return st;
-    const int vec_per_row = head_dim / 8;
-    const long long total = (long long)num_tokens * num_kv_heads * vec_per_row;
-    long long blocks = (total + 255) / 256;
-    if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dtype == PA_F16)
-        pa::pa_reshape_fp8_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(
-            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint2 *>(k_pool),
-            static_cast<uint2 *>(v_pool), slot_mapping, total, vec_per_row, num_kv_heads, block_size,
-            (long long)num_blocks * block_size, k_scale, v_scale);
-    else
-        pa::pa_reshape_fp8_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
-            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint2 *>(k_pool),
-            static_cast<uint2 *>(v_pool), slot_mapping, total, vec_per_row, num_kv_heads, block_size,
-            (long long)num_blocks * block_size, k_scale, v_scale);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "pa_reshape_and_cache_fp8 launch");
-    return PA_OK;
+    return reshape_kv8_impl(k, v, k_pool, v_pool, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                            num_blocks, dtype, false, k_scale, v_scale, nullptr, nullptr, stream);
+}
+
+pa_status pa_reshape_and_cache_quant(const void *k, const void *v, void *k_pool, void *v_pool,
+                                     const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                     int block_size, int num_blocks, int dtype, int kv_format, const float *k_scales,
+                                     const float *v_scales, pa_stream_t stream) {
+    g_last_error.clear();
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return fail(PA_ERR_INVALID, "size argument");
+    if (dtype != PA_F16 && dtype != PA_BF16) return fail(PA_ERR_INVALID, "dtype %d", dtype);
+    if (kv_format != PA_KV_E4M3 && kv_format != PA_KV_INT8) return fail(PA_ERR_INVALID, "kv_format %d", kv_format);
+    if (head_dim != 64 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d", head_dim);
+    if (block_size != 16 && block_size != 32 && block_size != 64)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d", block_size);
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !k_pool || !v_pool || !slot_mapping || !k_scales || !v_scales)
+        return fail(PA_ERR_INVALID, "null pointer");
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_pool, 8) || !aligned(v_pool, 8) ||
+        !aligned(slot_mapping, 8) || !aligned(k_scales, 4) || !aligned(v_scales, 4))
+        return fail(PA_ERR_INVALID, "misaligned pointer");
+    return reshape_kv8_impl(k, v, k_pool, v_pool, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                            num_blocks, dtype, kv_format == PA_KV_INT8, 1.f, 1.f, k_scales, v_scales, stream);
+}
+
+pa_status pa_decode_quant(void *out, const void *q, const void *k_pool, const void *v_pool,
+                          const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                          int max_context_len, float scale, int dtype, int kv_format, const float *k_scales,
+                          const float *v_scales, int partition_size, void *workspace, size_t workspace_bytes,
+                          pa_stream_t stream) {
+    g_last_error.clear();
+    if (kv_format != PA_KV_E4M3 && kv_format != PA_KV_INT8) return fail(PA_ERR_INVALID, "kv_format %d", kv_format);
+    if (num_seqs > 0 && (!k_scales || !v_scales)) return fail(PA_ERR_INVALID, "null scale array");
+    return decode_impl(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream, true, 1.f, 1.f, false,
+                       kv_format == PA_KV_INT8, k_scales, v_scales);
 }
 
 pa_status pa_copy_blocks(void *const *pools, int num_pools, const int64_t *src_dst_pairs, int num_pairs,

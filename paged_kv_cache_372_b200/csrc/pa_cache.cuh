@@ -45,17 +45,30 @@ __global__ void __launch_bounds__(256) pa_reshape_kernel(const uint4 *__restrict
     }
 }
 
-// Quantising cache write for an E4M3 (fp8) cache: code = E4M3(x / scale),
-// the division in fp32 (IEEE, round to nearest), the conversion rounding to
-// nearest even and saturating at +-448. One thread turns one 16-byte vector of
-// K (8 elements) into 8 codes, and the same for V.
-template <typename T>
-__global__ void __launch_bounds__(256) pa_reshape_fp8_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+// Two INT8 codes (excess-128) of two fp32 values already divided by their
+// scale: round to nearest even, clamp to [-127, 127], NaN stores zero.
+__device__ __forceinline__ uint32_t int8x2_encode(float2 y) {
+    const int a = isnan(y.x) ? 0 : min(127, max(-127, __float2int_rn(y.x)));
+    const int b = isnan(y.y) ? 0 : min(127, max(-127, __float2int_rn(y.y)));
+    return (uint32_t)(a + 128) | ((uint32_t)(b + 128) << 8);
+}
+
+// Quantising cache write for an 8-bit cache: code = encode(x / scale), the
+// division in fp32 (IEEE, round to nearest). E4M3 (I8 false): the conversion
+// rounds to nearest even and saturates at +-448; INT8 (I8 true): round to
+// nearest even, clamp to [-127, 127], stored excess-128. The scale is k_scale /
+// v_scale, or with k_scales / v_scales the entry of the row's KV head. One
+// thread turns one 16-byte vector of K (8 elements) into 8 codes, and the same
+// for V.
+template <typename T, bool I8>
+__global__ void __launch_bounds__(256) pa_reshape_kv8_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                                              uint2 *__restrict__ k_pool, uint2 *__restrict__ v_pool,
                                                              const int64_t *__restrict__ slot_mapping,
                                                              long long total_vectors, int vec_per_row,
                                                              int num_kv_heads, int block_size, long long num_slots,
-                                                             float k_scale, float v_scale) {
+                                                             float k_scale, float v_scale,
+                                                             const float *__restrict__ k_scales,
+                                                             const float *__restrict__ v_scales) {
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vectors; i += stride) {
         const long long row = i / vec_per_row;
@@ -72,7 +85,7 @@ __global__ void __launch_bounds__(256) pa_reshape_fp8_kernel(const uint4 *__rest
         const int64_t off = slot - blk * block_size;
         const size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * vec_per_row + vec;
         const uint4 src[2] = {k[i], v[i]};
-        const float sc[2] = {k_scale, v_scale};
+        const float sc[2] = {k_scales ? k_scales[h] : k_scale, v_scales ? v_scales[h] : v_scale};
         uint2 codes[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -82,7 +95,11 @@ __global__ void __launch_bounds__(256) pa_reshape_fp8_kernel(const uint4 *__rest
             for (int q = 0; q < 4; ++q) {
                 const float2 f = Elem<T>::pair(w[q]);
                 const float2 y = make_float2(__fdiv_rn(f.x, sc[j]), __fdiv_rn(f.y, sc[j]));
-                const uint32_t two = (uint32_t)__nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+                uint32_t two;
+                if constexpr (I8)
+                    two = int8x2_encode(y);
+                else
+                    two = (uint32_t)__nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
                 c[q >> 1] |= two << (16 * (q & 1));
             }
             codes[j] = make_uint2(c[0], c[1]);

@@ -50,37 +50,65 @@ struct DecodeParams {
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks;
     int ctx_limit;   // context lengths are clamped to [0, ctx_limit]
     int partition;   // P, tokens per partition
-    int max_parts;   // ceil(ctx_limit / P)
-    float qscale;    // scale * log2(e) (times k_scale for an fp8 cache)
-    float v_scale;   // fp8 cache: dequantisation scale of V (1 otherwise)
+    int max_parts;   // partial slots per (sequence, head): partitions, then chunk merges
+    int l1_base;     // first chunk-merge slot (= the most partitions a sequence has)
+    int max_chunks;  // chunk counters per (sequence, KV head); 0 without chunked merging
+    float qscale;    // scale * log2(e) (times k_scale for an fp8 cache with one scale)
+    float v_scale;   // fp8 cache with one scale: dequantisation scale of V (1 otherwise)
+    const float *k_scales;  // 8-bit cache with one scale per KV head: [num_kv_heads]
+    const float *v_scales;  // (null: the single scales above)
     int *counter;    // work-list cursor (reset by the plan kernel)
     int *num_entries;
     int4 *entries;   // {seq, partition, tokens, partitions of seq}
     float2 *ml;      // [seq][head][part] (max in log2 units, sum of weights)
     float *part_acc; // [seq][head][part][D] unnormalised outputs
-    int *merge_count;// [seq][kv head] finished partitions
+    int *merge_count;// [seq][kv head] finished partitions (or finished chunks)
+    int *chunk_count;// [seq][kv head][chunk] finished partitions of each chunk
     // Shared-prefix units (pa_decode_shared): a unit may serve several
     // sequences whose block tables begin with the same blocks.
     int4 *entries_b; // {first token, member offset, member count (0: one sequence), 0}
     int *members;    // sequences in grouping order
     int *member_nparts;  // partitions of members[i]
     int append_guard;    // 1: a sequence's last position never lies in a shared block
+    int early;           // 1: the attention kernel starts without waiting for the one-warp plan
+    int reduce_launch;   // 1: split partitions merge in pa_reduce_kernel, a launch of their own
 };
 
-// Workspace layout: header (counter, entry count), work list, partials.
+// Split merges: a (sequence, KV head) with more than MERGE_FANIN partitions
+// merges in two levels. The last partition to finish of each chunk of
+// MERGE_FANIN consecutive partitions merges that chunk into a chunk partial
+// (same form: max, sum, unnormalised output); the last chunk merge merges the
+// chunk partials into the output. Every merge reads a fixed set in a fixed
+// order, so the result does not depend on which warp finishes when, and the
+// serial merge at the end of a long sequence is MERGE_FANIN reads deep
+// instead of one per partition.
+constexpr int MERGE_FANIN = 8;
+
+__host__ __device__ inline int merge_chunks(int max_parts) {
+    return max_parts > MERGE_FANIN ? (max_parts + MERGE_FANIN - 1) / MERGE_FANIN : 0;
+}
+
+// Workspace layout: header (counter, entry count), work list, merge and chunk
+// counters, partials (partitions, then chunk partials).
 struct WsLayout {
-    size_t entries, ml, acc, count, entries_b, members, member_nparts, total;
+    size_t entries, ml, acc, count, chunk_count, entries_b, members, member_nparts, total;
+    int slots, chunks;
 };
 
 inline __host__ __device__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// max_parts: the most partitions a sequence can have. Shared-prefix decode
+// merges members in one level (no chunk partials).
 inline __host__ __device__ WsLayout ws_layout(int B, int H, int Hkv, int D, int max_parts, bool shared = false) {
     WsLayout L;
+    L.chunks = shared ? 0 : merge_chunks(max_parts);
+    L.slots = max_parts + L.chunks;
     size_t off = 256;
     L.entries = off;
     off = align256(off + sizeof(int4) * (size_t)B * max_parts);
-    L.count = off;
-    off = align256(off + sizeof(int) * (size_t)B * Hkv);
+    L.count = off;  // merge counters, then chunk counters: one region, zeroed together
+    L.chunk_count = off + sizeof(int) * (size_t)B * Hkv;
+    off = align256(off + sizeof(int) * (size_t)B * Hkv * (1 + L.chunks));
     L.entries_b = L.members = L.member_nparts = 0;
     if (shared) {
         L.entries_b = off;
@@ -90,7 +118,7 @@ inline __host__ __device__ WsLayout ws_layout(int B, int H, int Hkv, int D, int 
         L.member_nparts = off;
         off = align256(off + sizeof(int) * (size_t)B);
     }
-    const size_t parts = max_parts > 1 ? (size_t)max_parts : 0;  // no partials without a split
+    const size_t parts = max_parts > 1 ? (size_t)L.slots : 0;  // no partials without a split
     L.ml = off;
     off = align256(off + sizeof(float2) * (size_t)B * H * parts);
     L.acc = off;
@@ -109,78 +137,95 @@ __device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, boo
 }
 
 // ---- 1. work list -----------------------------------------------------------
-constexpr int PLAN_THREADS = 1024;
+constexpr int PLAN_THREADS = 1024;  // the grouping plan (pa_plan_shared_kernel)
 static_assert(PLAN_THREADS % 32 == 0 && PLAN_THREADS <= 1024, "plan block: whole warps, at most 32");
 constexpr int PLAN_MAX_BINS = 129;  // tiles per partition <= 128
 
-__global__ void __launch_bounds__(PLAN_THREADS) pa_plan_kernel(const DecodeParams p) {
+// Warp-wide inclusive prefix sum.
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(FULL_MASK, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+// The plain plan runs as ONE warp limited to 32 registers a thread, so that it
+// fits beside a persistent attention CTA on the SM it lands on (the attention
+// kernels leave at least 1024 registers of an SM free) and no attention CTA
+// waits for it to finish. The attention warps only need its results (work-list
+// tail order, zeroed cursor and merge counters) from their first dynamic claim
+// or first finished partition on; their first units come from the full
+// partitions, whose order they compute themselves (UnitSource::init).
+//
+// Work-list order: every sequence's full partitions in sequence order, then
+// the last, partial partitions, longest first.
+constexpr int PLAN_WARP_THREADS = 32;
+
+__global__ void __maxnreg__(32) pa_plan_kernel(const DecodeParams p) {
     __shared__ int s_bin_count[PLAN_MAX_BINS];
     __shared__ int s_bin_next[PLAN_MAX_BINS];
-    __shared__ int s_warp[32];
-    __shared__ int s_carry;
     // Let the attention kernel launch now; it waits for this grid's results.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int P = p.partition, tiles = P / 16;
-    for (int i = tid; i < PLAN_MAX_BINS; i += PLAN_THREADS) s_bin_count[i] = 0;
-    for (int i = tid; i < p.num_seqs * p.num_kv_heads; i += PLAN_THREADS) p.merge_count[i] = 0;
-    if (tid == 0) s_carry = 0;
-    __syncthreads();
+    const int lane = threadIdx.x;
+    const int B = p.num_seqs, P = p.partition, tiles = P / 16;
+    for (int i = lane; i < PLAN_MAX_BINS; i += 32) s_bin_count[i] = 0;
+    {
+        // Merge and chunk counters (one region): 16-byte stores (it is 256-byte aligned).
+        const int n = B * p.num_kv_heads * (1 + p.max_chunks);
+        int4 *c4 = reinterpret_cast<int4 *>(p.merge_count);
+        for (int i = lane; i < n / 4; i += 32) c4[i] = make_int4(0, 0, 0, 0);
+        for (int i = (n / 4) * 4 + lane; i < n; i += 32) p.merge_count[i] = 0;
+    }
+    __syncwarp();
 
     // Pass 1: full partitions in sequence order; histogram of the tails.
-    for (int base = 0; base < p.num_seqs; base += PLAN_THREADS) {
-        const int s = base + tid;
-        const int ctx = s < p.num_seqs ? clamped_context(p, s, true) : 0;
+    int carry = 0;
+    for (int base = 0; base < B; base += 32) {
+        const int s = base + lane;
+        const int ctx = s < B ? clamped_context(p, s, true) : 0;
         const int full = ctx / P, tail = ctx - full * P;
         if (tail > 0) atomicAdd(&s_bin_count[(tail + 15) >> 4], 1);
-        int incl = full;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(FULL_MASK, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) s_warp[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            const int w = lane < PLAN_THREADS / 32 ? s_warp[lane] : 0;  // warps of the block only
-            int wi = w;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(FULL_MASK, wi, o);
-                if (lane >= o) wi += v;
-            }
-            s_warp[lane] = wi - w;
-        }
-        __syncthreads();
-        const int off = s_carry + s_warp[warp] + incl - full;
+        const int incl = warp_incl_scan(full, lane);
+        const int off = carry + incl - full;
         const int nparts = full + (tail > 0);
         for (int j = 0; j < full; ++j) p.entries[off + j] = make_int4(s, j, P, nparts);
-        __syncthreads();
-        if (tid == PLAN_THREADS - 1) s_carry = off + full;
-        __syncthreads();
+        carry += __shfl_sync(FULL_MASK, incl, 31);
     }
-    if (tid == 0) {
-        int pos = s_carry;
-        for (int b = tiles; b >= 1; --b) {
-            s_bin_next[b] = pos;
-            pos += s_bin_count[b];
-        }
+    __syncwarp();
+    // Tails after the full partitions, longest first: start of each bin by a
+    // scan over the bins in descending order.
+    int pos = carry;
+    for (int b0 = tiles; b0 >= 1; b0 -= 32) {
+        const int b = b0 - lane;
+        const int cnt = b >= 1 ? s_bin_count[b] : 0;
+        const int incl = warp_incl_scan(cnt, lane);
+        if (b >= 1) s_bin_next[b] = pos + incl - cnt;
+        pos += __shfl_sync(FULL_MASK, incl, 31);
+    }
+    if (lane == 0) {
         *p.num_entries = pos;
         *p.counter = 0;
     }
-    __syncthreads();
-    // Pass 2: each sequence's last, partial partition, longest first. An
-    // empty sequence gets no work; its output rows are zeroed here.
-    for (int s = tid; s < p.num_seqs; s += PLAN_THREADS) {
-        const int ctx = clamped_context(p, s, false);
+    __syncwarp();
+    // Pass 2: each sequence's last, partial partition. An empty sequence gets
+    // no work; the warp zeroes its output rows here.
+    for (int base = 0; base < B; base += 32) {
+        const int s = base + lane;
+        const int ctx = s < B ? clamped_context(p, s, false) : -1;
         const int full = ctx / P, tail = ctx - full * P;
-        if (tail > 0) {
-            const int pos = atomicAdd(&s_bin_next[(tail + 15) >> 4], 1);
-            p.entries[pos] = make_int4(s, full, tail, full + 1);
-        } else if (ctx == 0) {
-            const int nvec = p.num_heads * p.head_dim / 8;
-            uint4 *row = static_cast<uint4 *>(p.out) + (size_t)s * nvec;
-            for (int i = 0; i < nvec; ++i) row[i] = make_uint4(0, 0, 0, 0);
+        if (s < B && tail > 0) {
+            const int at = atomicAdd(&s_bin_next[(tail + 15) >> 4], 1);
+            p.entries[at] = make_int4(s, full, tail, full + 1);
+        }
+        unsigned empty = __ballot_sync(FULL_MASK, ctx == 0);
+        const int nvec = p.num_heads * p.head_dim / 8;
+        while (empty) {
+            const int e = __ffs(empty) - 1;
+            empty &= empty - 1;
+            uint4 *row = static_cast<uint4 *>(p.out) + (size_t)(base + e) * nvec;
+            for (int i = lane; i < nvec; i += 32) row[i] = make_uint4(0, 0, 0, 0);
         }
     }
 }
@@ -547,11 +592,23 @@ struct Unit {
 // per CTA, at most the number of warps) are therefore spread: claim c takes
 // unit (c % K) * (wave1 / K) + c / K, K warps per CTA, so each CTA's first
 // units come from every part of the list; later claims go in list order.
+//
+// Early start (init_early, the tensor-core kernels with the one-warp plan):
+// the first wave is assigned statically instead — warp w of CTA b takes unit
+// w * (number of CTAs) + b, a spread over every CTA — and the warp computes that unit's
+// work-list entry itself when it is a full partition (the list starts with
+// every sequence's full partitions in sequence order, a prefix sum over the
+// context lengths). Later claims take wave1 + the cursor. The warp waits for
+// the plan kernel (griddepcontrol.wait) only before it first needs its
+// results: the cursor, a tail entry, or a merge counter.
 struct UnitSource {
     const DecodeParams *p;
     int lane, total_units, Hkv, bs, blocks_per_part;
     int k, wave1;  // warps per CTA; claims spread over the first wave
     bool shared;   // entries carry a second int4 (first token, members)
+    bool early;    // static first wave; cursor claims start at wave1
+    bool planned;  // the plan kernel's results are visible to this warp
+    bool claimed;  // u holds lane 0's raw cursor value, to be broadcast and mapped
     int state;    // 0 idle, 1 cursor claimed, 2 entry loaded, 3 table loaded, 4 list exhausted
     int u, tbl, mseq, mnp;
     int4 ent, entb;
@@ -567,6 +624,9 @@ struct UnitSource {
         bs = params.block_size;
         blocks_per_part = params.partition / params.block_size;
         shared = shared_units;
+        early = false;
+        planned = true;
+        claimed = false;
         state = 0;
         u = 0;
         tbl = 0;
@@ -574,19 +634,91 @@ struct UnitSource {
         ent = entb = make_int4(0, 0, 0, 0);
     }
 
+    // Early start: sets total_units from the context lengths and the warp's
+    // static first claim (warp `warp` of CTA `cta`); nothing here reads what
+    // the plan kernel writes. Returns total_units.
+    __device__ int init_early(const DecodeParams &params, int lane_id, int warps_per_cta, int warps_total, int cta,
+                              int warp) {
+        init(params, lane_id, 0, false, warps_per_cta, warps_total);
+        early = true;
+        planned = false;
+        const int B = params.num_seqs, P = params.partition;
+        int tfull = 0, ntail = 0;
+        for (int base = 0; base < B; base += 32) {
+            const int s = base + lane;
+            const int ctx = s < B ? clamped_context(params, s, false) : 0;
+            int f = ctx / P;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) f += __shfl_xor_sync(FULL_MASK, f, o);
+            tfull += f;
+            ntail += __popc(__ballot_sync(FULL_MASK, ctx % P != 0));
+        }
+        total_units = (tfull + ntail) * Hkv;
+        // Warp-major over the CTAs: every CTA gets first units, from every part
+        // of the longest-first list, even when there are fewer units than warps.
+        wave1 = min(warps_total, total_units);
+        u = warp * (warps_total / k) + cta;
+        if (u >= wave1) return total_units;  // no static claim: the cursor from the start
+        const int e = u / Hkv;
+        state = 1;  // a tail entry: read from the plan's list (step() waits for it)
+        if (e < tfull) {
+            // The full partition e: sequence s with pre(s) <= e < pre(s) + full(s).
+            int carry = 0;
+            for (int base = 0; base < B; base += 32) {
+                const int s = base + lane;
+                const int ctx = s < B ? clamped_context(params, s, false) : 0;
+                const int f = ctx / P;
+                int incl = f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(FULL_MASK, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const unsigned hit = __ballot_sync(FULL_MASK, carry + incl - f <= e && e < carry + incl);
+                if (hit) {
+                    const int src = __ffs(hit) - 1;
+                    const int j = __shfl_sync(FULL_MASK, e - (carry + incl - f), src);
+                    const int np = __shfl_sync(FULL_MASK, f + (ctx % P != 0), src);
+                    ent = make_int4(base + src, j, P, np);
+                    state = 2;
+                    break;
+                }
+                carry += __shfl_sync(FULL_MASK, incl, 31);
+            }
+        }
+        return total_units;
+    }
+
+    // Makes the plan kernel's results visible to this warp (once).
+    __device__ __forceinline__ void wait_plan() {
+        if (!planned) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            planned = true;
+        }
+    }
+
     __device__ __forceinline__ void step() {
         if (state == 0) {
+            wait_plan();
             int v = 0;
             if (lane == 0) v = atomicAdd(p->counter, 1);
             u = v;  // lane 0 only; broadcast in the next link
+            claimed = true;
             state = 1;
         } else if (state == 1) {
-            u = __shfl_sync(FULL_MASK, u, 0);
-            if (u < wave1) u = (u % k) * (wave1 / k) + u / k;
+            if (claimed) {
+                u = __shfl_sync(FULL_MASK, u, 0);
+                if (early)
+                    u += wave1;
+                else if (u < wave1)
+                    u = (u % k) * (wave1 / k) + u / k;
+                claimed = false;
+            }
             if (u >= total_units) {
                 state = 4;
                 return;
             }
+            wait_plan();
             ent = p->entries[u / Hkv];
             if (shared) entb = p->entries_b[u / Hkv];
             state = 2;

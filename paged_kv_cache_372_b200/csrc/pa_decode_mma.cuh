@@ -96,6 +96,18 @@ __device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t codes) {
     return r;
 }
 
+// INT8 cache, stored excess-128 (byte u holds u - 128): the f16 number with
+// high byte 0x64 and low byte u is exactly 1024 + u, so one byte permute per
+// pair of codes makes the MMA operand; the constant 1152 = 1024 + 128 is
+// taken off afterwards (from the scores per query row, from the outputs with
+// the softmax sum). Codes in bytes 0 and 1 (low byte first) -> two f16.
+__device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t codes) { return __byte_perm(codes, 0x64646464u, 0x4140); }
+// Codes in bytes 2 and 3 -> two f16.
+__device__ __forceinline__ uint32_t i8x2_hi_to_f16x2(uint32_t codes) {
+    return __byte_perm(codes, 0x64646464u, 0x4342);
+}
+constexpr float I8_OFFSET = 1152.f;
+
 // Two 16-bit query elements of type T -> f16x2 (bf16 -> f16 is exact in f16's
 // normal range). A bf16 element above f16's largest finite value (65504)
 // would become infinite: `big` is set so that the caller can flag it.
@@ -170,24 +182,29 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)((chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
-// Merge of one (sequence, KV head)'s partitions for this kernel's partial
-// layout: [part][D][G] floats and [part][G] (max, sum) pairs (head-innermost,
-// so the accumulator fragments store as pairs). All G heads in one pass: lane
-// j computes partition j's G weights (32 partitions per round), the weights
-// reach the other lanes by shuffle, and each lane reads its EPL x G contiguous
-// floats of every partition with vector loads.
+// Merge of partial slots [first, first + nparts) of one (sequence, KV head)
+// for this kernel's partial layout: [slot][D][G] floats and [slot][G] (max,
+// sum) pairs (head-innermost, so the accumulator fragments store as pairs).
+// All G heads in one pass: lane j computes slot j's G weights (32 slots per
+// round), the weights reach the other lanes by shuffle, and each lane reads
+// its EPL x G contiguous floats of every slot with vector loads. With
+// dst_slot < 0 the result is normalised into the output rows; otherwise it is
+// written, unnormalised with its (max, sum), to partial slot dst_slot (a chunk
+// merge, see MERGE_FANIN).
 // LEAN (kernels under a 128-register cap) keeps fewer values live: the
 // (max, sum) pairs are read twice and no partials are loaded ahead.
 template <int D, int G, typename T, bool LEAN = false>
-__device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, size_t head0, int nparts, int lane) {
+__device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, size_t head0, int first, int nparts,
+                                          int lane, int dst_slot = -1) {
     constexpr int EPL = D / 32;
     constexpr int F = EPL * G;                             // floats of one partition per lane
     constexpr int VW = F >= 4 ? 4 : F;                     // floats per vector load (4 or 2)
     constexpr int NV4 = F / VW;                            // vector loads per partition per lane
-    // partitions whose partials load up front
+    // partitions whose partials load up front, and in flight in the loop
     constexpr int PF = LEAN ? 0 : (F <= 8 ? 4 : (F <= 16 ? 1 : 0));
-    const float2 *ml = p.ml + group * p.max_parts * G;
-    const float *acc = p.part_acc + group * p.max_parts * (size_t)(D * G);
+    constexpr int MERGE_UNROLL = F >= 32 ? 2 : 4;
+    const float2 *ml = p.ml + (group * p.max_parts + first) * G;
+    const float *acc = p.part_acc + (group * p.max_parts + first) * (size_t)(D * G);
     auto load = [&](int j, float (&f)[F]) {
         const float *a = acc + (size_t)j * D * G + lane * F;
 #pragma unroll
@@ -257,7 +274,7 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
             }
             jj = PF;
         }
-#pragma unroll 4
+#pragma unroll MERGE_UNROLL
         for (; jj < n; ++jj) {
             float f[F];
             load(base + jj, f);
@@ -272,6 +289,22 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
     for (int off = 16; off >= 1; off >>= 1)
 #pragma unroll
         for (int g = 0; g < G; ++g) L[g] += __shfl_xor_sync(FULL_MASK, L[g], off);
+    if (dst_slot >= 0) {
+        const size_t slot = group * p.max_parts + dst_slot;
+        float *dst = p.part_acc + slot * (size_t)(D * G) + lane * F;
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) {
+            if constexpr (VW == 4)
+                __stcg(reinterpret_cast<float4 *>(dst) + i,
+                       make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
+            else
+                __stcg(reinterpret_cast<float2 *>(dst) + i, make_float2(o[2 * i], o[2 * i + 1]));
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            if (lane == g) p.ml[slot * G + g] = make_float2(M[g], L[g]);
+        return;
+    }
     T *out = static_cast<T *>(p.out);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -283,10 +316,74 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
     }
 }
 
-template <int D, int G, typename T, int NS, bool KV8 = false, bool SHARED = false>
+// The split-context merge as its own launch (DecodeParams::reduce_launch, for
+// sequences of many partitions; see REDUCE_LAUNCH_MIN_PARTS): one CTA
+// per (sequence, KV head), REDUCE_GROUPS thread groups of D*G/4 threads, each
+// thread one float4 of the [D][G] partial row of every partition in its
+// group's share (partitions r, r + REDUCE_GROUPS, ...); the groups' sums
+// combine in shared memory. The arithmetic of mma_merge:
+// out = sum_j 2^(m_j - M) acc_j / sum_j 2^(m_j - M) l_j.
+constexpr int REDUCE_GROUPS = 4;
+
+template <int D, int G, typename T>
+__global__ void pa_reduce_kernel(const DecodeParams p) {
+    constexpr int V4 = D * G / 4;
+    extern __shared__ float4 s_red[];  // [REDUCE_GROUPS][V4] sums, [REDUCE_GROUPS][V4] weight sums, (max, sum)s
+    float2 *s_ml = reinterpret_cast<float2 *>(s_red + 2 * REDUCE_GROUPS * V4);  // [nparts][G]
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int group = blockIdx.x, s = group / p.num_kv_heads, kvh = group - s * p.num_kv_heads;
+    const int ctx = clamped_context(p, s, false);
+    const int nparts = (ctx + p.partition - 1) / p.partition;
+    if (nparts <= 1) return;  // written by the attention kernel
+    const float2 *ml = p.ml + (size_t)group * p.max_parts * G;
+    for (int i = threadIdx.x; i < nparts * G; i += blockDim.x) s_ml[i] = __ldcg(ml + i);
+    __syncthreads();
+    const int v = threadIdx.x % V4, r = threadIdx.x / V4;
+    float M[4], acc[4] = {0.f, 0.f, 0.f, 0.f}, L[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int g = (4 * v + c) % G;
+        M[c] = -INFINITY;
+        for (int j = 0; j < nparts; ++j) M[c] = fmaxf(M[c], s_ml[j * G + g].x);
+    }
+    const float4 *part = reinterpret_cast<const float4 *>(p.part_acc + (size_t)group * p.max_parts * (D * G));
+#pragma unroll 4
+    for (int j = r; j < nparts; j += REDUCE_GROUPS) {
+        const float4 a = __ldcg(part + (size_t)j * V4 + v);
+        const float f[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float2 m = s_ml[j * G + (4 * v + c) % G];
+            const float w = exp2f(m.x - M[c]);
+            acc[c] = fmaf(w, f[c], acc[c]);
+            L[c] = fmaf(w, m.y, L[c]);
+        }
+    }
+    s_red[r * V4 + v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    s_red[(REDUCE_GROUPS + r) * V4 + v] = make_float4(L[0], L[1], L[2], L[3]);
+    __syncthreads();
+    if (r != 0) return;
+    float o[4] = {0.f, 0.f, 0.f, 0.f}, l[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < REDUCE_GROUPS; ++q) {
+        const float4 a = s_red[q * V4 + v], b = s_red[(REDUCE_GROUPS + q) * V4 + v];
+        o[0] += a.x; o[1] += a.y; o[2] += a.z; o[3] += a.w;
+        l[0] += b.x; l[1] += b.y; l[2] += b.z; l[3] += b.w;
+    }
+    T *out = static_cast<T *>(p.out);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int e = 4 * v + c, d = e / G, g = e % G;
+        out[((size_t)s * p.num_heads + (size_t)kvh * G + g) * D + d] = static_cast<T>(o[c] / l[c]);
+    }
+}
+
+template <int D, int G, typename T, int NS, bool KV8 = false, bool SHARED = false, bool I8 = false, bool HS = false>
 __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
+    static_assert(!I8 || KV8, "INT8 codes are an 8-bit cache");
+    static_assert(!HS || KV8, "per-head scales are an 8-bit cache's");
     using Gm = MmaGeo<D, G, KV8>;
     constexpr int QB = mma_q_slot_bytes<D, G, SHARED>();  // bytes of one query slot
     constexpr int QS = mma_q_slots<SHARED>();              // query slots per warp
@@ -317,13 +414,16 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
     }
     __syncwarp();
     const uint64_t policy = l2_policy_evict_first();
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-
     const T *qg = static_cast<const T *>(p.q);
-    const int total_units = *p.num_entries * Hkv;
 
     UnitSource src;
-    src.init(p, lane, total_units, SHARED, warps, warps * (int)gridDim.x);
+    if (!SHARED && p.early) {
+        // The plan kernel runs alongside: first units from the contexts alone.
+        src.init_early(p, lane, warps, warps * (int)gridDim.x, blockIdx.x, warp);
+    } else {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        src.init(p, lane, *p.num_entries * Hkv, SHARED, warps, warps * (int)gridDim.x);
+    }
     auto fetch = [&](Unit &x) { src.take(x); };
 
     // Item `it` of a unit is its tile `it`: the K and V rows of 16 tokens;
@@ -431,6 +531,8 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
         }
     };
 
+    // Waits for the next item to consume; on a timeout it flags it, waits
+    // (bounded) for every copy still in flight, and reports failure.
     auto wait_item = [&]() -> bool {
         const uint32_t stage = consumed % NS, parity = (consumed / NS) & 1;
         bool ok = mbar_wait_bounded(bar_s + 8 * stage, parity, WAIT_LIMIT_NS);
@@ -472,6 +574,15 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
         // Lanes [0, NVR) hold one 16-byte vector of the new K row, lanes
         // [NVR, 2*NVR) of the new V row; loaded now, used at the last tile.
         const bool app_unit = append && cur.part == cur.nparts - 1;
+        // Dequantisation of an 8-bit cache: the key scale folds into the
+        // score scale uq, the value scale uv applies at the store (per unit
+        // with per-head scales, HS; kernel parameters otherwise). kc0 / kc1
+        // take the INT8 offset off the scores of query rows h0 / h1.
+        float uq = p.qscale, uv = p.v_scale, kc0 = 0.f, kc1 = 0.f;
+        if constexpr (HS) {
+            uq = p.qscale * __ldg(p.k_scales + cur.kvh);
+            uv = __ldg(p.v_scales + cur.kvh);
+        }
         uint4 newrow = make_uint4(0, 0, 0, 0);
         if (app_unit && lane < 2 * NVR) {
             const size_t rowoff = ((size_t)cur.s * Hkv + cur.kvh) * D;
@@ -509,6 +620,21 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                 if constexpr (KV8 && !std::is_same<T, __half>::value) {
                     if (__any_sync(FULL_MASK, qbig) && lane == 0) raise_error(PA_DEVERR_QRANGE);
                 }
+                if constexpr (I8) {
+                    // Sum of query row g8 (the f16 values the MMA multiplies),
+                    // over the quad's lanes, then rows h0 and h1 of this lane.
+                    float qs = 0.f;
+#pragma unroll
+                    for (int i = 0; i < Gm::KS; ++i) {
+                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&qb[i][0]));
+                        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&qb[i][1]));
+                        qs += (a.x + a.y) + (b.x + b.y);
+                    }
+                    qs += __shfl_xor_sync(FULL_MASK, qs, 1);
+                    qs += __shfl_xor_sync(FULL_MASK, qs, 2);
+                    kc0 = -I8_OFFSET * uq * __shfl_sync(FULL_MASK, qs, 8 * t4);
+                    kc1 = -I8_OFFSET * uq * __shfl_sync(FULL_MASK, qs, 8 * t4 + 4);
+                }
             }
             const int valid = min(16, cur.ntok - 16 * k);
             if (app_unit && k == cur.ntiles - 1) {
@@ -545,8 +671,14 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
-                        const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi), e4m3x2_hi_to_f16x2(lo),
-                                               e4m3x2_hi_to_f16x2(hi)};
+                        uint32_t a[4];
+                        if constexpr (I8) {
+                            a[0] = i8x2_to_f16x2(lo); a[1] = i8x2_to_f16x2(hi);
+                            a[2] = i8x2_hi_to_f16x2(lo); a[3] = i8x2_hi_to_f16x2(hi);
+                        } else {
+                            a[0] = e4m3x2_to_f16x2(lo); a[1] = e4m3x2_to_f16x2(hi);
+                            a[2] = e4m3x2_hi_to_f16x2(lo); a[3] = e4m3x2_hi_to_f16x2(hi);
+                        }
                         MmaType<__half>::mma(h ? s2 : s, a, qb[i + h][0], qb[i + h][1]);
                     }
                 }
@@ -564,10 +696,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             for (int j = 0; j < 4; ++j) s[j] += s2[j];
             // s[0], s[1]: token g8, heads h0, h1; s[2], s[3]: token g8 + 8.
             const bool v_lo = g8 < valid, v_hi = g8 + 8 < valid;
-            float x0 = v_lo ? s[0] * p.qscale : -INFINITY;
-            float x1 = v_lo ? s[1] * p.qscale : -INFINITY;
-            float x2 = v_hi ? s[2] * p.qscale : -INFINITY;
-            float x3 = v_hi ? s[3] * p.qscale : -INFINITY;
+            float x0 = v_lo ? fmaf(s[0], uq, kc0) : -INFINITY;
+            float x1 = v_lo ? fmaf(s[1], uq, kc1) : -INFINITY;
+            float x2 = v_hi ? fmaf(s[2], uq, kc0) : -INFINITY;
+            float x3 = v_hi ? fmaf(s[3], uq, kc1) : -INFINITY;
             bool raise = (hv0 && !(fmaxf(x0, x2) <= M0 + LAZY_MAX_LOG2)) ||
                          (hv1 && !(fmaxf(x1, x3) <= M1 + LAZY_MAX_LOG2));
             if (__any_sync(FULL_MASK, raise)) {
@@ -627,10 +759,19 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                     ldsm_x4_trans(r, vs_s + swz(row, i + csel));
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const uint32_t x = __byte_perm(r[2 * h], 0, 0x3120);      // tokens 0-7
-                        const uint32_t y = __byte_perm(r[2 * h + 1], 0, 0x3120);  // tokens 8-15
-                        const uint32_t a[4] = {e4m3x2_to_f16x2(x), e4m3x2_hi_to_f16x2(x), e4m3x2_to_f16x2(y),
-                                               e4m3x2_hi_to_f16x2(y)};
+                        uint32_t a[4];
+                        if constexpr (I8) {
+                            // Bytes 0 / 2 are element 2*g8 of the two tokens, 1 / 3 element 2*g8+1.
+                            a[0] = __byte_perm(r[2 * h], 0x64646464u, 0x4240);
+                            a[1] = __byte_perm(r[2 * h], 0x64646464u, 0x4341);
+                            a[2] = __byte_perm(r[2 * h + 1], 0x64646464u, 0x4240);
+                            a[3] = __byte_perm(r[2 * h + 1], 0x64646464u, 0x4341);
+                        } else {
+                            const uint32_t x = __byte_perm(r[2 * h], 0, 0x3120);      // tokens 0-7
+                            const uint32_t y = __byte_perm(r[2 * h + 1], 0, 0x3120);  // tokens 8-15
+                            a[0] = e4m3x2_to_f16x2(x); a[1] = e4m3x2_hi_to_f16x2(x);
+                            a[2] = e4m3x2_to_f16x2(y); a[3] = e4m3x2_hi_to_f16x2(y);
+                        }
                         MmaType<__half>::mma(o[i + h], a, pb0, pb1);
                     }
                 }
@@ -658,6 +799,16 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             l0 += __shfl_xor_sync(FULL_MASK, l0, off);
             l1 += __shfl_xor_sync(FULL_MASK, l1, off);
         }
+        if constexpr (I8) {
+            // The values were multiplied as 1152 + code: take 1152 * (sum of the weights) off.
+#pragma unroll
+            for (int i = 0; i < Gm::KS; ++i) {
+                o[i][0] = fmaf(-I8_OFFSET, l0, o[i][0]);
+                o[i][2] = fmaf(-I8_OFFSET, l0, o[i][2]);
+                o[i][1] = fmaf(-I8_OFFSET, l1, o[i][1]);
+                o[i][3] = fmaf(-I8_OFFSET, l1, o[i][3]);
+            }
+        }
         const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;
         if (SHARED && cur.mcnt > 0) {
             // Partials of every member: column h of the accumulators is query
@@ -669,7 +820,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             float *acc0 = p.part_acc + row0 * (size_t)(D * G);
             float *acc1 = p.part_acc + row1 * (size_t)(D * G);
             const int g0 = h0 % G, g1 = h1 % G;
-            const float vs = KV8 ? p.v_scale : 1.f;
+            const float vs = KV8 ? uv : 1.f;
 #pragma unroll
             for (int i = 0; i < Gm::KS; ++i) {
                 const int d = KV8 ? 16 * i + 2 * g8 : 16 * i + g8;
@@ -691,20 +842,25 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             if (g8 == 0 && hv0) p.ml[row0 * G + g0] = make_float2(M0, l0);
             if (g8 == 0 && hv1) p.ml[row1 * G + g1] = make_float2(M1, l1);
             // Lane j counts member j's partition.
+            src.wait_plan();  // the merge counters are zeroed by the plan kernel
             const bool last = count_partition(&p.merge_count[(size_t)cur.mseq * Hkv + cur.kvh], cur.mnp,
                                               lane < cur.mcnt);
+            // Members whose last partition this was, merged one after another
+            // (merging them together, with all members' loads in flight at
+            // once, was measured slower: it needs more registers).
             unsigned lm = __ballot_sync(FULL_MASK, last);
             while (lm) {
                 const int j = __ffs(lm) - 1;
                 lm &= lm - 1;
                 const int sj = __shfl_sync(FULL_MASK, cur.mseq, j);
                 const int nj = __shfl_sync(FULL_MASK, cur.mnp, j);
-                mma_merge<D, G, T, KV8>(p, (size_t)sj * Hkv + cur.kvh, (size_t)sj * H + (size_t)cur.kvh * G, nj, lane);
+                mma_merge<D, G, T, KV8>(p, (size_t)sj * Hkv + cur.kvh, (size_t)sj * H + (size_t)cur.kvh * G, 0, nj,
+                                        lane);
             }
         } else if (KV8 && cur.nparts == 1) {
             // Accumulator rows g8 / g8+8 of slice i are elements 16i + 2*g8 / + 1:
             // pairs of adjacent elements per head, stored directly.
-            const float i0 = hv0 ? p.v_scale / l0 : 0.f, i1 = hv1 ? p.v_scale / l1 : 0.f;
+            const float i0 = hv0 ? uv / l0 : 0.f, i1 = hv1 ? uv / l1 : 0.f;
             T *out = static_cast<T *>(p.out) + head0 * D;
 #pragma unroll
             for (int i = 0; i < Gm::KS; ++i) {
@@ -731,7 +887,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             float *acc = p.part_acc + row * (size_t)(D * G);
             // Rows g8 / g8+8 of slice i: elements 16i + g8 / + 8 (16-bit cache)
             // or 16i + 2*g8 / + 1 (fp8 cache, values scaled by v_scale).
-            const float vs = KV8 ? p.v_scale : 1.f;
+            const float vs = KV8 ? uv : 1.f;
 #pragma unroll
             for (int i = 0; i < Gm::KS; ++i) {
                 const int d = KV8 ? 16 * i + 2 * g8 : 16 * i + g8;
@@ -748,10 +904,37 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             }
             if (g8 == 0 && hv0) p.ml[row * G + h0] = make_float2(M0, l0);
             if (g8 == 0 && hv1) p.ml[row * G + h1] = make_float2(M1, l1);
-            const bool last = count_partition(&p.merge_count[group], cur.nparts, lane == 0);
-            if (__shfl_sync(FULL_MASK, last, 0)) mma_merge<D, G, T, KV8>(p, group, head0, cur.nparts, lane);
+            if (!SHARED && p.reduce_launch) goto next_unit;  // merged by pa_reduce_kernel
+            src.wait_plan();  // the merge counters are zeroed by the plan kernel
+            // One level (at most MERGE_FANIN partitions, or shared-prefix units'
+            // workspace), or two: this partition's chunk into its chunk
+            // partial, then the chunk partials. One merge call site in a loop
+            // keeps the merge inlined once.
+            const bool chunked = cur.nparts > MERGE_FANIN && p.max_chunks > 0;
+            const int nch = (cur.nparts + MERGE_FANIN - 1) / MERGE_FANIN;
+            int first = 0, n = cur.nparts, dst = -1;
+            bool go;
+            if (chunked) {
+                const int c = cur.part / MERGE_FANIN;
+                first = c * MERGE_FANIN;
+                n = min(MERGE_FANIN, cur.nparts - first);
+                dst = p.l1_base + c;
+                go = count_partition(&p.chunk_count[group * p.max_chunks + c], n, lane == 0);
+            } else {
+                go = count_partition(&p.merge_count[group], cur.nparts, lane == 0);
+            }
+#pragma unroll 1
+            while (__shfl_sync(FULL_MASK, go, 0)) {
+                mma_merge<D, G, T, KV8>(p, group, head0, first, n, lane, dst);
+                if (dst < 0) break;
+                go = count_partition(&p.merge_count[group], nch, lane == 0);
+                first = p.l1_base;
+                n = nch;
+                dst = -1;
+            }
         }
 
+    next_unit:
         while (!prod_on_nxt && !exhausted) produce();
         if (!prod_on_nxt) break;
         cur = nxt;

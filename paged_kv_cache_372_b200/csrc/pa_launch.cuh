@@ -5,6 +5,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "pa_decode.cuh"
 #include "pa_decode_mma.cuh"
 
@@ -56,6 +58,17 @@ int resolve_partition(int group, int block_size, int max_context_len, int reques
     return auto_p;
 }
 
+// Raises kernel Kernel's dynamic shared-memory limit on this device, once per
+// (kernel, device, size): one flag array per kernel function, not per type.
+template <auto Kernel>
+cudaError_t set_dynamic_smem(int dev, int smem) {
+    static std::atomic<int> done[kMaxDevices];
+    if (done[dev].load(std::memory_order_acquire) == smem) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) done[dev].store(smem, std::memory_order_release);
+    return e;
+}
+
 template <int D, int G, typename T>
 pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
     constexpr int NS = pa::DECODE_STAGES;
@@ -68,7 +81,7 @@ pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
     if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "%d bytes of shared memory per warp", per_warp);
     const int smem = warps * per_warp;
     auto kernel = pa::pa_decode_kernel<D, G, T, NS>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_dynamic_smem<pa::pa_decode_kernel<D, G, T, NS>>(info.dev, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
     if (p.k_new) {
@@ -78,7 +91,7 @@ pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
         if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
         pa::pa_append_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
     }
-    pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
+    pa::pa_plan_kernel<<<1, pa::PLAN_WARP_THREADS, 0, stream>>>(p);
     // Programmatic dependent launch: the attention CTAs start their set-up
     // while the plan kernel runs and wait for its results in-kernel.
     cudaLaunchConfig_t cfg = {};
@@ -117,9 +130,33 @@ pa_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled *out) {
 
 // A pool [num_blocks][num_kv_heads][block_size][D] as a 2-D tensor of
 // rows x D elements, read in boxes of 16 rows x 128 bytes (64 16-bit or 128
-// 8-bit elements) with the 128-byte shared-memory swizzle.
+// 8-bit elements) with the 128-byte shared-memory swizzle. Encoded maps are
+// kept (the last kMapCache distinct pools), since a serving loop decodes over
+// the same pools call after call.
+constexpr int kMapCache = 16;
+
 pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, int D, int elem_bytes,
-                          CUtensorMapDataType type) {
+                          CUtensorMapDataType type, int dev) {
+    struct Entry {
+        const void *pool;
+        long long rows;
+        int D, elem_bytes, type, dev;
+        CUtensorMap map;
+    };
+    static std::mutex mu;
+    static Entry cache[kMapCache];
+    static int filled = 0, next = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < filled; ++i) {
+            const Entry &c = cache[i];
+            if (c.pool == pool && c.rows == rows && c.D == D && c.elem_bytes == elem_bytes && c.type == (int)type &&
+                c.dev == dev) {
+                *map = c.map;
+                return PA_OK;
+            }
+        }
+    }
     PFN_cuTensorMapEncodeTiled enc;
     pa_status st = tensor_map_encoder(&enc);
     if (st != PA_OK) return st;
@@ -130,10 +167,42 @@ pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, in
     CUresult r = enc(map, type, 2, const_cast<void *>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    std::lock_guard<std::mutex> lock(mu);
+    Entry &c = cache[next];
+    c.pool = pool;
+    c.rows = rows;
+    c.D = D;
+    c.elem_bytes = elem_bytes;
+    c.type = (int)type;
+    c.dev = dev;
+    c.map = *map;
+    next = (next + 1) % kMapCache;
+    if (filled < kMapCache) ++filled;
     return PA_OK;
 }
 
-template <int D, int G, typename T, bool KV8 = false, bool SHARED = false>
+// Sequences up to which the tensor-core kernels start without waiting for the
+// plan (each warp passes over the context lengths once or twice at start).
+constexpr int EARLY_MAX_SEQS = 512;
+
+// Partitions a sequence can have above which the split merge runs as its own
+// launch (pa_reduce_kernel, one CTA per (sequence, KV head), its partitions
+// shared by four thread groups) instead of in the attention kernel's
+// last-arriving warps. Measured: long32k with 64 partitions per sequence
+// 189.3 -> 178.1 us (fp8 cache 119.3 -> 107.9 us); llama3_8b, where the few
+// long sequences have up to 11, 146.2 -> 149.5 us (the launch costs more than
+// the merges it moves), so only above this many.
+constexpr int REDUCE_LAUNCH_MIN_PARTS = 16;
+constexpr int REDUCE_SMEM_MAX = 200 * 1024;
+
+// Dynamic shared memory of pa_reduce_kernel<D, G>: the thread groups' sums and
+// the (max, sum) pairs of up to `parts` partitions.
+template <int D, int G>
+size_t reduce_smem_bytes(int parts) {
+    return 2 * pa::REDUCE_GROUPS * (D * G / 4) * 16 + (size_t)parts * G * 8;
+}
+
+template <int D, int G, typename T, bool KV8 = false, bool SHARED = false, bool I8 = false, bool HS = false>
 pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     constexpr int NS = KV8 ? pa::DECODE_MMA_STAGES_FP8 : pa::DECODE_MMA_STAGES;
     DeviceInfo info;
@@ -143,21 +212,26 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     if (rows >= (1ll << 31)) return fail(PA_ERR_UNSUPPORTED, "pool has %lld rows, above 2^31", rows);
     CUtensorMap tmk, tmv;
     const CUtensorMapDataType type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : pa::MmaType<T>::tma_type;
-    if ((st = encode_pool_map(&tmk, p.k_pool, rows, D, KV8 ? 1 : 2, type)) != PA_OK) return st;
-    if ((st = encode_pool_map(&tmv, p.v_pool, rows, D, KV8 ? 1 : 2, type)) != PA_OK) return st;
+    if ((st = encode_pool_map(&tmk, p.k_pool, rows, D, KV8 ? 1 : 2, type, info.dev)) != PA_OK) return st;
+    if ((st = encode_pool_map(&tmv, p.v_pool, rows, D, KV8 ? 1 : 2, type, info.dev)) != PA_OK) return st;
     constexpr int max_warps = pa::mma_max_warps<G, KV8>();
     int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS, KV8, SHARED>();
     if (warps > max_warps) warps = max_warps;
     if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "not enough shared memory for one warp");
     const int smem = pa::mma_smem_bytes<D, G, NS, KV8, SHARED>(warps);
-    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS, KV8, SHARED>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kernel = pa::pa_decode_mma_kernel<D, G, T, NS, KV8, SHARED, I8, HS>;
+    cudaError_t e = set_dynamic_smem<pa::pa_decode_mma_kernel<D, G, T, NS, KV8, SHARED, I8, HS>>(info.dev, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
-    if constexpr (SHARED)
+    if constexpr (SHARED) {
         pa::pa_plan_shared_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
-    else
-        pa::pa_plan_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
+    } else {
+        p.early = p.num_seqs <= EARLY_MAX_SEQS;
+        // Many partitions per sequence: merge them in a launch of their own
+        // (while its (max, sum) pairs fit the reduce kernel's shared memory).
+        p.reduce_launch = p.l1_base > REDUCE_LAUNCH_MIN_PARTS && reduce_smem_bytes<D, G>(p.l1_base) <= REDUCE_SMEM_MAX;
+        pa::pa_plan_kernel<<<1, pa::PLAN_WARP_THREADS, 0, stream>>>(p);
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sms);
     cfg.blockDim = dim3(warps * 32);
@@ -170,19 +244,35 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, p, tmk, tmv);
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+    if constexpr (!SHARED) {
+        if (p.reduce_launch) {
+            constexpr int V4 = D * G / 4;
+            cudaLaunchConfig_t rc = {};
+            rc.gridDim = dim3((unsigned)(p.num_seqs * p.num_kv_heads));
+            rc.blockDim = dim3(pa::REDUCE_GROUPS * V4);
+            rc.dynamicSmemBytes = reduce_smem_bytes<D, G>(p.l1_base);
+            rc.stream = stream;
+            rc.attrs = attr;
+            rc.numAttrs = 1;
+            e = set_dynamic_smem<pa::pa_reduce_kernel<D, G, T>>(info.dev, REDUCE_SMEM_MAX);
+            if (e == cudaSuccess) e = cudaLaunchKernelEx(&rc, pa::pa_reduce_kernel<D, G, T>, p);
+            if (e != cudaSuccess) return cuda_fail(e, "pa_reduce_kernel launch");
+        }
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
     return PA_OK;
 }
 
-// fp8 (E4M3) cache: tensor-core kernel, head_dim 128.
-template <typename T>
+// 8-bit cache (E4M3, or INT8 with I8; per-head scales with HS): tensor-core
+// kernel, head_dim 128.
+template <typename T, bool I8 = false, bool HS = false>
 pa_status dispatch_group_fp8(pa::DecodeParams &p, int group, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_decode_mma<128, 1, T, true>(p, stream);
-        case 2: return launch_decode_mma<128, 2, T, true>(p, stream);
-        case 4: return launch_decode_mma<128, 4, T, true>(p, stream);
-        case 8: return launch_decode_mma<128, 8, T, true>(p, stream);
+        case 1: return launch_decode_mma<128, 1, T, true, false, I8, HS>(p, stream);
+        case 2: return launch_decode_mma<128, 2, T, true, false, I8, HS>(p, stream);
+        case 4: return launch_decode_mma<128, 4, T, true, false, I8, HS>(p, stream);
+        case 8: return launch_decode_mma<128, 8, T, true, false, I8, HS>(p, stream);
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }

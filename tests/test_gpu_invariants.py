@@ -20,12 +20,16 @@ def decode(wl, kp, vp, tables, ctx, q=None, partition=0):
     return out
 
 
-def test_block_permutation_bit_identical():
-    """Physical placement of blocks does not change the result."""
+@pytest.mark.parametrize("partition", [0, 256, 16])
+def test_block_permutation_bit_identical(partition):
+    """Physical placement of blocks does not change the result: with one merge
+    level (auto: at most 8 partitions a sequence here), two (256-token
+    partitions: up to 16, in chunks of 8) and the merge in a launch of its own
+    (16-token partitions: up to 248)."""
     wl = workloads.llama3_8b(4, num_seqs=16)
     st = wl.steps[0]
     kp, vp = wl.k_pool.cuda(), wl.v_pool.cuda()
-    a = decode(wl, kp, vp, st.block_tables, st.context_lens)
+    a = decode(wl, kp, vp, st.block_tables, st.context_lens, partition=partition)
     pi = torch.randperm(wl.num_blocks, generator=torch.Generator().manual_seed(0))
     kp2 = torch.empty_like(kp)
     vp2 = torch.empty_like(vp)
@@ -33,7 +37,7 @@ def test_block_permutation_bit_identical():
     vp2[pi.cuda()] = vp
     tab = st.block_tables.copy()
     tab[tab >= 0] = pi.numpy()[tab[tab >= 0]]
-    b = decode(wl, kp2, vp2, tab, st.context_lens)
+    b = decode(wl, kp2, vp2, tab, st.context_lens, partition=partition)
     assert torch.equal(a, b)
 
 

@@ -69,6 +69,19 @@ def test_long32k_full():
     run_and_compare(workloads.long32k(0))
 
 
+@pytest.mark.parametrize("num_seqs", [512, 513, 700])
+def test_batch_sizes_around_the_early_start_limit(num_seqs):
+    """Up to 512 sequences the attention kernel starts before the plan kernel
+    has finished (each warp derives its first unit from the contexts); above
+    it, it waits for the plan first. Both agree with the oracle."""
+    from paged_kv_cache_372_b200 import inputs
+    gen = inputs.generator(9000 + num_seqs)
+    ctx = inputs.uniform_int(1, 700, num_seqs, gen)
+    wl, _ = workloads._decode_batch("batch", ctx, heads=16, kv_heads=4, head_dim=128, block_size=16,
+                                    dtype="bf16", seed=9100 + num_seqs)
+    run_and_compare(wl, partition_size=128, label=f"batch B={num_seqs} bf16 P=128")
+
+
 @pytest.mark.parametrize("partition", [16, 32, 128, 256])
 def test_split_partitions(partition):
     wl = workloads.llama3_8b(3, num_seqs=10)

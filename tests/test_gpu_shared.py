@@ -254,20 +254,28 @@ def test_beam_workloads(name, fused):
 
 
 def test_without_sharing_equals_plain_decode():
-    """No shared blocks: every unit is an ordinary one, the partitions are
-    pa_decode's, and so the result is bit-identical."""
+    """No shared blocks: every unit is an ordinary one and the partitions are
+    pa_decode's. Where no sequence has more than 8 partitions both merge them
+    in one level, in the same order, so the result is bit-identical; longer
+    sequences merge in two levels in pa_decode (chunks of 8) and in one here,
+    which agree up to fp32 rounding."""
     wl = workloads.llama3_8b(1, num_seqs=24)
     st = wl.steps[0]
     dev = torch.device("cuda")
     kp, vp = wl.k_pool.to(dev), wl.v_pool.to(dev)
     q = st.q.to(dev)
-    tab, ctx = torch.from_numpy(st.block_tables).to(dev), torch.from_numpy(st.context_lens).to(dev)
-    mx = int(st.context_lens.max())
-    a, b = torch.empty_like(q), torch.empty_like(q)
-    pa.pa_decode(a, q, kp, vp, tab, ctx, wl.scale, mx, 128)
-    pa.pa_decode_shared(b, q, kp, vp, tab, ctx, wl.scale, mx, 128)
-    torch.cuda.synchronize()
-    assert torch.equal(a, b)
+    tab = torch.from_numpy(st.block_tables).to(dev)
+    for ctx_np in (np.minimum(st.context_lens, 8 * 128), st.context_lens):
+        ctx = torch.from_numpy(np.ascontiguousarray(ctx_np)).to(dev)
+        mx = int(ctx_np.max())
+        a, b = torch.empty_like(q), torch.empty_like(q)
+        pa.pa_decode(a, q, kp, vp, tab, ctx, wl.scale, mx, 128)
+        pa.pa_decode_shared(b, q, kp, vp, tab, ctx, wl.scale, mx, 128)
+        torch.cuda.synchronize()
+        if mx <= 8 * 128:
+            assert torch.equal(a, b)
+        else:
+            assert float((a.float() - b.float()).abs().max()) <= H.TOL[wl.dtype]
 
 
 def test_too_many_sequences_rejected():
