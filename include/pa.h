@@ -168,15 +168,17 @@ PA_API pa_status pa_decode_append(void *out, const void *q, const void *k_new, c
  * 解析：PagedAttention如何实现高吞吐LLM推理", section KV Cache内存共享; "别再让
  * GPU内存拖后腿了", section 2.2). The library finds them on the device: it
  * sorts the sequences by their first block and, within a run of sequences
- * with the same first block, forms groups of up to 8 / (num_heads /
+ * with the same first block, forms groups of up to 16 / (num_heads /
  * num_kv_heads) consecutive ones. A group's shared part is the leading full
  * blocks that all members have in common with its first member (with k_new,
  * only blocks below the one holding each member's last position). That part
  * is streamed once per KV head for the whole group, with the group's queries
- * side by side in one tensor-core tile. Each member's remaining tokens run
- * as ordinary partitions, and the partitions merge by the log-sum-exp
- * identity. Without shared blocks, the result and the work are those of
- * pa_decode.
+ * side by side in the columns of the tensor-core tiles. Each member's
+ * remaining tokens run as ordinary partitions, and the partitions merge by
+ * the log-sum-exp identity, in a launch of its own after the attention
+ * kernel (one CTA per (member, KV head)). Without shared blocks, the
+ * partitions are those of pa_decode and the result equals pa_decode's up to
+ * the order of the merge's fp32 sums.
  *
  * partition_size 0 picks 16 blocks for grouped heads (group >= 2; smaller
  * units balance better once the shared tiles are streamed once per group),

@@ -235,13 +235,13 @@ __global__ void __maxnreg__(32) pa_plan_kernel(const DecodeParams p) {
 // same physical blocks at the start of their tables ("vLLM架构深度解析：
 // PagedAttention如何实现高吞吐LLM推理", section KV Cache内存共享). Their
 // attention over those blocks is the same product with different queries, so
-// one unit can stream the shared tiles once for up to 8 / G sequences: their
-// G query rows each fill the 8 columns of the MMA tile. Each member's own
+// one unit can stream the shared tiles once for up to 16 / G sequences: their
+// G query rows each fill columns of the MMA tile (two halves of 8). Each member's own
 // blocks run as ordinary units, and the partitions merge by the usual
 // log-sum-exp identity (the definition's sum over all tokens, regrouped).
 //
 // Grouping: sequences are sorted by their first block; within a run of equal
-// first blocks, consecutive members form sub-groups of up to 8 / G. A
+// first blocks, consecutive members form sub-groups of up to 16 / G. A
 // sub-group shares the leading full blocks that every member has in common
 // with its first member (a block is shared only below each member's context;
 // with append_guard, only below the block of the member's last position, so
@@ -249,6 +249,7 @@ __global__ void __maxnreg__(32) pa_plan_kernel(const DecodeParams p) {
 // are cut into partitions 0 .. pp-1 written for every member, the rest of each
 // member into pp, pp+1, ...
 constexpr int SHARE_MAX_SEQS = PLAN_THREADS;  // one sequence per plan thread
+constexpr int SHARE_RANK_MAX = 256;           // batches sorted by rank rather than bitonically
 constexpr int NO_SHARE = 0x7fffffff;
 
 __device__ __forceinline__ int shared_full_blocks(const DecodeParams &p, int ctx) {
@@ -258,6 +259,7 @@ __device__ __forceinline__ int shared_full_blocks(const DecodeParams &p, int ctx
 
 __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const DecodeParams p) {
     __shared__ unsigned long long s_key[SHARE_MAX_SEQS];  // (first block << 32) | sequence, sorted
+    __shared__ unsigned long long s_in[SHARE_RANK_MAX];   // keys before sorting (rank sort)
     __shared__ int s_ctx[SHARE_MAX_SEQS];                 // clamped context of each sequence
     __shared__ int s_grp[SHARE_MAX_SEQS];                 // sub-group of a position: first | count << 16
     __shared__ int s_lcp[SHARE_MAX_SEQS];                 // leading blocks shared with the sub-group's first
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int B = p.num_seqs, P = p.partition, tiles = P / 16, bs = p.block_size, W = p.max_blocks_per_seq;
-    const int cap = 8 / (p.num_heads / p.num_kv_heads);  // sequences per shared unit
+    const int cap = 16 / (p.num_heads / p.num_kv_heads);  // sequences per shared unit (16 query rows)
     int n = 1;
     while (n < B) n <<= 1;
     for (int i = tid; i < PLAN_MAX_BINS; i += PLAN_THREADS) s_bin_count[i] = 0;
@@ -282,10 +284,25 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
         const int b0 = shared_full_blocks(p, ctx) > 0 && first >= 0 && first < p.num_blocks ? first : NO_SHARE;
         key = ((unsigned long long)(unsigned)b0 << 32) | (unsigned)tid;
     }
-    // Bitonic sort, one key per thread: strides below 32 by shuffles within
+    // Up to SHARE_RANK_MAX sequences: rank sort (keys are distinct, so each
+    // key's rank, the number of smaller keys, is its position). Beyond:
+    // bitonic sort, one key per thread: strides below 32 by shuffles within
     // the warp (only the warps that hold keys), larger ones through shared
     // memory (every thread takes the block barriers).
     const bool keyed_warp = warp * 32 < n;
+    if (B <= SHARE_RANK_MAX) {
+        if (tid < B) s_in[tid] = key;
+        __syncthreads();
+        if (tid < B) {
+            int rank = 0;
+#pragma unroll 8
+            for (int j = 0; j < B; ++j) rank += s_in[j] < key;
+            s_key[rank] = key;
+        }
+        __syncthreads();
+        if (tid < B) key = s_key[tid];
+        n = 0;  // skips the bitonic steps
+    }
     for (int k = 2; k <= n; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
             unsigned long long other = key;

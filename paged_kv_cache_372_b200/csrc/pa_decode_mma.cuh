@@ -16,10 +16,11 @@
 // input type for the second product and the softmax denominator sums the
 // same rounded values.
 //
-// Variants (template flags): KV8 reads an E4M3 cache (byte tiles widened to
-// f16 in registers, 16 warps per CTA for head groups up to 4); SHARED lets a
-// unit serve up to 8 / G sequences that share the unit's blocks, their G
-// query rows each filling the MMA's 8 columns (pa_decode_shared).
+// Variants (template flags): KV8 reads an 8-bit cache (byte tiles widened to
+// f16 in registers, 16 warps per CTA for head groups up to 4), I8 with INT8
+// codes, HS with one scale per KV head; SHARED lets a unit serve up to 16 / G
+// sequences that share the unit's blocks, their G query rows each filling
+// columns of two 8-column MMA tiles (pa_decode_shared, 8 warps per CTA).
 #pragma once
 
 #include <cuda.h>
@@ -45,13 +46,17 @@ struct MmaGeo {
     static constexpr int STAGE_BYTES = 2 * HALF_BYTES;    // K then V of one tile
 };
 
+// Query rows of a unit shared by several sequences: two n8 column halves of
+// the MMA tile, the G rows of each of up to 16 / G member sequences.
+constexpr int SHARE_ROWS = 16;
+
 // Query slots of a warp: the G rows of one sequence, double-buffered (the
 // next unit's rows arrive while the current unit runs), or for units shared
-// by several sequences one slot of 8 rows (the MMA's N) that the next unit's
-// rows may fill once the current unit has read its own.
+// by several sequences one slot of SHARE_ROWS rows that the next unit's rows
+// may fill once the current unit has read its own.
 template <int D, int G, bool SHARED>
 __host__ __device__ constexpr int mma_q_slot_bytes() {
-    return (SHARED ? 8 : G) * D * 2;
+    return (SHARED ? SHARE_ROWS : G) * D * 2;
 }
 template <bool SHARED>
 __host__ __device__ constexpr int mma_q_slots() {
@@ -75,9 +80,12 @@ __host__ __device__ constexpr int mma_smem_bytes(int warps) {
 #ifndef PA_FP8_WIDE_MAX_GROUP
 #define PA_FP8_WIDE_MAX_GROUP 4
 #endif
-template <int G, bool KV8>
+// Shared-prefix units keep a second half of query columns (accumulators and
+// query fragments): 8 warps per CTA, so each thread has up to 255 registers.
+constexpr int SHARE_MAX_WARPS = 8;
+template <int G, bool KV8, bool SHARED = false>
 __host__ __device__ constexpr int mma_max_warps() {
-    return KV8 && G <= PA_FP8_WIDE_MAX_GROUP ? DECODE_MAX_WARPS_FP8 : DECODE_MAX_WARPS;
+    return SHARED ? SHARE_MAX_WARPS : KV8 && G <= PA_FP8_WIDE_MAX_GROUP ? DECODE_MAX_WARPS_FP8 : DECODE_MAX_WARPS;
 }
 
 // E4M3 -> f16 widening: every E4M3 value is exactly an f16. One cvt converts
@@ -325,17 +333,44 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
 // out = sum_j 2^(m_j - M) acc_j / sum_j 2^(m_j - M) l_j.
 constexpr int REDUCE_GROUPS = 4;
 
+// The merge launch of shared-prefix decode: a member has few partitions (its
+// shared ones and its own), so one warp merges one (grouping position, KV
+// head) with mma_merge, 8 per CTA; the sequence and its partition count come
+// from the grouping plan's members / member_nparts.
 template <int D, int G, typename T>
+__global__ void __launch_bounds__(256) pa_reduce_members_kernel(const DecodeParams p) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (item >= p.num_seqs * p.num_kv_heads) return;
+    const int pos = item / p.num_kv_heads, kvh = item - pos * p.num_kv_heads;
+    const int s = p.members[pos], nparts = p.member_nparts[pos];
+    if (nparts <= 1) return;  // written by the attention kernel
+    mma_merge<D, G, T>(p, (size_t)s * p.num_kv_heads + kvh, (size_t)s * p.num_heads + (size_t)kvh * G, 0, nparts,
+                       lane);
+}
+
+// SM (shared-prefix decode): CTA = (grouping position, KV head); the
+// sequence and its partition count come from the grouping plan's members /
+// member_nparts.
+template <int D, int G, typename T, bool SM = false>
 __global__ void pa_reduce_kernel(const DecodeParams p) {
     constexpr int V4 = D * G / 4;
     extern __shared__ float4 s_red[];  // [REDUCE_GROUPS][V4] sums, [REDUCE_GROUPS][V4] weight sums, (max, sum)s
     float2 *s_ml = reinterpret_cast<float2 *>(s_red + 2 * REDUCE_GROUPS * V4);  // [nparts][G]
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int group = blockIdx.x, s = group / p.num_kv_heads, kvh = group - s * p.num_kv_heads;
-    const int ctx = clamped_context(p, s, false);
-    const int nparts = (ctx + p.partition - 1) / p.partition;
+    const int pos = blockIdx.x / p.num_kv_heads, kvh = blockIdx.x - pos * p.num_kv_heads;
+    int s, nparts;
+    if constexpr (SM) {
+        s = p.members[pos];
+        nparts = p.member_nparts[pos];
+    } else {
+        s = pos;
+        nparts = (clamped_context(p, s, false) + p.partition - 1) / p.partition;
+    }
     if (nparts <= 1) return;  // written by the attention kernel
-    const float2 *ml = p.ml + (size_t)group * p.max_parts * G;
+    const size_t group = (size_t)s * p.num_kv_heads + kvh;
+    const float2 *ml = p.ml + group * p.max_parts * G;
     for (int i = threadIdx.x; i < nparts * G; i += blockDim.x) s_ml[i] = __ldcg(ml + i);
     __syncthreads();
     const int v = threadIdx.x % V4, r = threadIdx.x / V4;
@@ -346,7 +381,7 @@ __global__ void pa_reduce_kernel(const DecodeParams p) {
         M[c] = -INFINITY;
         for (int j = 0; j < nparts; ++j) M[c] = fmaxf(M[c], s_ml[j * G + g].x);
     }
-    const float4 *part = reinterpret_cast<const float4 *>(p.part_acc + (size_t)group * p.max_parts * (D * G));
+    const float4 *part = reinterpret_cast<const float4 *>(p.part_acc + group * p.max_parts * (D * G));
 #pragma unroll 4
     for (int j = r; j < nparts; j += REDUCE_GROUPS) {
         const float4 a = __ldcg(part + (size_t)j * V4 + v);
@@ -379,7 +414,7 @@ __global__ void pa_reduce_kernel(const DecodeParams p) {
 }
 
 template <int D, int G, typename T, int NS, bool KV8 = false, bool SHARED = false, bool I8 = false, bool HS = false>
-__global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
+__global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
     pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
     static_assert(!I8 || KV8, "INT8 codes are an 8-bit cache");
@@ -434,10 +469,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
         const int bi = tok / bs;
         const int pb = __shfl_sync(FULL_MASK, tbl, bi);
         // Member sequences of a shared unit reach the issuing lane by shuffle.
-        int mid[SHARED ? 8 : 1];
+        int mid[SHARED ? SHARE_ROWS : 1];
         if constexpr (SHARED) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) mid[j] = __shfl_sync(FULL_MASK, mseq, j);
+            for (int j = 0; j < SHARE_ROWS; ++j) mid[j] = __shfl_sync(FULL_MASK, mseq, j);
         }
         if (lane == 0) {
             const uint32_t bar = bar_s + 8 * stage;
@@ -461,7 +496,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                     if constexpr (SHARED) {
                         if (mcnt > 0) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
+                            for (int j = 0; j < SHARE_ROWS; ++j)
                                 if (j < mcnt)
                                     bulk_load(qbuf_s + qslot * QB + j * QG,
                                               qg + ((size_t)mid[j] * H + kvh * G) * D, QG, bar, policy);
@@ -571,6 +606,19 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
         for (int i = 0; i < Gm::KS; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+        // Shared units with more than 8 query rows: the second column half
+        // (rows 8 + h0, 8 + h1), with its own fragments, maxima, sums and
+        // accumulators.
+        constexpr int K2 = SHARED ? Gm::KS : 1;
+        const bool two = SHARED && nrows > 8;
+        const bool hw0 = 8 + h0 < nrows, hw1 = 8 + h1 < nrows;
+        uint32_t qc[K2][2];
+        float o2[K2][4];
+        float N0 = -INFINITY, N1 = -INFINITY, m0s = 0.f, m1s = 0.f;  // maxima and sums of the second half
+#pragma unroll
+        for (int i = 0; i < K2; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o2[i][j] = 0.f;
         // Lanes [0, NVR) hold one 16-byte vector of the new K row, lanes
         // [NVR, 2*NVR) of the new V row; loaded now, used at the last tile.
         const bool app_unit = append && cur.part == cur.nparts - 1;
@@ -615,6 +663,11 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                         const int d = 16 * i + 2 * t4;
                         qb[i][0] = g8 < nrows ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
                         qb[i][1] = g8 < nrows ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 8) * 2) : 0u;
+                        if constexpr (SHARED) {
+                            const int r = 8 + g8;
+                            qc[i][0] = r < nrows ? *reinterpret_cast<const uint32_t *>(qs + (r * D + d) * 2) : 0u;
+                            qc[i][1] = r < nrows ? *reinterpret_cast<const uint32_t *>(qs + (r * D + d + 8) * 2) : 0u;
+                        }
                     }
                 }
                 if constexpr (KV8 && !std::is_same<T, __half>::value) {
@@ -659,6 +712,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             // ---------------- S^T = K . Q^T ------------------------------------
             // Two accumulators (even / odd slices) halve the chain of dependent MMAs.
             float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+            float u[4] = {0.f, 0.f, 0.f, 0.f}, u2[4] = {0.f, 0.f, 0.f, 0.f};  // second half
             if constexpr (KV8) {
                 // A 16-byte chunk holds 16 codes of a row; ldmatrix on byte pairs
                 // gives each thread codes 4*t4 .. 4*t4+3 of rows g8 and g8+8.
@@ -690,6 +744,9 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                     uint32_t a[4];
                     ldsm_x4(a, ks_s + swz(row, 2 * i + csel));
                     MmaType<T>::mma((i & 1) ? s2 : s, a, qb[i][0], qb[i][1]);
+                    if constexpr (SHARED) {
+                        if (two) MmaType<T>::mma((i & 1) ? u2 : u, a, qc[i][0], qc[i][1]);
+                    }
                 }
             }
 #pragma unroll
@@ -732,6 +789,46 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             }
             // P^T B fragments: head g8, tokens 2*t4 (+1) and 8 + 2*t4 (+1).
             const uint32_t pb0 = movmatrix_trans(w_lo), pb1 = movmatrix_trans(w_hi);
+            // The same for the second column half of a wide shared unit.
+            uint32_t pc0 = 0u, pc1 = 0u;
+            if constexpr (SHARED) {
+                if (two) {
+                    const float y0 = v_lo ? (u[0] + u2[0]) * uq : -INFINITY;
+                    const float y1 = v_lo ? (u[1] + u2[1]) * uq : -INFINITY;
+                    const float y2 = v_hi ? (u[2] + u2[2]) * uq : -INFINITY;
+                    const float y3 = v_hi ? (u[3] + u2[3]) * uq : -INFINITY;
+                    const bool raise2 = (hw0 && !(fmaxf(y0, y2) <= N0 + LAZY_MAX_LOG2)) ||
+                                        (hw1 && !(fmaxf(y1, y3) <= N1 + LAZY_MAX_LOG2));
+                    if (__any_sync(FULL_MASK, raise2)) {
+                        float n0 = fmaxf(y0, y2), n1 = fmaxf(y1, y3);
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) {
+                            n0 = fmaxf(n0, __shfl_xor_sync(FULL_MASK, n0, off));
+                            n1 = fmaxf(n1, __shfl_xor_sync(FULL_MASK, n1, off));
+                        }
+                        n0 = fmaxf(N0, n0);
+                        n1 = fmaxf(N1, n1);
+                        const float a0 = exp2f(N0 - n0), a1 = exp2f(N1 - n1);
+                        N0 = n0;
+                        N1 = n1;
+                        m0s *= a0;
+                        m1s *= a1;
+#pragma unroll
+                        for (int i = 0; i < K2; ++i) {
+                            o2[i][0] *= a0; o2[i][1] *= a1;
+                            o2[i][2] *= a0; o2[i][3] *= a1;
+                        }
+                    }
+                    const float q0 = hw0 ? exp2f(y0 - N0) : 0.f, q1 = hw1 ? exp2f(y1 - N1) : 0.f;
+                    const float q2 = hw0 ? exp2f(y2 - N0) : 0.f, q3 = hw1 ? exp2f(y3 - N1) : 0.f;
+                    const uint32_t z_lo = Elem<MT>::pack(q0, q1), z_hi = Elem<MT>::pack(q2, q3);
+                    const float2 r_lo = Elem<MT>::pair(z_lo), r_hi = Elem<MT>::pair(z_hi);
+                    m0s += r_lo.x + r_hi.x;
+                    m1s += r_lo.y + r_hi.y;
+                    pc0 = movmatrix_trans(z_lo);
+                    pc1 = movmatrix_trans(z_hi);
+                }
+            }
 
             // ---------------- O^T += V^T . P^T ----------------------------------
             if (valid < 16) {
@@ -783,6 +880,9 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
                     uint32_t a[4];
                     ldsm_x4_trans(a, vs_s + swz(row, 2 * i + csel));
                     MmaType<T>::mma(o[i], a, pb0, pb1);
+                    if constexpr (SHARED) {
+                        if (two) MmaType<T>::mma(o2[i], a, pc0, pc1);
+                    }
                 }
             }
             ++consumed;
@@ -798,6 +898,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
         for (int off = 4; off < 32; off <<= 1) {
             l0 += __shfl_xor_sync(FULL_MASK, l0, off);
             l1 += __shfl_xor_sync(FULL_MASK, l1, off);
+            if constexpr (SHARED) {
+                m0s += __shfl_xor_sync(FULL_MASK, m0s, off);
+                m1s += __shfl_xor_sync(FULL_MASK, m1s, off);
+            }
         }
         if constexpr (I8) {
             // The values were multiplied as 1152 + code: take 1152 * (sum of the weights) off.
@@ -811,36 +915,44 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
         }
         const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;
         if (SHARED && cur.mcnt > 0) {
-            // Partials of every member: column h of the accumulators is query
-            // row h, i.e. head h % G of member h / G.
-            const int seq0 = __shfl_sync(FULL_MASK, cur.mseq, (h0 / G) & 7);
-            const int seq1 = __shfl_sync(FULL_MASK, cur.mseq, (h1 / G) & 7);
-            const size_t row0 = ((size_t)seq0 * Hkv + cur.kvh) * p.max_parts + cur.part;
-            const size_t row1 = ((size_t)seq1 * Hkv + cur.kvh) * p.max_parts + cur.part;
-            float *acc0 = p.part_acc + row0 * (size_t)(D * G);
-            float *acc1 = p.part_acc + row1 * (size_t)(D * G);
-            const int g0 = h0 % G, g1 = h1 % G;
+            // Partials of every member: query row r (column r of the first
+            // half, or r - 8 of the second) is head r % G of member r / G.
             const float vs = KV8 ? uv : 1.f;
+            auto store_half = [&](const float (&oo)[Gm::KS][4], int r0, int r1, bool va, bool vb, float Ma, float Mb,
+                                  float la, float lb) {
+                const int seq0 = __shfl_sync(FULL_MASK, cur.mseq, (r0 / G) & (SHARE_ROWS - 1));
+                const int seq1 = __shfl_sync(FULL_MASK, cur.mseq, (r1 / G) & (SHARE_ROWS - 1));
+                const size_t row0 = ((size_t)seq0 * Hkv + cur.kvh) * p.max_parts + cur.part;
+                const size_t row1 = ((size_t)seq1 * Hkv + cur.kvh) * p.max_parts + cur.part;
+                float *acc0 = p.part_acc + row0 * (size_t)(D * G);
+                float *acc1 = p.part_acc + row1 * (size_t)(D * G);
+                const int g0 = r0 % G, g1 = r1 % G;
 #pragma unroll
-            for (int i = 0; i < Gm::KS; ++i) {
-                const int d = KV8 ? 16 * i + 2 * g8 : 16 * i + g8;
-                const int d2 = KV8 ? d + 1 : d + 8;
-                if constexpr (G == 1) {
-                    if (hv0) {
-                        acc0[d] = o[i][0] * vs;
-                        acc0[d2] = o[i][2] * vs;
+                for (int i = 0; i < Gm::KS; ++i) {
+                    const int d = KV8 ? 16 * i + 2 * g8 : 16 * i + g8;
+                    const int d2 = KV8 ? d + 1 : d + 8;
+                    if constexpr (G == 1) {
+                        if (va) {
+                            acc0[d] = oo[i][0] * vs;
+                            acc0[d2] = oo[i][2] * vs;
+                        }
+                        if (vb) {
+                            acc1[d] = oo[i][1] * vs;
+                            acc1[d2] = oo[i][3] * vs;
+                        }
+                    } else if (vb) {  // G even: rows r0, r0 + 1 are heads g0, g0 + 1 of one member
+                        *reinterpret_cast<float2 *>(acc0 + d * G + g0) = make_float2(oo[i][0] * vs, oo[i][1] * vs);
+                        *reinterpret_cast<float2 *>(acc0 + d2 * G + g0) = make_float2(oo[i][2] * vs, oo[i][3] * vs);
                     }
-                    if (hv1) {
-                        acc1[d] = o[i][1] * vs;
-                        acc1[d2] = o[i][3] * vs;
-                    }
-                } else if (hv1) {  // G even: columns h0, h1 are heads g0, g0 + 1 of one member
-                    *reinterpret_cast<float2 *>(acc0 + d * G + g0) = make_float2(o[i][0] * vs, o[i][1] * vs);
-                    *reinterpret_cast<float2 *>(acc0 + d2 * G + g0) = make_float2(o[i][2] * vs, o[i][3] * vs);
                 }
+                if (g8 == 0 && va) p.ml[row0 * G + g0] = make_float2(Ma, la);
+                if (g8 == 0 && vb) p.ml[row1 * G + g1] = make_float2(Mb, lb);
+            };
+            store_half(o, h0, h1, hv0, hv1, M0, M1, l0, l1);
+            if constexpr (SHARED) {
+                if (two) store_half(o2, 8 + h0, 8 + h1, hw0, hw1, N0, N1, m0s, m1s);
             }
-            if (g8 == 0 && hv0) p.ml[row0 * G + g0] = make_float2(M0, l0);
-            if (g8 == 0 && hv1) p.ml[row1 * G + g1] = make_float2(M1, l1);
+            if (p.reduce_launch) goto next_unit;  // merged by pa_reduce_kernel
             // Lane j counts member j's partition.
             src.wait_plan();  // the merge counters are zeroed by the plan kernel
             const bool last = count_partition(&p.merge_count[(size_t)cur.mseq * Hkv + cur.kvh], cur.mnp,
@@ -904,13 +1016,15 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8>() * 32, 1)
             }
             if (g8 == 0 && hv0) p.ml[row * G + h0] = make_float2(M0, l0);
             if (g8 == 0 && hv1) p.ml[row * G + h1] = make_float2(M1, l1);
-            if (!SHARED && p.reduce_launch) goto next_unit;  // merged by pa_reduce_kernel
+            if (p.reduce_launch) goto next_unit;  // merged by pa_reduce_kernel
             src.wait_plan();  // the merge counters are zeroed by the plan kernel
             // One level (at most MERGE_FANIN partitions, or shared-prefix units'
             // workspace), or two: this partition's chunk into its chunk
             // partial, then the chunk partials. One merge call site in a loop
-            // keeps the merge inlined once.
-            const bool chunked = cur.nparts > MERGE_FANIN && p.max_chunks > 0;
+            // keeps the merge inlined once. The 8-bit kernels, under a
+            // 128-register cap, keep one level (beyond REDUCE_LAUNCH_MIN_PARTS
+            // partitions their merges run in the separate launch anyway).
+            const bool chunked = !KV8 && cur.nparts > MERGE_FANIN && p.max_chunks > 0;
             const int nch = (cur.nparts + MERGE_FANIN - 1) / MERGE_FANIN;
             int first = 0, n = cur.nparts, dst = -1;
             bool go;

@@ -214,7 +214,7 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     const CUtensorMapDataType type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : pa::MmaType<T>::tma_type;
     if ((st = encode_pool_map(&tmk, p.k_pool, rows, D, KV8 ? 1 : 2, type, info.dev)) != PA_OK) return st;
     if ((st = encode_pool_map(&tmv, p.v_pool, rows, D, KV8 ? 1 : 2, type, info.dev)) != PA_OK) return st;
-    constexpr int max_warps = pa::mma_max_warps<G, KV8>();
+    constexpr int max_warps = pa::mma_max_warps<G, KV8, SHARED>();
     int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS, KV8, SHARED>();
     if (warps > max_warps) warps = max_warps;
     if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "not enough shared memory for one warp");
@@ -224,6 +224,9 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
     if constexpr (SHARED) {
+        // Shared units end with several members' merges; they run in the
+        // merge launch, one CTA per (member, KV head), all at once.
+        p.reduce_launch = p.max_parts > 1 && reduce_smem_bytes<D, G>(p.max_parts) <= REDUCE_SMEM_MAX;
         pa::pa_plan_shared_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
     } else {
         p.early = p.num_seqs <= EARLY_MAX_SEQS;
@@ -244,7 +247,7 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, p, tmk, tmv);
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
-    if constexpr (!SHARED) {
+    {
         if (p.reduce_launch) {
             constexpr int V4 = D * G / 4;
             cudaLaunchConfig_t rc = {};
@@ -254,8 +257,15 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
             rc.stream = stream;
             rc.attrs = attr;
             rc.numAttrs = 1;
-            e = set_dynamic_smem<pa::pa_reduce_kernel<D, G, T>>(info.dev, REDUCE_SMEM_MAX);
-            if (e == cudaSuccess) e = cudaLaunchKernelEx(&rc, pa::pa_reduce_kernel<D, G, T>, p);
+            if constexpr (SHARED) {
+                rc.gridDim = dim3((unsigned)((p.num_seqs * p.num_kv_heads + 7) / 8));
+                rc.blockDim = dim3(256);
+                rc.dynamicSmemBytes = 0;
+                e = cudaLaunchKernelEx(&rc, pa::pa_reduce_members_kernel<D, G, T>, p);
+            } else {
+                e = set_dynamic_smem<pa::pa_reduce_kernel<D, G, T>>(info.dev, REDUCE_SMEM_MAX);
+                if (e == cudaSuccess) e = cudaLaunchKernelEx(&rc, pa::pa_reduce_kernel<D, G, T>, p);
+            }
             if (e != cudaSuccess) return cuda_fail(e, "pa_reduce_kernel launch");
         }
     }
@@ -286,11 +296,7 @@ pa_status dispatch_group_shared(pa::DecodeParams &p, int group, cudaStream_t str
         case 1: return launch_decode_mma<D, 1, T, false, true>(p, stream);
         case 2: return launch_decode_mma<D, 2, T, false, true>(p, stream);
         case 4: return launch_decode_mma<D, 4, T, false, true>(p, stream);
-        case 8: {
-            // Eight query heads fill a unit's 8 query rows: nothing to share.
-            p.entries_b = nullptr;
-            return launch_decode_mma<D, 8, T>(p, stream);
-        }
+        case 8: return launch_decode_mma<D, 8, T, false, true>(p, stream);
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }

@@ -108,7 +108,7 @@ def expected_entries(case, P, append):
     """Work-list entries (per KV head) of the grouping the header describes,
     counted directly from the tables."""
     bs, seqs = case["bs"], case["seqs"]
-    cap = 8 // (case["heads"] // case["kv_heads"])
+    cap = 16 // (case["heads"] // case["kv_heads"])
 
     def nfull(c):
         p = c - 1 if append else c
@@ -219,7 +219,7 @@ def test_sharing_patterns_match_oracle(shape, append):
         Pr = pa.pa_decode_shared_partition_size(len(case["ctx"]), heads, kv_heads, D, bs, int(case["ctx"].max()), P)
         n_expect, n_shared = expected_entries(case, Pr, append)
         assert int(ws[4:8].view(torch.int32).item()) == n_expect
-        assert n_shared >= 10 or heads // kv_heads == 8  # 8 query heads fill a unit alone
+        assert n_shared >= 10  # sequences that share blocks do share units (G = 8 included: 2 per unit)
         # Same inputs through the plain path.
         plain, pkp, pvp = run_plain(case, P, append)
         assert float((plain.float() - out.float()).abs().max()) <= H.TOL[dtype]
@@ -255,10 +255,10 @@ def test_beam_workloads(name, fused):
 
 def test_without_sharing_equals_plain_decode():
     """No shared blocks: every unit is an ordinary one and the partitions are
-    pa_decode's. Where no sequence has more than 8 partitions both merge them
-    in one level, in the same order, so the result is bit-identical; longer
-    sequences merge in two levels in pa_decode (chunks of 8) and in one here,
-    which agree up to fp32 rounding."""
+    pa_decode's, so the unnormalised partials are the same; the merges differ
+    only in the order of their fp32 sums (pa_decode: in the attention kernel,
+    in one level up to 8 partitions and two beyond; here: in the separate
+    merge launch), so the results agree up to that rounding."""
     wl = workloads.llama3_8b(1, num_seqs=24)
     st = wl.steps[0]
     dev = torch.device("cuda")
@@ -272,10 +272,7 @@ def test_without_sharing_equals_plain_decode():
         pa.pa_decode(a, q, kp, vp, tab, ctx, wl.scale, mx, 128)
         pa.pa_decode_shared(b, q, kp, vp, tab, ctx, wl.scale, mx, 128)
         torch.cuda.synchronize()
-        if mx <= 8 * 128:
-            assert torch.equal(a, b)
-        else:
-            assert float((a.float() - b.float()).abs().max()) <= H.TOL[wl.dtype]
+        assert float((a.float() - b.float()).abs().max()) <= H.TOL[wl.dtype]
 
 
 def test_too_many_sequences_rejected():
