@@ -199,8 +199,8 @@ PA_API pa_status pa_decode_shared(void *out, const void *q, const void *k_new, c
                                   float scale, int dtype, int partition_size, void *workspace,
                                   size_t workspace_bytes, pa_stream_t stream);
 
-/* Partition and workspace bytes pa_decode_fp8 uses for these arguments
- * (0 if invalid, e.g. head_dim other than 128). */
+/* Partition and workspace bytes pa_decode_fp8 (and pa_decode_quant) uses for
+ * these arguments (0 if invalid). */
 PA_API int pa_decode_fp8_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                         int block_size, int max_context_len, int partition_size);
 PA_API size_t pa_decode_fp8_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
@@ -220,7 +220,8 @@ PA_API size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int n
  * per-tensor scales: key element = k_scale * E4M3 code, value element =
  * v_scale * E4M3 code; otherwise exactly pa_decode (q and out stay fp16/bf16
  * by `dtype`). k_pool, v_pool: uint8 codes [num_blocks][num_kv_heads]
- * [block_size][head_dim], written by pa_reshape_and_cache_fp8. head_dim 128.
+ * [block_size][head_dim], written by pa_reshape_and_cache_fp8. head_dim 64 or
+ * 128.
  * The products run on tensor cores with the codes widened to fp16 (exact) and
  * the queries converted to fp16 (exact for |q| in fp16's normal range; a bf16
  * query element above 65504 in magnitude has no fp16 value: the kernel sets
@@ -283,7 +284,7 @@ PA_API pa_status pa_reshape_and_cache_quant(const void *k, const void *v, void *
  * element of KV head j = k_scales[j] * decode(code), value element =
  * v_scales[j] * decode(code), decode being E4M3 (PA_KV_E4M3) or code - 128
  * (PA_KV_INT8); otherwise exactly pa_decode (q and out fp16/bf16 by dtype).
- * head_dim 128. The partition and the workspace are those of pa_decode_fp8
+ * head_dim 64 or 128. The partition and the workspace are those of pa_decode_fp8
  * (pa_decode_fp8_partition_size, pa_decode_fp8_workspace_size). INT8 codes
  * enter the tensor-core products as the exact fp16 numbers 1152 + (code - 128);
  * the constant is taken off the scores (per query row) and the outputs (times

@@ -133,7 +133,7 @@ int pa_decode_shared_partition_size(int num_seqs, int num_heads, int num_kv_head
 
 int pa_decode_fp8_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                                  int max_context_len, int partition_size) {
-    if (num_seqs < 0 || max_context_len < 0 || partition_size < 0 || head_dim != 128) return 0;
+    if (num_seqs < 0 || max_context_len < 0 || partition_size < 0) return 0;
     if (!shape_supported(num_heads, num_kv_heads, head_dim, block_size)) return 0;
     return resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size, PartMode::fp8);
 }
@@ -173,7 +173,6 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     if (shared && num_seqs > pa::SHARE_MAX_SEQS)
         return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode takes at most %d sequences, got %d", pa::SHARE_MAX_SEQS,
                     num_seqs);
-    if (kv8 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "fp8 cache supports head_dim 128, got %d", head_dim);
     if (kv8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || k_scale == INFINITY || v_scale == INFINITY))
         return fail(PA_ERR_INVALID, "k_scale and v_scale must be positive and finite");
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 || partition_size < 0)
@@ -250,14 +249,23 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int group = num_heads / num_kv_heads;
-    if (kv8 && int8)
-        return dtype == PA_F16 ? dispatch_group_fp8<__half, true, true>(p, group, s)
-                               : dispatch_group_fp8<__nv_bfloat16, true, true>(p, group, s);
-    if (kv8 && k_scales)
-        return dtype == PA_F16 ? dispatch_group_fp8<__half, false, true>(p, group, s)
-                               : dispatch_group_fp8<__nv_bfloat16, false, true>(p, group, s);
-    if (kv8)
-        return dtype == PA_F16 ? dispatch_group_fp8<__half>(p, group, s) : dispatch_group_fp8<__nv_bfloat16>(p, group, s);
+    if (kv8) {
+        const bool d128 = head_dim == 128, f16 = dtype == PA_F16;
+        if (int8)
+            return d128 ? (f16 ? dispatch_group_fp8<128, __half, true, true>(p, group, s)
+                               : dispatch_group_fp8<128, __nv_bfloat16, true, true>(p, group, s))
+                        : (f16 ? dispatch_group_fp8<64, __half, true, true>(p, group, s)
+                               : dispatch_group_fp8<64, __nv_bfloat16, true, true>(p, group, s));
+        if (k_scales)
+            return d128 ? (f16 ? dispatch_group_fp8<128, __half, false, true>(p, group, s)
+                               : dispatch_group_fp8<128, __nv_bfloat16, false, true>(p, group, s))
+                        : (f16 ? dispatch_group_fp8<64, __half, false, true>(p, group, s)
+                               : dispatch_group_fp8<64, __nv_bfloat16, false, true>(p, group, s));
+        return d128 ? (f16 ? dispatch_group_fp8<128, __half>(p, group, s)
+                           : dispatch_group_fp8<128, __nv_bfloat16>(p, group, s))
+                    : (f16 ? dispatch_group_fp8<64, __half>(p, group, s)
+                           : dispatch_group_fp8<64, __nv_bfloat16>(p, group, s));
+    }
     if (shared) {
         if (head_dim == 128)
             return dtype == PA_F16 ? dispatch_group_shared<128, __half>(p, group, s)

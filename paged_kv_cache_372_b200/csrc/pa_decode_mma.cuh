@@ -35,15 +35,26 @@ namespace pa {
 // KV8: the pools hold E4M3 (fp8) codes, one byte per element, dequantised
 // with per-tensor scales (k_scale folded into the score scale, v_scale into
 // the output scale).
+//
+// A tile row is D * EB bytes: 256 or 128 (loaded in 128-byte boxes with the
+// 128-byte swizzle) or 64 (an 8-bit cache at head_dim 64: one 64-byte box
+// with the 64-byte swizzle).
 template <int D, int G, bool KV8 = false>
 struct MmaGeo {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "head group size");
-    static_assert(!KV8 || D == 128, "fp8 cache: head_dim 128");
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static constexpr int EB = KV8 ? 1 : 2;                // bytes per pool element
     static constexpr int KS = D / 16;                     // 16-wide slices of a row
-    static constexpr int NBOX = D * EB / 128;             // 128-byte TMA boxes per row
+    static constexpr int ROW_BYTES = D * EB;
+    static constexpr int BOX_ROW = ROW_BYTES < 128 ? ROW_BYTES : 128;  // bytes of a box row
+    static constexpr int BOX_ELEMS = BOX_ROW / EB;        // elements of a box row (TMA box width)
+    static constexpr int NBOX = ROW_BYTES / BOX_ROW;      // TMA boxes per row
+    static constexpr int BOX_BYTES = 16 * BOX_ROW;        // one box of a 16-row tile
+    static constexpr int CHUNKS = ROW_BYTES / 16;         // 16-byte chunks of a row
     static constexpr int HALF_BYTES = 16 * D * EB;        // one K (or V) tile
     static constexpr int STAGE_BYTES = 2 * HALF_BYTES;    // K then V of one tile
+    // Byte offset of 16-byte chunk `chunk` of row `row` of a tile.
+    static __device__ __forceinline__ uint32_t addr(int row, int chunk);
 };
 
 // Query rows of a unit shared by several sequences: two n8 column halves of
@@ -184,10 +195,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` inside a tile loaded as
-// NBOX boxes of [16 rows][64 columns] with the 128-byte swizzle: within each
+// NBOX boxes of [16 rows][128 bytes] with the 128-byte swizzle: within each
 // 1024-byte group of 8 rows the chunk index is XORed with the row index.
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)((chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+// The same for one box of [16 rows][64 bytes] with the 64-byte swizzle: the
+// chunk index (0..3) is XORed with bits 1..2 of the row index, so the 8 rows
+// an ldmatrix phase reads fall in distinct banks.
+__device__ __forceinline__ uint32_t swz64(int row, int chunk) {
+    return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+
+template <int D, int G, bool KV8>
+__device__ __forceinline__ uint32_t MmaGeo<D, G, KV8>::addr(int row, int chunk) {
+    if constexpr (BOX_ROW == 64)
+        return swz64(row, chunk);
+    else
+        return swz(row, chunk);
 }
 
 // Merge of partial slots [first, first + nparts) of one (sequence, KV head)
@@ -488,8 +514,9 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                     const uint32_t dst = ring_s + stage * Gm::STAGE_BYTES;
 #pragma unroll
                     for (int b = 0; b < Gm::NBOX; ++b) {
-                        tma_load_2d(dst + b * 2048, &tm_k, 64 * b, row, bar, policy);
-                        tma_load_2d(dst + Gm::HALF_BYTES + b * 2048, &tm_v, 64 * b, row, bar, policy);
+                        tma_load_2d(dst + b * Gm::BOX_BYTES, &tm_k, Gm::BOX_ELEMS * b, row, bar, policy);
+                        tma_load_2d(dst + Gm::HALF_BYTES + b * Gm::BOX_BYTES, &tm_v, Gm::BOX_ELEMS * b, row, bar,
+                                    policy);
                     }
                 }
                 if (it == 0) {
@@ -696,7 +723,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                 if (lane < 2 * NVR) {
                     const int half = lane / NVR, c = lane % NVR;
                     uint8_t *st = ring + stage * Gm::STAGE_BYTES + half * Gm::HALF_BYTES;
-                    *reinterpret_cast<uint4 *>(st + swz(tok & 15, c)) = newrow;
+                    *reinterpret_cast<uint4 *>(st + Gm::addr(tok & 15, c)) = newrow;
                     if ((unsigned)pb < (unsigned)p.num_blocks) {
                         T *pool = static_cast<T *>(const_cast<void *>(half ? p.v_pool : p.k_pool));
                         *reinterpret_cast<uint4 *>(pool + (((size_t)pb * Hkv + cur.kvh) * bs + tok % bs) * D + c * 8) =
@@ -721,7 +748,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
 #pragma unroll
                 for (int i = 0; i < Gm::KS; i += 2) {
                     uint32_t r[4];
-                    ldsm_x4(r, ks_s + swz(row, i + csel));
+                    ldsm_x4(r, ks_s + Gm::addr(row, i + csel));
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
@@ -742,7 +769,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
 #pragma unroll
                 for (int i = 0; i < Gm::KS; ++i) {
                     uint32_t a[4];
-                    ldsm_x4(a, ks_s + swz(row, 2 * i + csel));
+                    ldsm_x4(a, ks_s + Gm::addr(row, 2 * i + csel));
                     MmaType<T>::mma((i & 1) ? s2 : s, a, qb[i][0], qb[i][1]);
                     if constexpr (SHARED) {
                         if (two) MmaType<T>::mma((i & 1) ? u2 : u, a, qc[i][0], qc[i][1]);
@@ -835,10 +862,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                 // Stale or never-written slots past the context must not reach
                 // the product (their weight is 0 but 0 * NaN is NaN): zero them.
                 uint8_t *vt = ring + stage * Gm::STAGE_BYTES + Gm::HALF_BYTES;
-                for (int idx = lane; idx < (16 - valid) * Gm::NBOX * 8; idx += 32) {
-                    const int r = valid + idx / (Gm::NBOX * 8);
-                    const int c = idx % (Gm::NBOX * 8);
-                    *reinterpret_cast<uint4 *>(vt + swz(r, c)) = make_uint4(0, 0, 0, 0);
+                for (int idx = lane; idx < (16 - valid) * Gm::CHUNKS; idx += 32) {
+                    const int r = valid + idx / Gm::CHUNKS;
+                    const int c = idx % Gm::CHUNKS;
+                    *reinterpret_cast<uint4 *>(vt + Gm::addr(r, c)) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
                 __syncwarp();
@@ -853,7 +880,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
 #pragma unroll
                 for (int i = 0; i < Gm::KS; i += 2) {
                     uint32_t r[4];
-                    ldsm_x4_trans(r, vs_s + swz(row, i + csel));
+                    ldsm_x4_trans(r, vs_s + Gm::addr(row, i + csel));
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         uint32_t a[4];
@@ -878,7 +905,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
 #pragma unroll
                 for (int i = 0; i < Gm::KS; ++i) {
                     uint32_t a[4];
-                    ldsm_x4_trans(a, vs_s + swz(row, 2 * i + csel));
+                    ldsm_x4_trans(a, vs_s + Gm::addr(row, 2 * i + csel));
                     MmaType<T>::mma(o[i], a, pb0, pb1);
                     if constexpr (SHARED) {
                         if (two) MmaType<T>::mma(o2[i], a, pc0, pc1);

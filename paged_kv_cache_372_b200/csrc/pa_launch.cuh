@@ -162,10 +162,14 @@ pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, in
     if (st != PA_OK) return st;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)D * elem_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), 16};
+    // Box rows of 128 bytes with the 128-byte swizzle, or (an 8-bit cache at
+    // head_dim 64) one 64-byte box with the 64-byte swizzle.
+    const int box_row = D * elem_bytes < 128 ? D * elem_bytes : 128;
+    const cuuint32_t box[2] = {(cuuint32_t)(box_row / elem_bytes), 16};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, type, 2, const_cast<void *>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     box_row == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     std::lock_guard<std::mutex> lock(mu);
     Entry &c = cache[next];
@@ -275,14 +279,14 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
 }
 
 // 8-bit cache (E4M3, or INT8 with I8; per-head scales with HS): tensor-core
-// kernel, head_dim 128.
-template <typename T, bool I8 = false, bool HS = false>
+// kernel, head_dim 64 or 128.
+template <int D, typename T, bool I8 = false, bool HS = false>
 pa_status dispatch_group_fp8(pa::DecodeParams &p, int group, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_decode_mma<128, 1, T, true, false, I8, HS>(p, stream);
-        case 2: return launch_decode_mma<128, 2, T, true, false, I8, HS>(p, stream);
-        case 4: return launch_decode_mma<128, 4, T, true, false, I8, HS>(p, stream);
-        case 8: return launch_decode_mma<128, 8, T, true, false, I8, HS>(p, stream);
+        case 1: return launch_decode_mma<D, 1, T, true, false, I8, HS>(p, stream);
+        case 2: return launch_decode_mma<D, 2, T, true, false, I8, HS>(p, stream);
+        case 4: return launch_decode_mma<D, 4, T, true, false, I8, HS>(p, stream);
+        case 8: return launch_decode_mma<D, 8, T, true, false, I8, HS>(p, stream);
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }

@@ -52,11 +52,12 @@ def test_shared_decode_host_checks_without_a_device():
     parts = 2048 // 512
     assert shared >= plain + 64 * 32 * (8 + 128 * 4) + 64 * (parts + 1) * 16 + 2 * 64 * 4
     assert lib.pa_decode_shared_workspace_size(4, 2, 2, 96, 16, 33, 0) == 0
-    # fp8 cache: 512 tokens for one query head per KV head, max(256, 8 blocks) otherwise, head_dim 128 only
+    # fp8 cache: 512 tokens for one query head per KV head, max(256, 8 blocks) otherwise, head_dim 64 or 128
     assert pa.pa_decode_fp8_partition_size(64, 32, 32, 128, 16, 2048, 0) == 512
     assert pa.pa_decode_fp8_partition_size(256, 32, 8, 128, 16, 8192, 0) == 256
     assert pa.pa_decode_fp8_partition_size(8, 32, 8, 128, 64, 32768, 0) == 512
-    assert pa.pa_decode_fp8_partition_size(8, 32, 8, 64, 16, 4096, 0) == 0
+    assert pa.pa_decode_fp8_partition_size(8, 32, 8, 64, 16, 4096, 0) == 256
+    assert pa.pa_decode_fp8_partition_size(8, 32, 8, 96, 16, 4096, 0) == 0
     assert pa.pa_decode_fp8_workspace_size(256, 32, 8, 128, 16, 8192, 0) > pa.pa_decode_workspace_size(
         256, 32, 8, 128, 16, 8192, 0)
     # shared-prefix units: 16 blocks for grouped heads, as pa_decode otherwise

@@ -125,14 +125,19 @@ def test_fp8_write_then_decode_end_to_end():
     assert float(np.abs(out.float().cpu().double().numpy() - ref).max()) <= TOL[wl.dtype]
 
 
-def test_fp8_rejects_unsupported_head_dim():
-    wl = workloads.tiny(0)                                    # head_dim 64
-    st = wl.steps[0]
-    k8 = torch.zeros((32, 2, 16, 64), dtype=torch.uint8, device="cuda")
-    with pytest.raises(pa.PagedAttentionError):
-        pa.pa_decode_fp8(torch.empty_like(st.q).cuda(), st.q.cuda(), k8, k8,
-                         torch.as_tensor(st.block_tables).cuda(), torch.as_tensor(st.context_lens).cuda(),
-                         wl.scale, 33, K_SCALE, V_SCALE)
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("llama7b", {"num_seqs": 8, "head_dim": 64}),
+                                     ("llama3_8b", {"num_seqs": 24, "head_dim": 64})])
+def test_fp8_head_dim_64(name, kw):
+    """head_dim 64: 64-byte tile rows (one 64-byte TMA box with the 64-byte
+    swizzle) against the oracle, one partition and split."""
+    wl = workloads.build(name, 37, **kw)
+    k8, v8 = fp8_pools(wl)
+    ref = oracle_decode(wl, k8, v8)
+    for partition in (None, 64):
+        out = run_decode(wl, k8, v8, partition)
+        err = float(np.abs(out.float().cpu().double().numpy() - ref).max())
+        assert err <= TOL[wl.dtype], (partition, err)
+        margins.record(f"fp8 D=64 {name} {wl.dtype} P={partition or 'auto'}", err, TOL[wl.dtype])
 
 
 def test_fp8_flags_bf16_queries_outside_f16_range():

@@ -181,18 +181,18 @@ def test_quant_rejects_bad_arguments():
 @pytest.mark.parametrize("fmt", FORMATS)
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
-def test_quant_every_head_group(fmt, group, dtype):
-    """Every query-head group size over both 8-bit formats, ragged contexts
-    (1 token to several partitions, partial last tiles), both query types."""
-    from paged_kv_cache_372_b200 import inputs
-    gen = inputs.generator(4800 + 10 * group + (dtype == "bf16"))
+@pytest.mark.parametrize("head_dim", [128, 64])
+def test_quant_every_head_group(fmt, group, dtype, head_dim):
+    """Every query-head group size over both 8-bit formats and both head sizes,
+    ragged contexts (1 token to several partitions, partial last tiles), both
+    query types."""
     ctx = [1, 15, 16, 17, 100, 333, 700, 1500]
-    wl, _ = workloads._decode_batch("groups", ctx, heads=2 * group, kv_heads=2, head_dim=128, block_size=16,
-                                    dtype=dtype, seed=4900 + group)
+    wl, _ = workloads._decode_batch("groups", ctx, heads=2 * group, kv_heads=2, head_dim=head_dim, block_size=16,
+                                    dtype=dtype, seed=4900 + group + head_dim)
     k8, v8, ks, vs = quant_pools(wl, fmt)
     for partition in (0, 64):
         out = run_decode(wl, fmt, k8, v8, ks, vs, partition)
         ref = oracle_decode(wl, fmt, k8, v8, ks, vs)
         err = float(np.abs(out.float().cpu().double().numpy() - ref).max())
         assert err <= TOL[dtype], (partition, err)
-        margins.record(f"{fmt} per-head G={group} {dtype} P={partition or 'auto'}", err, TOL[dtype])
+        margins.record(f"{fmt} per-head G={group} D={head_dim} {dtype} P={partition or 'auto'}", err, TOL[dtype])
