@@ -280,7 +280,6 @@ def run_ours(args, world, rank, local, extras=True):
             k=st.k_new.to(dev), v=st.v_new.to(dev), slots=torch.from_numpy(st.slot_mapping).to(dev),
             pairs=torch.from_numpy(st.copy_pairs).to(dev)))
     stream = torch.cuda.current_stream(dev)
-    launches_per_decode = 2  # plan + attention (split merge is fused)
     flush = needs_flush(wl)
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
 
@@ -295,7 +294,8 @@ def run_ours(args, world, rank, local, extras=True):
         ws = pa.alloc_workspace(B, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, max_ctx, P, dev,
                                 fp8=True)
     fused = not args.unfused and not kv8 and appends_at_last_positions(wl)
-    share = not kv8 and (args.share == "on" or (args.share == "auto" and wl.kv_bytes_unique() < wl.kv_bytes()))
+    share = (quant or not kv8) and (args.share == "on" or
+                                     (args.share == "auto" and wl.kv_bytes_unique() < wl.kv_bytes()))
     if share:
         ws = pa.alloc_workspace(B, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, max_ctx, P, dev,
                                 shared=True)
@@ -320,26 +320,23 @@ def run_ours(args, world, rank, local, extras=True):
 
     def step(i, ev=None):
         d = dev_steps[i % nsteps]
-        n = 0
         if d["pairs"].shape[0]:
             pa.pa_copy_blocks([kp, vp], d["pairs"])
-            n += 1
         if quant:
             pa.pa_reshape_and_cache_quant(d["k"], d["v"], kp, vp, d["slots"], qfmt, ksc, vsc)
-            n += 1
         elif kv8:
             pa.pa_reshape_and_cache_fp8(d["k"], d["v"], kp, vp, d["slots"], FP8_SCALE, FP8_SCALE)
-            n += 1
         elif fused:
             if d["slots_extra"].shape[0]:
                 pa.pa_reshape_and_cache(d["k_extra"], d["v_extra"], kp, vp, d["slots_extra"])
-                n += 1
         else:
             pa.pa_reshape_and_cache(d["k"], d["v"], kp, vp, d["slots"])
-            n += 1
         if ev is not None:
             ev[0].record(stream)
-        if quant:
+        if quant and share:
+            pa.pa_decode_shared_quant(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, qfmt,
+                                      ksc, vsc, P, ws)
+        elif quant:
             pa.pa_decode_quant(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, qfmt, ksc, vsc,
                                P, ws)
         elif kv8:
@@ -355,7 +352,6 @@ def run_ours(args, world, rank, local, extras=True):
             pa.pa_decode(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, P, ws)
         if ev is not None:
             ev[1].record(stream)
-        return n + launches_per_decode
 
     for i in range(args.warmup):
         step(i)
@@ -370,7 +366,7 @@ def run_ours(args, world, rank, local, extras=True):
     clocks = Clocks(dev.index) if rank == 0 else None
     barrier(world)
     torch.cuda.synchronize(dev)
-    launches = 0
+    launches0 = pa.pa_launch_count()
     # The K steps of the headline figure: no event between the kernels of a
     # step (an event record between two kernels idles the GPU for a moment),
     # unless the L2 flush has to be kept out of the step's time.
@@ -379,10 +375,11 @@ def run_ours(args, world, rank, local, extras=True):
         if flush:
             flush_buf.fill_(i & 0xff)        # evict the previous step's blocks from L2
             step_evs[i][0].record(stream)
-        launches += step(i)
+        step(i)
         if flush:
             step_evs[i][1].record(stream)
     stop.record(stream)
+    launches = pa.pa_launch_count() - launches0  # this library's kernels in the K steps
     torch.cuda.synchronize(dev)
     barrier(world)
     total_ms = (sum(a.elapsed_time(b) for a, b in step_evs) if flush else start.elapsed_time(stop))
@@ -434,20 +431,24 @@ def run_ours(args, world, rank, local, extras=True):
         "hbm_frac_of_nominal_8000": achieved / 8000.0,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
-                     "kernel": ("pa_decode_quant call (plan + attention launches; split merge fused)" if quant else
+                     "kernel": ("pa_decode_shared_quant call (grouping plan + attention launches; split merge "
+                                "in a launch of its own)" if quant and share else
+                                "pa_decode_quant call (plan + attention launches; split merge fused)" if quant else
                                 "pa_decode_fp8 call (plan + attention launches; split merge fused)" if kv8 else
-                                "pa_decode_shared call (grouping plan + attention launches; cache write and "
-                                "split merge fused)" if share and fused else
-                                "pa_decode_shared call (grouping plan + attention launches; split merge fused)"
-                                if share else
-                                "pa_decode_append call (plan + attention launches; cache write and split "
-                                "merge fused)" if fused else
-                                "pa_decode call (plan + attention launches; split merge fused)"),
+                                "pa_decode_shared call (grouping plan + attention launches; cache write fused, "
+                                "split merge in a launch of its own)" if share and fused else
+                                "pa_decode_shared call (grouping plan + attention launches; split merge in a "
+                                "launch of its own)" if share else
+                                "pa_decode_append call (plan + attention launches; cache write fused, split "
+                                "merge fused up to 16 partitions, a launch of its own beyond)" if fused else
+                                "pa_decode call (plan + attention launches; split merge fused up to 16 "
+                                "partitions, a launch of its own beyond)"),
                      "bytes": "unique K+V bytes of valid tokens per call",
                      "traffic": profiled_traffic(wl.name + (f"@{args.kv}" if kv8 else "") + ("@shared" if share else "")
                                                  + ("" if args.partition is None else f"@P{args.partition}"))},
         "gpu_launches": launches,
-        "step": ("pa_copy_blocks (if any), pa_reshape_and_cache_quant, pa_decode_quant" if quant else
+        "step": ("pa_copy_blocks (if any), pa_reshape_and_cache_quant, pa_decode_shared_quant" if quant and share
+                 else "pa_copy_blocks (if any), pa_reshape_and_cache_quant, pa_decode_quant" if quant else
                  "pa_copy_blocks (if any), pa_reshape_and_cache_fp8, pa_decode_fp8" if kv8 else
                  "pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_shared with "
                  "the new tokens" if share and fused else

@@ -92,6 +92,12 @@ PA_API const char *pa_status_string(int status);
 /* Text of the last failure on this host thread ("" if none). */
 PA_API const char *pa_last_error(void);
 
+/* Number of kernels this library has launched from the calling thread since
+ * it was loaded, over every entry point (a decode call is 2 or 3: plan,
+ * attention and, when it runs, the merge launch; a cache write 1). Host only;
+ * take the difference around a region to count its launches. */
+PA_API unsigned long long pa_launch_count(void);
+
 /*
  * Paged decode attention.
  *
@@ -198,6 +204,25 @@ PA_API pa_status pa_decode_shared(void *out, const void *q, const void *k_new, c
                                   int max_blocks_per_seq, int num_blocks, int max_context_len,
                                   float scale, int dtype, int partition_size, void *workspace,
                                   size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_decode_shared over an 8-bit cache: the codes, formats and per-KV-head
+ * scales of pa_decode_quant, the grouping and shared units of
+ * pa_decode_shared (without the fused append). Workspace and partition:
+ * pa_decode_shared_workspace_size / pa_decode_shared_partition_size. Same
+ * result as pa_decode_quant up to the order of the fp32 sums.
+ *
+ * Defined by: the sharing of "vLLM架构深度解析：PagedAttention如何实现高吞吐LLM推理",
+ * section KV Cache内存共享, over the compressed cache of "别再让GPU内存拖后腿了",
+ * section 3.2.
+ */
+PA_API pa_status pa_decode_shared_quant(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                        const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                        int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                        int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                                        int dtype, int kv_format, const float *k_scales, const float *v_scales,
+                                        int partition_size, void *workspace, size_t workspace_bytes,
+                                        pa_stream_t stream);
 
 /* Partition and workspace bytes pa_decode_fp8 (and pa_decode_quant) uses for
  * these arguments (0 if invalid). */

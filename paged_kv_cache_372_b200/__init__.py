@@ -92,6 +92,11 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_quant.restype = _I
         L.pa_decode_quant.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P,
                                       _I, _P, _SZ, _P]
+        L.pa_decode_shared_quant.restype = _I
+        L.pa_decode_shared_quant.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
+                                             _P, _P, _I, _P, _SZ, _P]
+        L.pa_launch_count.restype = ctypes.c_ulonglong
+        L.pa_launch_count.argtypes = []
         L.pa_decode_noalloc.restype = _I
         L.pa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]
         _lib = L
@@ -351,6 +356,30 @@ def pa_decode_quant(out, q, k_pool, v_pool, block_tables, context_lens, scale, m
     return out
 
 
+def pa_decode_shared_quant(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len, kv_format,
+                           k_scales, v_scales, partition_size=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode_shared over an 8-bit cache ("e4m3" or "int8" codes) with one
+    scale per KV head (float32 CUDA tensors [Hkv])."""
+    B, H, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch between q, out and the pools")
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("8-bit pools must be uint8 tensors of codes")
+    if q.dtype not in _DTYPES or out.dtype != q.dtype:
+        raise ValueError("q and out must share one dtype, fp16 or bf16")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device, shared=True)
+    _check(lib().pa_decode_shared_quant(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
+        B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
+        KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv), _scales(v_scales, "v_scales", Hkv),
+        int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return out
+
+
 def pa_reshape_and_cache(k, v, k_pool, v_pool, slot_mapping, stream=None) -> None:
     """k_pool[slot // bs][h][slot % bs] = k[t][h] (and v) for every t with slot >= 0."""
     T, Hkv, D = k.shape
@@ -415,6 +444,12 @@ def pa_swap_blocks(dst_pools, src_pools, src_dst_pairs, stream=None) -> None:
     sp = (_P * len(src_pools))(*[ptr(t, "src pool") for t in src_pools])
     _check(lib().pa_swap_blocks(dp, sp, len(dst_pools), ptr(pairs, "src_dst_pairs"), pairs.shape[0],
                                 block_bytes, src_pools[0].shape[0], dst_pools[0].shape[0], _stream(stream)))
+
+
+def pa_launch_count() -> int:
+    """Kernels the library has launched from the calling thread so far (all
+    entry points); the difference around a region is that region's count."""
+    return int(lib().pa_launch_count())
 
 
 def pa_device_errors(clear: bool = True, stream=None) -> int:

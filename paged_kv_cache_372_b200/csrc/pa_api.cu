@@ -18,6 +18,8 @@
 namespace {
 
 thread_local std::string g_last_error;
+// Kernels launched from this thread (every entry point; read by pa_launch_count).
+thread_local unsigned long long g_launches = 0;
 
 pa_status fail(pa_status st, const char *fmt, ...) {
     char buf[512];
@@ -106,6 +108,8 @@ const char *pa_status_string(int status) {
 }
 
 const char *pa_last_error(void) { return g_last_error.c_str(); }
+
+unsigned long long pa_launch_count(void) { return g_launches; }
 
 int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                              int max_context_len, int partition_size) {
@@ -249,6 +253,18 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int group = num_heads / num_kv_heads;
+    if (kv8 && shared) {
+        const bool d128 = head_dim == 128, f16 = dtype == PA_F16;
+        if (int8)
+            return d128 ? (f16 ? dispatch_group_shared_kv8<128, __half, true>(p, group, s)
+                               : dispatch_group_shared_kv8<128, __nv_bfloat16, true>(p, group, s))
+                        : (f16 ? dispatch_group_shared_kv8<64, __half, true>(p, group, s)
+                               : dispatch_group_shared_kv8<64, __nv_bfloat16, true>(p, group, s));
+        return d128 ? (f16 ? dispatch_group_shared_kv8<128, __half, false>(p, group, s)
+                           : dispatch_group_shared_kv8<128, __nv_bfloat16, false>(p, group, s))
+                    : (f16 ? dispatch_group_shared_kv8<64, __half, false>(p, group, s)
+                           : dispatch_group_shared_kv8<64, __nv_bfloat16, false>(p, group, s));
+    }
     if (kv8) {
         const bool d128 = head_dim == 128, f16 = dtype == PA_F16;
         if (int8)
@@ -330,6 +346,21 @@ pa_status pa_decode_shared(void *out, const void *q, const void *k_new, const vo
                        dtype, partition_size, workspace, workspace_bytes, stream, false, 1.f, 1.f, true);
 }
 
+pa_status pa_decode_shared_quant(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                 const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                 int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                                 int dtype, int kv_format, const float *k_scales, const float *v_scales,
+                                 int partition_size, void *workspace, size_t workspace_bytes, pa_stream_t stream) {
+    g_last_error.clear();
+    if (kv_format != PA_KV_E4M3 && kv_format != PA_KV_INT8) return fail(PA_ERR_INVALID, "kv_format %d", kv_format);
+    if (num_seqs > 0 && (!k_scales || !v_scales)) return fail(PA_ERR_INVALID, "null scale array");
+    return decode_impl(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream, true, 1.f, 1.f, true,
+                       kv_format == PA_KV_INT8, k_scales, v_scales);
+}
+
 pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void *v_pool, const int64_t *slot_mapping,
                                int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
                                int dtype, pa_stream_t stream) {
@@ -352,6 +383,7 @@ pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void 
     long long blocks = (total + 255) / 256;
     const long long cap = (long long)info.sms * 16;
     if (blocks > cap) blocks = cap;
+    ++g_launches;
     pa::pa_reshape_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(k_pool),
         static_cast<uint4 *>(v_pool), slot_mapping, total, vec_per_row, num_kv_heads, block_size,
@@ -380,6 +412,7 @@ pa_status reshape_kv8_impl(const void *k, const void *v, void *k_pool, void *v_p
     if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto launch = [&](auto kernel) {
+        ++g_launches;
         kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
                                                  static_cast<uint2 *>(k_pool), static_cast<uint2 *>(v_pool),
                                                  slot_mapping, total, vec_per_row, num_kv_heads, block_size,
@@ -473,6 +506,7 @@ pa_status pa_copy_blocks(void *const *pools, int num_pools, const int64_t *src_d
         pa::PoolList list;
         for (int i = 0; i < pa::COPY_MAX_POOLS; ++i) list.ptr[i] = i < n ? static_cast<uint4 *>(pools[first + i]) : nullptr;
         const dim3 grid((unsigned)num_pairs, (unsigned)n);
+        ++g_launches;
         pa::pa_copy_blocks_kernel<<<grid, 256, 0, s>>>(list, src_dst_pairs, (long long)(block_bytes / 16),
                                                        (long long)num_blocks);
     }
@@ -545,6 +579,7 @@ pa_status pa_swap_blocks(void *const *dst_pools, const void *const *src_pools, i
             src.ptr[i] = static_cast<const uint4 *>(sp);
         }
         const dim3 grid((unsigned)num_pairs, (unsigned)n);
+        ++g_launches;
         pa::pa_swap_blocks_kernel<<<grid, 256, 0, s>>>(dst, src, static_cast<const int64_t *>(pairs),
                                                        (long long)(block_bytes / 16), (long long)num_src_blocks,
                                                        (long long)num_dst_blocks);
@@ -574,6 +609,7 @@ pa_status pa_selftest_bounded_wait(unsigned long long limit_ns, pa_stream_t stre
     g_last_error.clear();
     if (limit_ns < 1000000ull || limit_ns > 10000000000ull)
         return fail(PA_ERR_INVALID, "limit %llu ns outside [1 ms, 10 s]", limit_ns);
+    ++g_launches;
     pa_bounded_wait_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "bounded-wait probe launch");

@@ -68,7 +68,7 @@ struct DecodeParams {
     // sequences whose block tables begin with the same blocks.
     int4 *entries_b; // {first token, member offset, member count (0: one sequence), 0}
     int *members;    // sequences in grouping order
-    int *member_nparts;  // partitions of members[i]
+    int *member_nparts;  // partitions of members[i] to merge (0: none, or written directly)
     int append_guard;    // 1: a sequence's last position never lies in a shared block
     int early;           // 1: the attention kernel starts without waiting for the one-warp plan
     int reduce_launch;   // 1: split partitions merge in pa_reduce_kernel, a launch of their own
@@ -418,7 +418,11 @@ __global__ void __launch_bounds__(PLAN_THREADS) pa_plan_shared_kernel(const Deco
             ptail = S - pfull * P;
         }
         p.members[tid] = m;
-        p.member_nparts[tid] = nparts;
+        // A sequence with one partition and no shared blocks has its output
+        // written by the attention kernel: 0 tells the merge launch to skip
+        // it. With shared blocks, even one partition (its whole context in a
+        // shared unit) is a partial that the merge normalises.
+        p.member_nparts[tid] = S == 0 && nparts == 1 ? 0 : nparts;
         if (stail > 0) atomicAdd(&s_bin_count[(stail + 15) >> 4], 1);
         if (ptail > 0) atomicAdd(&s_bin_count[(ptail + 15) >> 4], 1);
     }

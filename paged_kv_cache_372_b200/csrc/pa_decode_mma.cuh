@@ -117,15 +117,24 @@ __device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t codes) {
 
 // INT8 cache, stored excess-128 (byte u holds u - 128): the f16 number with
 // high byte 0x64 and low byte u is exactly 1024 + u, so one byte permute per
-// pair of codes makes the MMA operand; the constant 1152 = 1024 + 128 is
-// taken off afterwards (from the scores per query row, from the outputs with
-// the softmax sum). Codes in bytes 0 and 1 (low byte first) -> two f16.
+// pair of codes makes the MMA operand. For keys the constant 1152 = 1024 + 128
+// is taken off the scores afterwards (one correction per query row). Values
+// take it off in f16 before their product (i8_unbias, exact), since the
+// output sums grow over a whole partition and 1152 * (sum of the weights) in
+// fp32 would cost them about ten bits.
+// Codes in bytes 0 and 1 (low byte first) -> two f16.
 __device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t codes) { return __byte_perm(codes, 0x64646464u, 0x4140); }
 // Codes in bytes 2 and 3 -> two f16.
 __device__ __forceinline__ uint32_t i8x2_hi_to_f16x2(uint32_t codes) {
     return __byte_perm(codes, 0x64646464u, 0x4342);
 }
 constexpr float I8_OFFSET = 1152.f;
+// (1024 + u) - 1152 = u - 128, the signed code, exactly (two f16 at once).
+__device__ __forceinline__ uint32_t i8_unbias(uint32_t w) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0x64806480u));  // f16 1152 = 0x6480
+    return r;
+}
 
 // Two 16-bit query elements of type T -> f16x2 (bf16 -> f16 is exact in f16's
 // normal range). A bf16 element above f16's largest finite value (65504)
@@ -371,7 +380,7 @@ __global__ void __launch_bounds__(256) pa_reduce_members_kernel(const DecodePara
     if (item >= p.num_seqs * p.num_kv_heads) return;
     const int pos = item / p.num_kv_heads, kvh = item - pos * p.num_kv_heads;
     const int s = p.members[pos], nparts = p.member_nparts[pos];
-    if (nparts <= 1) return;  // written by the attention kernel
+    if (nparts < 1) return;  // empty, or written by the attention kernel (member_nparts 0)
     mma_merge<D, G, T>(p, (size_t)s * p.num_kv_heads + kvh, (size_t)s * p.num_heads + (size_t)kvh * G, 0, nparts,
                        lane);
 }
@@ -390,11 +399,12 @@ __global__ void pa_reduce_kernel(const DecodeParams p) {
     if constexpr (SM) {
         s = p.members[pos];
         nparts = p.member_nparts[pos];
+        if (nparts < 1) return;  // empty, or written by the attention kernel (member_nparts 0)
     } else {
         s = pos;
         nparts = (clamped_context(p, s, false) + p.partition - 1) / p.partition;
+        if (nparts <= 1) return;  // written by the attention kernel
     }
-    if (nparts <= 1) return;  // written by the attention kernel
     const size_t group = (size_t)s * p.num_kv_heads + kvh;
     const float2 *ml = p.ml + group * p.max_parts * G;
     for (int i = threadIdx.x; i < nparts * G; i += blockDim.x) s_ml[i] = __ldcg(ml + i);
@@ -653,7 +663,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
         // score scale uq, the value scale uv applies at the store (per unit
         // with per-head scales, HS; kernel parameters otherwise). kc0 / kc1
         // take the INT8 offset off the scores of query rows h0 / h1.
-        float uq = p.qscale, uv = p.v_scale, kc0 = 0.f, kc1 = 0.f;
+        float uq = p.qscale, uv = p.v_scale, kc0 = 0.f, kc1 = 0.f, kd0 = 0.f, kd1 = 0.f;
         if constexpr (HS) {
             uq = p.qscale * __ldg(p.k_scales + cur.kvh);
             uv = __ldg(p.v_scales + cur.kvh);
@@ -686,6 +696,15 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                         qb[i][1] = g8 < nrows ? to_f16x2<T>(
                                                     *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d + 2) * 2), qbig)
                                               : 0u;
+                        if constexpr (SHARED) {
+                            const int r = 8 + g8;
+                            qc[i][0] = r < nrows
+                                           ? to_f16x2<T>(*reinterpret_cast<const uint32_t *>(qs + (r * D + d) * 2), qbig)
+                                           : 0u;
+                            qc[i][1] = r < nrows ? to_f16x2<T>(
+                                                       *reinterpret_cast<const uint32_t *>(qs + (r * D + d + 2) * 2), qbig)
+                                                 : 0u;
+                        }
                     } else {
                         const int d = 16 * i + 2 * t4;
                         qb[i][0] = g8 < nrows ? *reinterpret_cast<const uint32_t *>(qs + (g8 * D + d) * 2) : 0u;
@@ -714,6 +733,19 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                     qs += __shfl_xor_sync(FULL_MASK, qs, 2);
                     kc0 = -I8_OFFSET * uq * __shfl_sync(FULL_MASK, qs, 8 * t4);
                     kc1 = -I8_OFFSET * uq * __shfl_sync(FULL_MASK, qs, 8 * t4 + 4);
+                    if constexpr (SHARED) {
+                        float qt = 0.f;  // the same for rows 8 + g8 (second half)
+#pragma unroll
+                        for (int i = 0; i < Gm::KS; ++i) {
+                            const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&qc[i][0]));
+                            const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&qc[i][1]));
+                            qt += (a.x + a.y) + (b.x + b.y);
+                        }
+                        qt += __shfl_xor_sync(FULL_MASK, qt, 1);
+                        qt += __shfl_xor_sync(FULL_MASK, qt, 2);
+                        kd0 = -I8_OFFSET * uq * __shfl_sync(FULL_MASK, qt, 8 * t4);
+                        kd1 = -I8_OFFSET * uq * __shfl_sync(FULL_MASK, qt, 8 * t4 + 4);
+                    }
                 }
             }
             const int valid = min(16, cur.ntok - 16 * k);
@@ -761,6 +793,9 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                             a[2] = e4m3x2_hi_to_f16x2(lo); a[3] = e4m3x2_hi_to_f16x2(hi);
                         }
                         MmaType<__half>::mma(h ? s2 : s, a, qb[i + h][0], qb[i + h][1]);
+                        if constexpr (SHARED) {
+                            if (two) MmaType<__half>::mma(h ? u2 : u, a, qc[i + h][0], qc[i + h][1]);
+                        }
                     }
                 }
             } else {
@@ -820,10 +855,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
             uint32_t pc0 = 0u, pc1 = 0u;
             if constexpr (SHARED) {
                 if (two) {
-                    const float y0 = v_lo ? (u[0] + u2[0]) * uq : -INFINITY;
-                    const float y1 = v_lo ? (u[1] + u2[1]) * uq : -INFINITY;
-                    const float y2 = v_hi ? (u[2] + u2[2]) * uq : -INFINITY;
-                    const float y3 = v_hi ? (u[3] + u2[3]) * uq : -INFINITY;
+                    const float y0 = v_lo ? fmaf(u[0] + u2[0], uq, kd0) : -INFINITY;
+                    const float y1 = v_lo ? fmaf(u[1] + u2[1], uq, kd1) : -INFINITY;
+                    const float y2 = v_hi ? fmaf(u[2] + u2[2], uq, kd0) : -INFINITY;
+                    const float y3 = v_hi ? fmaf(u[3] + u2[3], uq, kd1) : -INFINITY;
                     const bool raise2 = (hw0 && !(fmaxf(y0, y2) <= N0 + LAZY_MAX_LOG2)) ||
                                         (hw1 && !(fmaxf(y1, y3) <= N1 + LAZY_MAX_LOG2));
                     if (__any_sync(FULL_MASK, raise2)) {
@@ -886,10 +921,10 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                         uint32_t a[4];
                         if constexpr (I8) {
                             // Bytes 0 / 2 are element 2*g8 of the two tokens, 1 / 3 element 2*g8+1.
-                            a[0] = __byte_perm(r[2 * h], 0x64646464u, 0x4240);
-                            a[1] = __byte_perm(r[2 * h], 0x64646464u, 0x4341);
-                            a[2] = __byte_perm(r[2 * h + 1], 0x64646464u, 0x4240);
-                            a[3] = __byte_perm(r[2 * h + 1], 0x64646464u, 0x4341);
+                            a[0] = i8_unbias(__byte_perm(r[2 * h], 0x64646464u, 0x4240));
+                            a[1] = i8_unbias(__byte_perm(r[2 * h], 0x64646464u, 0x4341));
+                            a[2] = i8_unbias(__byte_perm(r[2 * h + 1], 0x64646464u, 0x4240));
+                            a[3] = i8_unbias(__byte_perm(r[2 * h + 1], 0x64646464u, 0x4341));
                         } else {
                             const uint32_t x = __byte_perm(r[2 * h], 0, 0x3120);      // tokens 0-7
                             const uint32_t y = __byte_perm(r[2 * h + 1], 0, 0x3120);  // tokens 8-15
@@ -897,6 +932,9 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                             a[2] = e4m3x2_to_f16x2(y); a[3] = e4m3x2_hi_to_f16x2(y);
                         }
                         MmaType<__half>::mma(o[i + h], a, pb0, pb1);
+                        if constexpr (SHARED) {
+                            if (two) MmaType<__half>::mma(o2[i + h], a, pc0, pc1);
+                        }
                     }
                 }
             } else {
@@ -928,16 +966,6 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
             if constexpr (SHARED) {
                 m0s += __shfl_xor_sync(FULL_MASK, m0s, off);
                 m1s += __shfl_xor_sync(FULL_MASK, m1s, off);
-            }
-        }
-        if constexpr (I8) {
-            // The values were multiplied as 1152 + code: take 1152 * (sum of the weights) off.
-#pragma unroll
-            for (int i = 0; i < Gm::KS; ++i) {
-                o[i][0] = fmaf(-I8_OFFSET, l0, o[i][0]);
-                o[i][2] = fmaf(-I8_OFFSET, l0, o[i][2]);
-                o[i][1] = fmaf(-I8_OFFSET, l1, o[i][1]);
-                o[i][3] = fmaf(-I8_OFFSET, l1, o[i][3]);
             }
         }
         const size_t head0 = (size_t)cur.s * H + (size_t)cur.kvh * G;

@@ -90,8 +90,10 @@ pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
         long long blocks = (total + 255) / 256;
         if (blocks > (long long)info.sms * 16) blocks = (long long)info.sms * 16;
         pa::pa_append_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
+        ++g_launches;
     }
     pa::pa_plan_kernel<<<1, pa::PLAN_WARP_THREADS, 0, stream>>>(p);
+    ++g_launches;
     // Programmatic dependent launch: the attention CTAs start their set-up
     // while the plan kernel runs and wait for its results in-kernel.
     cudaLaunchConfig_t cfg = {};
@@ -106,6 +108,7 @@ pa_status launch_decode(pa::DecodeParams &p, cudaStream_t stream) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, p);
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+    ++g_launches;
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
     return PA_OK;
@@ -232,12 +235,14 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
         // merge launch, one CTA per (member, KV head), all at once.
         p.reduce_launch = p.max_parts > 1 && reduce_smem_bytes<D, G>(p.max_parts) <= REDUCE_SMEM_MAX;
         pa::pa_plan_shared_kernel<<<1, pa::PLAN_THREADS, 0, stream>>>(p);
+        ++g_launches;
     } else {
         p.early = p.num_seqs <= EARLY_MAX_SEQS;
         // Many partitions per sequence: merge them in a launch of their own
         // (while its (max, sum) pairs fit the reduce kernel's shared memory).
         p.reduce_launch = p.l1_base > REDUCE_LAUNCH_MIN_PARTS && reduce_smem_bytes<D, G>(p.l1_base) <= REDUCE_SMEM_MAX;
         pa::pa_plan_kernel<<<1, pa::PLAN_WARP_THREADS, 0, stream>>>(p);
+        ++g_launches;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sms);
@@ -251,6 +256,7 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, p, tmk, tmv);
     if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+    ++g_launches;
     {
         if (p.reduce_launch) {
             constexpr int V4 = D * G / 4;
@@ -271,6 +277,7 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
                 if (e == cudaSuccess) e = cudaLaunchKernelEx(&rc, pa::pa_reduce_kernel<D, G, T>, p);
             }
             if (e != cudaSuccess) return cuda_fail(e, "pa_reduce_kernel launch");
+            ++g_launches;
         }
     }
     e = cudaGetLastError();
@@ -301,6 +308,18 @@ pa_status dispatch_group_shared(pa::DecodeParams &p, int group, cudaStream_t str
         case 2: return launch_decode_mma<D, 2, T, false, true>(p, stream);
         case 4: return launch_decode_mma<D, 4, T, false, true>(p, stream);
         case 8: return launch_decode_mma<D, 8, T, false, true>(p, stream);
+    }
+    return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
+}
+
+// Shared-prefix units over an 8-bit cache (one scale per KV head).
+template <int D, typename T, bool I8>
+pa_status dispatch_group_shared_kv8(pa::DecodeParams &p, int group, cudaStream_t stream) {
+    switch (group) {
+        case 1: return launch_decode_mma<D, 1, T, true, true, I8, true>(p, stream);
+        case 2: return launch_decode_mma<D, 2, T, true, true, I8, true>(p, stream);
+        case 4: return launch_decode_mma<D, 4, T, true, true, I8, true>(p, stream);
+        case 8: return launch_decode_mma<D, 8, T, true, true, I8, true>(p, stream);
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }

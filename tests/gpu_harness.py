@@ -28,7 +28,7 @@ def gpu_step(wl, step, kp, vp, partition_size=None, workspace=None):
     pa.pa_reshape_and_cache(st.k_new.to(dev), st.v_new.to(dev), kp, vp,
                             torch.from_numpy(st.slot_mapping).to(dev))
     q = st.q.to(dev)
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     P = wl.partition_size if partition_size is None else partition_size
     pa.pa_decode(out, q, kp, vp, torch.from_numpy(st.block_tables).to(dev),
                  torch.from_numpy(st.context_lens).to(dev), wl.scale,
@@ -77,7 +77,7 @@ def gpu_step_fused(wl, step, kp, vp, partition_size=None, workspace=None):
         pa.pa_reshape_and_cache(st.k_new[B:].to(dev), st.v_new[B:].to(dev), kp, vp,
                                 torch.from_numpy(st.slot_mapping[B:]).to(dev))
     q = st.q.to(dev)
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     P = wl.partition_size if partition_size is None else partition_size
     pa.pa_decode_append(out, q, st.k_new[:B].contiguous().to(dev), st.v_new[:B].contiguous().to(dev), kp, vp,
                         torch.from_numpy(st.block_tables).to(dev), torch.from_numpy(st.context_lens).to(dev),
@@ -99,7 +99,7 @@ def gpu_step_shared(wl, step, kp, vp, partition_size=None, workspace=None, fused
         pa.pa_reshape_and_cache(st.k_new[first:].to(dev), st.v_new[first:].to(dev), kp, vp,
                                 torch.from_numpy(st.slot_mapping[first:]).to(dev))
     q = st.q.to(dev)
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     P = wl.partition_size if partition_size is None else partition_size
     kw = {}
     if fused:

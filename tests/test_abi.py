@@ -73,6 +73,14 @@ def test_shared_decode_host_checks_without_a_device():
     # more sequences than the grouping takes
     assert lib.pa_decode_shared(*args, 1025, *rest) == pa.PA_ERR_UNSUPPORTED
     assert b"1024" in lib.pa_last_error()
+    # 8-bit cache: format, scale arrays, then the same limits
+    qargs = [dummy, dummy, dummy, dummy, dummy, dummy]
+    qrest = [32, 8, 128, 16, 64, 4096, 1024, ctypes.c_float(0.1), 0]
+    tail = [0, dummy, 1 << 30, None]
+    assert lib.pa_decode_shared_quant(*qargs, 8, *qrest, 7, dummy, dummy, *tail) == pa.PA_ERR_INVALID
+    assert lib.pa_decode_shared_quant(*qargs, 8, *qrest, pa.PA_KV_INT8, None, dummy, *tail) == pa.PA_ERR_INVALID
+    assert lib.pa_decode_shared_quant(*qargs, 1025, *qrest, pa.PA_KV_E4M3, dummy, dummy, *tail) == \
+        pa.PA_ERR_UNSUPPORTED
 
 
 def _header_declarations():

@@ -32,7 +32,7 @@ def fp8_pools(wl):
 def run_decode(wl, k8, v8, partition=None, tables=None):
     st = wl.steps[0]
     q = st.q.cuda()
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     tab = st.block_tables if tables is None else tables
     pa.pa_decode_fp8(out, q, k8.cuda(), v8.cuda(), torch.as_tensor(tab).cuda(),
                      torch.from_numpy(st.context_lens).cuda(), wl.scale, int(st.context_lens.max()),
@@ -149,7 +149,7 @@ def test_fp8_flags_bf16_queries_outside_f16_range():
     st = wl.steps[0]
     q = st.q.clone()
     q[2, 5, 17] = 1.0e5                           # representable in bf16, not in f16
-    out = torch.empty_like(q).cuda()
+    out = torch.full_like(q, float("nan")).cuda()
     pa.pa_decode_fp8(out, q.cuda(), k8.cuda(), v8.cuda(), torch.from_numpy(st.block_tables).cuda(),
                      torch.from_numpy(st.context_lens).cuda(), wl.scale, int(st.context_lens.max()),
                      K_SCALE, V_SCALE)

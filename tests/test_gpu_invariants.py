@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 def decode(wl, kp, vp, tables, ctx, q=None, partition=0):
     st = wl.steps[0]
     q = (st.q if q is None else q).cuda()
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     pa.pa_decode(out, q, kp, vp, torch.as_tensor(tables).cuda(), torch.as_tensor(ctx).cuda(),
                  wl.scale, int(np.max(ctx)), partition)
     torch.cuda.synchronize()
@@ -137,7 +137,7 @@ def test_context_above_limit_is_clamped_and_flagged():
     st = wl.steps[0]
     kp, vp = wl.k_pool.cuda(), wl.v_pool.cuda()
     q = st.q.cuda()
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     pa.pa_device_errors(clear=True)
     ctx = torch.as_tensor(st.context_lens).cuda()
     pa.pa_decode(out, q, kp, vp, torch.as_tensor(st.block_tables).cuda(), ctx, wl.scale, 20)
@@ -162,7 +162,7 @@ def test_invalid_arguments_return_status():
     st = wl.steps[0]
     kp, vp = wl.k_pool.cuda(), wl.v_pool.cuda()
     q = st.q.cuda()
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     tab = torch.as_tensor(st.block_tables).cuda()
     ctx = torch.as_tensor(st.context_lens).cuda()
     L = pa.lib()

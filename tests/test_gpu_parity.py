@@ -141,3 +141,24 @@ def test_fused_append_matches_oracle_and_unfused_path(name, kw):
         err = H.max_err(fused, ref)
         assert err <= H.TOL[wl.dtype]
         margins.record(f"fused append {name} {wl.dtype}", err, H.TOL[wl.dtype])
+
+
+@pytest.mark.parametrize("partition,launches", [(512, 2), (128, 3)])
+def test_launch_count(partition, launches):
+    """A decode call is the plan and the attention launch; with more than 16
+    partitions a sequence's merge runs in a third launch. The library's
+    counter (the bench's gpu_launches) sees exactly these."""
+    wl = workloads.long32k(3, num_seqs=2, ctx_len=4096, prefill_tokens=0)
+    st = wl.steps[0]
+    dev = torch.device("cuda")
+    q = st.q.to(dev)
+    out = torch.full_like(q, float("nan"))  # every row must be written
+    kp, vp = wl.k_pool.to(dev), wl.v_pool.to(dev)
+    tab, ctx = torch.from_numpy(st.block_tables).to(dev), torch.from_numpy(st.context_lens).to(dev)
+    ws = pa.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, 4096,
+                            partition, dev)
+    n0 = pa.pa_launch_count()
+    pa.pa_decode(out, q, kp, vp, tab, ctx, wl.scale, 4096, partition, ws)
+    assert pa.pa_launch_count() - n0 == launches
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0

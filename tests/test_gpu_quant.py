@@ -46,7 +46,7 @@ def quant_pools(wl, fmt):
 def run_decode(wl, fmt, k8, v8, ks, vs, partition=None, tables=None):
     st = wl.steps[0]
     q = st.q.cuda()
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     tab = st.block_tables if tables is None else tables
     pa.pa_decode_quant(out, q, k8.cuda(), v8.cuda(), torch.as_tensor(tab).cuda(),
                        torch.from_numpy(st.context_lens).cuda(), wl.scale, int(st.context_lens.max()), fmt,
@@ -85,6 +85,20 @@ def test_quant_split_partitions(fmt, partition):
     assert float(np.abs(out.float().cpu().double().numpy() - ref).max()) <= TOL[wl.dtype]
 
 
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_quant_longest_partitions(fmt):
+    """2048-token partitions (32 blocks of 64): the value sums of a whole
+    partition stay within the tolerance (INT8 values enter the product as
+    exact signed codes, not offset by a constant that the sums would carry)."""
+    wl = workloads.long32k(48, num_seqs=2, ctx_len=5000, prefill_tokens=0)
+    k8, v8, ks, vs = quant_pools(wl, fmt)
+    out = run_decode(wl, fmt, k8, v8, ks, vs, 2048)
+    ref = oracle_decode(wl, fmt, k8, v8, ks, vs)
+    err = float(np.abs(out.float().cpu().double().numpy() - ref).max())
+    assert err <= TOL[wl.dtype], err
+    margins.record(f"{fmt} per-head long32k {wl.dtype} P=2048", err, TOL[wl.dtype])
+
+
 def test_quant_e4m3_with_equal_scales_is_the_fp8_path():
     """Per-head scales all equal to s give pa_decode_fp8's result with k_scale =
     v_scale = s, bit for bit (the same kernel, the scales only moved)."""
@@ -95,7 +109,7 @@ def test_quant_e4m3_with_equal_scales_is_the_fp8_path():
     one = torch.full((wl.num_kv_heads,), s, dtype=torch.float32)
     a = run_decode(wl, "e4m3", k8, v8, one, one)
     st = wl.steps[0]
-    b = torch.empty_like(a)
+    b = torch.full_like(a, float("nan"))
     pa.pa_decode_fp8(b, st.q.cuda(), k8.cuda(), v8.cuda(), torch.from_numpy(st.block_tables).cuda(),
                      torch.from_numpy(st.context_lens).cuda(), wl.scale, int(st.context_lens.max()), s, s)
     torch.cuda.synchronize()

@@ -150,7 +150,7 @@ def run_shared(case, P, append, workspace=None):
     dev = torch.device("cuda")
     kp, vp = case["kp"].to(dev), case["vp"].to(dev)
     q = case["q"].to(dev)
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     B, H_, D = q.shape
     mx = int(case["ctx"].max())
     if workspace is None:
@@ -169,7 +169,7 @@ def run_plain(case, P, append):
     dev = torch.device("cuda")
     kp, vp = case["kp"].to(dev), case["vp"].to(dev)
     q = case["q"].to(dev)
-    out = torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))  # every row must be written
     mx = int(case["ctx"].max())
     tab, ctx = torch.from_numpy(case["tables"]).to(dev), torch.from_numpy(case["ctx"]).to(dev)
     if append:
@@ -268,7 +268,7 @@ def test_without_sharing_equals_plain_decode():
     for ctx_np in (np.minimum(st.context_lens, 8 * 128), st.context_lens):
         ctx = torch.from_numpy(np.ascontiguousarray(ctx_np)).to(dev)
         mx = int(ctx_np.max())
-        a, b = torch.empty_like(q), torch.empty_like(q)
+        a, b = torch.full_like(q, float("nan")), torch.full_like(q, float("nan"))
         pa.pa_decode(a, q, kp, vp, tab, ctx, wl.scale, mx, 128)
         pa.pa_decode_shared(b, q, kp, vp, tab, ctx, wl.scale, mx, 128)
         torch.cuda.synchronize()
@@ -286,3 +286,39 @@ def test_too_many_sequences_rejected():
     with pytest.raises(pa.PagedAttentionError) as e:
         pa.pa_decode_shared(torch.empty_like(q), q, kp, kp.clone(), tab, ctx, 0.125, 1, 0, ws)
     assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+def whole_unit_case(group):
+    """Three sequences with identical tables whose whole 64-token context is one
+    shared unit (at partitions longer than that), next to a sequence with one
+    partition of its own and one with several."""
+    from paged_kv_cache_372_b200 import inputs
+    gen = inputs.generator(90 + group)
+    bs, D, kvh = 16, 128, 2
+    heads = kvh * group
+    NB = 64
+    tables = np.full((5, 8), -1, dtype=np.int32)
+    same = [3, 17, 9, 40]
+    tables[0, :4] = same
+    tables[1, :4] = same
+    tables[2, :4] = same
+    tables[3, :2] = [5, 6]
+    tables[4, :8] = [20, 21, 22, 23, 24, 25, 26, 27]
+    ctx = np.array([64, 64, 64, 20, 128], dtype=np.int32)
+    return dict(kp=inputs.normal((NB, kvh, bs, D), "f16", gen), vp=inputs.normal((NB, kvh, bs, D), "f16", gen),
+                q=inputs.normal((5, heads, D), "f16", gen), tables=tables, ctx=ctx, scale=D ** -0.5, dtype="f16",
+                bs=bs, heads=heads, kv_heads=kvh)
+
+
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+def test_whole_context_in_one_shared_unit(group):
+    """A member whose only partial is a shared unit's still has it normalised
+    into the output (by the merge launch); the sequence with one partition of
+    its own is written directly."""
+    case = whole_unit_case(group)
+    ref, _, _ = run_oracle(case, False)
+    for P in (256, 32):
+        out = run_shared(case, P, False)[0]
+        assert not torch.isnan(out).any()
+        err = H.max_err(out, ref)
+        assert err <= H.TOL["f16"], (P, err)
