@@ -310,10 +310,11 @@ PA_API pa_status pa_reshape_and_cache_quant(const void *k, const void *v, void *
  * v_scales[j] * decode(code), decode being E4M3 (PA_KV_E4M3) or code - 128
  * (PA_KV_INT8); otherwise exactly pa_decode (q and out fp16/bf16 by dtype).
  * head_dim 64 or 128. The partition and the workspace are those of pa_decode_fp8
- * (pa_decode_fp8_partition_size, pa_decode_fp8_workspace_size). INT8 codes
- * enter the tensor-core products as the exact fp16 numbers 1152 + (code - 128);
- * the constant is taken off the scores (per query row) and the outputs (times
- * the softmax sum) in fp32. Queries are converted to fp16 as in pa_decode_fp8
+ * (pa_decode_fp8_partition_size, pa_decode_fp8_workspace_size). INT8 key
+ * codes enter the tensor-core product as the exact fp16 numbers
+ * 1152 + (code - 128), the constant taken off each score (per query row) in
+ * fp32; value codes enter it as the exact fp16 numbers code - 128 (one fp16
+ * subtraction per pair). Queries are converted to fp16 as in pa_decode_fp8
  * (PA_DEVERR_QRANGE for bf16 elements above 65504).
  *
  * Defined by: the same section 3.2; the attention is that of section 3.1.

@@ -39,10 +39,11 @@ namespace pa {
 // A tile row is D * EB bytes: 256 or 128 (loaded in 128-byte boxes with the
 // 128-byte swizzle) or 64 (an 8-bit cache at head_dim 64: one 64-byte box
 // with the 64-byte swizzle).
-template <int D, int G, bool KV8 = false>
+template <int D, int G, bool KV8 = false, int TR_ = 16>
 struct MmaGeo {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "head group size");
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static constexpr int TR = TR_;                        // tokens (rows) of one item
     static constexpr int EB = KV8 ? 1 : 2;                // bytes per pool element
     static constexpr int KS = D / 16;                     // 16-wide slices of a row
     static constexpr int ROW_BYTES = D * EB;
@@ -51,11 +52,21 @@ struct MmaGeo {
     static constexpr int NBOX = ROW_BYTES / BOX_ROW;      // TMA boxes per row
     static constexpr int BOX_BYTES = 16 * BOX_ROW;        // one box of a 16-row tile
     static constexpr int CHUNKS = ROW_BYTES / 16;         // 16-byte chunks of a row
-    static constexpr int HALF_BYTES = 16 * D * EB;        // one K (or V) tile
+    static constexpr int HALF_BYTES = TR * D * EB;        // one K (or V) tile
     static constexpr int STAGE_BYTES = 2 * HALF_BYTES;    // K then V of one tile
+    static constexpr int SUB_BYTES = 2 * 16 * D * EB;     // K and V rows of one 16-row sub-tile
+    static_assert(TR == 16 || (TR == 32 && NBOX == 1), "32-row tiles take one box per row");
     // Byte offset of 16-byte chunk `chunk` of row `row` of a tile.
     static __device__ __forceinline__ uint32_t addr(int row, int chunk);
 };
+
+// Tokens per item (stage): 32 for the 8-bit kernels without shared units (two
+// 16-token MMA sub-tiles behind one wait, one softmax update and one issue,
+// which halves the per-token share of that fixed work), 16 otherwise.
+template <bool KV8, bool SHARED>
+__host__ __device__ constexpr int mma_tile_rows() {
+    return KV8 && !SHARED ? 32 : 16;
+}
 
 // Query rows of a unit shared by several sequences: two n8 column halves of
 // the MMA tile, the G rows of each of up to 16 / G member sequences.
@@ -76,7 +87,8 @@ __host__ __device__ constexpr int mma_q_slots() {
 
 template <int D, int G, int NS, bool KV8 = false, bool SHARED = false>
 __host__ __device__ constexpr int mma_warp_bytes() {
-    return NS * MmaGeo<D, G, KV8>::STAGE_BYTES + mma_q_slots<SHARED>() * mma_q_slot_bytes<D, G, SHARED>() + NS * 8;
+    return NS * MmaGeo<D, G, KV8, mma_tile_rows<KV8, SHARED>()>::STAGE_BYTES +
+           mma_q_slots<SHARED>() * mma_q_slot_bytes<D, G, SHARED>() + NS * 8;
 }
 
 template <int D, int G, int NS, bool KV8 = false, bool SHARED = false>
@@ -85,18 +97,20 @@ __host__ __device__ constexpr int mma_smem_bytes(int warps) {
     return 1024 + warps * mma_warp_bytes<D, G, NS, KV8, SHARED>();
 }
 
-// Warps per CTA: the fp8 kernel runs DECODE_MAX_WARPS_FP8 warps for small head
-// groups (up to 4 query heads per KV head, where it fits 128 registers a
-// thread), DECODE_MAX_WARPS otherwise.
+// Warps per CTA: the 8-bit kernel at head_dim 64 runs DECODE_MAX_WARPS_FP8
+// warps for small head groups (up to 4 query heads per KV head, where it fits
+// 128 registers a thread); at head_dim 128 its 32-token stages leave shared
+// memory for DECODE_MAX_WARPS (up to 170 registers a thread).
 #ifndef PA_FP8_WIDE_MAX_GROUP
 #define PA_FP8_WIDE_MAX_GROUP 4
 #endif
 // Shared-prefix units keep a second half of query columns (accumulators and
 // query fragments): 8 warps per CTA, so each thread has up to 255 registers.
 constexpr int SHARE_MAX_WARPS = 8;
-template <int G, bool KV8, bool SHARED = false>
+template <int D, int G, bool KV8, bool SHARED = false>
 __host__ __device__ constexpr int mma_max_warps() {
-    return SHARED ? SHARE_MAX_WARPS : KV8 && G <= PA_FP8_WIDE_MAX_GROUP ? DECODE_MAX_WARPS_FP8 : DECODE_MAX_WARPS;
+    return SHARED ? SHARE_MAX_WARPS
+                  : KV8 && D == 64 && G <= PA_FP8_WIDE_MAX_GROUP ? DECODE_MAX_WARPS_FP8 : DECODE_MAX_WARPS;
 }
 
 // E4M3 -> f16 widening: every E4M3 value is exactly an f16. One cvt converts
@@ -217,8 +231,8 @@ __device__ __forceinline__ uint32_t swz64(int row, int chunk) {
     return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
 }
 
-template <int D, int G, bool KV8>
-__device__ __forceinline__ uint32_t MmaGeo<D, G, KV8>::addr(int row, int chunk) {
+template <int D, int G, bool KV8, int TR_>
+__device__ __forceinline__ uint32_t MmaGeo<D, G, KV8, TR_>::addr(int row, int chunk) {
     if constexpr (BOX_ROW == 64)
         return swz64(row, chunk);
     else
@@ -450,12 +464,15 @@ __global__ void pa_reduce_kernel(const DecodeParams p) {
 }
 
 template <int D, int G, typename T, int NS, bool KV8 = false, bool SHARED = false, bool I8 = false, bool HS = false>
-__global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
+__global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
     pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
     static_assert(!I8 || KV8, "INT8 codes are an 8-bit cache");
     static_assert(!HS || KV8, "per-head scales are an 8-bit cache's");
-    using Gm = MmaGeo<D, G, KV8>;
+    using Gm = MmaGeo<D, G, KV8, mma_tile_rows<KV8, SHARED>()>;
+    constexpr int TR = Gm::TR;   // tokens of an item
+    constexpr int NT = TR / 16;  // its 16-token MMA sub-tiles
+    static_assert(!SHARED || NT == 1, "shared units keep 16-token items");
     constexpr int QB = mma_q_slot_bytes<D, G, SHARED>();  // bytes of one query slot
     constexpr int QS = mma_q_slots<SHARED>();              // query slots per warp
     constexpr int QG = G * D * 2;                          // query rows of one sequence
@@ -495,15 +512,23 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
         asm volatile("griddepcontrol.wait;" ::: "memory");
         src.init(p, lane, *p.num_entries * Hkv, SHARED, warps, warps * (int)gridDim.x);
     }
-    auto fetch = [&](Unit &x) { src.take(x); };
+    auto fetch = [&](Unit &x) {
+        src.take(x);
+        if constexpr (NT > 1) x.ntiles = (x.ntok + TR - 1) / TR;  // items of TR tokens
+    };
 
-    // Item `it` of a unit is its tile `it`: the K and V rows of 16 tokens;
+    // Item `it` of a unit is its tile `it`: the K and V rows of TR tokens (one
+    // 16-row box per sub-tile; a sub-tile past the unit's end is not loaded);
     // item 0 also brings the unit's query rows (G per member sequence; mseq
     // is lane j's member sequence for a unit of mcnt > 0 members).
-    auto issue = [&](int s, int kvh, int tbl, int qslot, int mcnt, int mseq, int it, uint32_t stage) {
-        const int tok = 16 * it;
+    auto issue = [&](int s, int kvh, int tbl, int ntok, int qslot, int mcnt, int mseq, int it, uint32_t stage) {
+        const int tok = TR * it;
         const int bi = tok / bs;
         const int pb = __shfl_sync(FULL_MASK, tbl, bi);
+        // Second sub-tile (TR = 32): its block, if it holds tokens of the unit.
+        const bool sub1 = NT > 1 && tok + 16 < ntok;
+        const int bi1 = (tok + 16) / bs;
+        const int pb1 = NT > 1 ? __shfl_sync(FULL_MASK, tbl, bi1 & 31) : 0;
         // Member sequences of a shared unit reach the issuing lane by shuffle.
         int mid[SHARED ? SHARE_ROWS : 1];
         if constexpr (SHARED) {
@@ -513,20 +538,28 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
         if (lane == 0) {
             const uint32_t bar = bar_s + 8 * stage;
             const bool ok = (unsigned)pb < (unsigned)p.num_blocks;
-            if (!ok) raise_error(PA_DEVERR_BLOCK_ID);
+            const bool ok1 = sub1 && (unsigned)pb1 < (unsigned)p.num_blocks;
+            if (!ok || sub1 != ok1) raise_error(PA_DEVERR_BLOCK_ID);
             const int qrows_bytes = it != 0 ? 0 : (SHARED && mcnt > 0 ? mcnt * QG : QG);
-            const uint32_t bytes = (ok ? Gm::STAGE_BYTES : 0) + qrows_bytes;
+            const uint32_t bytes = (ok ? Gm::SUB_BYTES : 0) + (ok1 ? Gm::SUB_BYTES : 0) + qrows_bytes;
             fence_proxy_async_smem();
             if (bytes) {
                 mbar_arrive_expect_tx(bar, bytes);
+                const uint32_t dst = ring_s + stage * Gm::STAGE_BYTES;
                 if (ok) {
                     const int row = (pb * Hkv + kvh) * bs + (tok - bi * bs);
-                    const uint32_t dst = ring_s + stage * Gm::STAGE_BYTES;
 #pragma unroll
                     for (int b = 0; b < Gm::NBOX; ++b) {
                         tma_load_2d(dst + b * Gm::BOX_BYTES, &tm_k, Gm::BOX_ELEMS * b, row, bar, policy);
                         tma_load_2d(dst + Gm::HALF_BYTES + b * Gm::BOX_BYTES, &tm_v, Gm::BOX_ELEMS * b, row, bar,
                                     policy);
+                    }
+                }
+                if constexpr (NT > 1) {
+                    if (ok1) {  // rows 16..31 of the tile (one box per row)
+                        const int row1 = (pb1 * Hkv + kvh) * bs + (tok + 16 - bi1 * bs);
+                        tma_load_2d(dst + Gm::BOX_BYTES, &tm_k, 0, row1, bar, policy);
+                        tma_load_2d(dst + Gm::HALF_BYTES + Gm::BOX_BYTES, &tm_v, 0, row1, bar, policy);
                     }
                 }
                 if (it == 0) {
@@ -586,9 +619,9 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                 cur_q_item = issued;
         }
         if (prod_on_nxt)
-            issue(nxt.s, nxt.kvh, nxt.tbl, nxt.slot, nxt.mcnt, nxt.mseq, pitem, issued % NS);
+            issue(nxt.s, nxt.kvh, nxt.tbl, nxt.ntok, nxt.slot, nxt.mcnt, nxt.mseq, pitem, issued % NS);
         else
-            issue(cur.s, cur.kvh, cur.tbl, cur.slot, cur.mcnt, cur.mseq, pitem, issued % NS);
+            issue(cur.s, cur.kvh, cur.tbl, cur.ntok, cur.slot, cur.mcnt, cur.mseq, pitem, issued % NS);
         ++pitem;
         ++issued;
         // One link of the next unit's claim per issued item, over the unit's
@@ -748,14 +781,14 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                     }
                 }
             }
-            const int valid = min(16, cur.ntok - 16 * k);
+            const int valid = min(TR, cur.ntok - TR * k);  // tokens of the item
             if (app_unit && k == cur.ntiles - 1) {
                 const int tok = cur.ntok - 1;  // the sequence's last position, in this tile
                 const int pb = __shfl_sync(FULL_MASK, cur.tbl, tok / bs);
                 if (lane < 2 * NVR) {
                     const int half = lane / NVR, c = lane % NVR;
                     uint8_t *st = ring + stage * Gm::STAGE_BYTES + half * Gm::HALF_BYTES;
-                    *reinterpret_cast<uint4 *>(st + Gm::addr(tok & 15, c)) = newrow;
+                    *reinterpret_cast<uint4 *>(st + Gm::addr(tok % TR, c)) = newrow;
                     if ((unsigned)pb < (unsigned)p.num_blocks) {
                         T *pool = static_cast<T *>(const_cast<void *>(half ? p.v_pool : p.k_pool));
                         *reinterpret_cast<uint4 *>(pool + (((size_t)pb * Hkv + cur.kvh) * bs + tok % bs) * D + c * 8) =
@@ -769,8 +802,15 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
             }
 
             // ---------------- S^T = K . Q^T ------------------------------------
-            // Two accumulators (even / odd slices) halve the chain of dependent MMAs.
-            float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+            // Per 16-token sub-tile j of the item: two accumulators (even / odd
+            // slices) halve the chain of dependent MMAs, and the sub-tiles'
+            // chains are independent of each other. A sub-tile with no token of
+            // the unit was not loaded and is skipped (warp-uniform).
+            float s[NT][4], s2[NT][4];
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) s[j][c] = s2[j][c] = 0.f;
             float u[4] = {0.f, 0.f, 0.f, 0.f}, u2[4] = {0.f, 0.f, 0.f, 0.f};  // second half
             if constexpr (KV8) {
                 // A 16-byte chunk holds 16 codes of a row; ldmatrix on byte pairs
@@ -778,23 +818,27 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                 const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
                 const int csel = lane >> 4;
 #pragma unroll
-                for (int i = 0; i < Gm::KS; i += 2) {
-                    uint32_t r[4];
-                    ldsm_x4(r, ks_s + Gm::addr(row, i + csel));
+                for (int j = 0; j < NT; ++j) {
+                    if (j > 0 && valid <= 16 * j) break;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
-                        uint32_t a[4];
-                        if constexpr (I8) {
-                            a[0] = i8x2_to_f16x2(lo); a[1] = i8x2_to_f16x2(hi);
-                            a[2] = i8x2_hi_to_f16x2(lo); a[3] = i8x2_hi_to_f16x2(hi);
-                        } else {
-                            a[0] = e4m3x2_to_f16x2(lo); a[1] = e4m3x2_to_f16x2(hi);
-                            a[2] = e4m3x2_hi_to_f16x2(lo); a[3] = e4m3x2_hi_to_f16x2(hi);
-                        }
-                        MmaType<__half>::mma(h ? s2 : s, a, qb[i + h][0], qb[i + h][1]);
-                        if constexpr (SHARED) {
-                            if (two) MmaType<__half>::mma(h ? u2 : u, a, qc[i + h][0], qc[i + h][1]);
+                    for (int i = 0; i < Gm::KS; i += 2) {
+                        uint32_t r[4];
+                        ldsm_x4(r, ks_s + Gm::addr(16 * j + row, i + csel));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t lo = r[2 * h], hi = r[2 * h + 1];
+                            uint32_t a[4];
+                            if constexpr (I8) {
+                                a[0] = i8x2_to_f16x2(lo); a[1] = i8x2_to_f16x2(hi);
+                                a[2] = i8x2_hi_to_f16x2(lo); a[3] = i8x2_hi_to_f16x2(hi);
+                            } else {
+                                a[0] = e4m3x2_to_f16x2(lo); a[1] = e4m3x2_to_f16x2(hi);
+                                a[2] = e4m3x2_hi_to_f16x2(lo); a[3] = e4m3x2_hi_to_f16x2(hi);
+                            }
+                            MmaType<__half>::mma(h ? s2[j] : s[j], a, qb[i + h][0], qb[i + h][1]);
+                            if constexpr (SHARED) {
+                                if (two) MmaType<__half>::mma(h ? u2 : u, a, qc[i + h][0], qc[i + h][1]);
+                            }
                         }
                     }
                 }
@@ -805,24 +849,28 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                 for (int i = 0; i < Gm::KS; ++i) {
                     uint32_t a[4];
                     ldsm_x4(a, ks_s + Gm::addr(row, 2 * i + csel));
-                    MmaType<T>::mma((i & 1) ? s2 : s, a, qb[i][0], qb[i][1]);
+                    MmaType<T>::mma((i & 1) ? s2[0] : s[0], a, qb[i][0], qb[i][1]);
                     if constexpr (SHARED) {
                         if (two) MmaType<T>::mma((i & 1) ? u2 : u, a, qc[i][0], qc[i][1]);
                     }
                 }
             }
+            // s[j][0], s[j][1]: token 16j + g8, heads h0, h1; s[j][2], s[j][3]: token 16j + g8 + 8.
+            float x[NT][4];
+            float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) s[j] += s2[j];
-            // s[0], s[1]: token g8, heads h0, h1; s[2], s[3]: token g8 + 8.
-            const bool v_lo = g8 < valid, v_hi = g8 + 8 < valid;
-            float x0 = v_lo ? fmaf(s[0], uq, kc0) : -INFINITY;
-            float x1 = v_lo ? fmaf(s[1], uq, kc1) : -INFINITY;
-            float x2 = v_hi ? fmaf(s[2], uq, kc0) : -INFINITY;
-            float x3 = v_hi ? fmaf(s[3], uq, kc1) : -INFINITY;
-            bool raise = (hv0 && !(fmaxf(x0, x2) <= M0 + LAZY_MAX_LOG2)) ||
-                         (hv1 && !(fmaxf(x1, x3) <= M1 + LAZY_MAX_LOG2));
+            for (int j = 0; j < NT; ++j) {
+                const bool lo_in = 16 * j + g8 < valid, hi_in = 16 * j + g8 + 8 < valid;
+                x[j][0] = lo_in ? fmaf(s[j][0] + s2[j][0], uq, kc0) : -INFINITY;
+                x[j][1] = lo_in ? fmaf(s[j][1] + s2[j][1], uq, kc1) : -INFINITY;
+                x[j][2] = hi_in ? fmaf(s[j][2] + s2[j][2], uq, kc0) : -INFINITY;
+                x[j][3] = hi_in ? fmaf(s[j][3] + s2[j][3], uq, kc1) : -INFINITY;
+                mx0 = fmaxf(mx0, fmaxf(x[j][0], x[j][2]));
+                mx1 = fmaxf(mx1, fmaxf(x[j][1], x[j][3]));
+            }
+            bool raise = (hv0 && !(mx0 <= M0 + LAZY_MAX_LOG2)) || (hv1 && !(mx1 <= M1 + LAZY_MAX_LOG2));
             if (__any_sync(FULL_MASK, raise)) {
-                float m0 = fmaxf(x0, x2), m1 = fmaxf(x1, x3);
+                float m0 = mx0, m1 = mx1;
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) {
                     m0 = fmaxf(m0, __shfl_xor_sync(FULL_MASK, m0, off));
@@ -840,21 +888,25 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                     o[i][2] *= a0; o[i][3] *= a1;
                 }
             }
+            // P^T B fragments per sub-tile: head g8, tokens 2*t4 (+1) and 8 + 2*t4 (+1).
             // Padding heads (>= G) carry zero scores; give them weight 0.
-            const float p0 = hv0 ? exp2f(x0 - M0) : 0.f, p1 = hv1 ? exp2f(x1 - M1) : 0.f;
-            const float p2 = hv0 ? exp2f(x2 - M0) : 0.f, p3 = hv1 ? exp2f(x3 - M1) : 0.f;
-            const uint32_t w_lo = Elem<MT>::pack(p0, p1), w_hi = Elem<MT>::pack(p2, p3);
-            {
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const float p0 = hv0 ? exp2f(x[j][0] - M0) : 0.f, p1 = hv1 ? exp2f(x[j][1] - M1) : 0.f;
+                const float p2 = hv0 ? exp2f(x[j][2] - M0) : 0.f, p3 = hv1 ? exp2f(x[j][3] - M1) : 0.f;
+                const uint32_t w_lo = Elem<MT>::pack(p0, p1), w_hi = Elem<MT>::pack(p2, p3);
                 const float2 r_lo = Elem<MT>::pair(w_lo), r_hi = Elem<MT>::pair(w_hi);
                 l0 += r_lo.x + r_hi.x;
                 l1 += r_lo.y + r_hi.y;
+                pb[j][0] = movmatrix_trans(w_lo);
+                pb[j][1] = movmatrix_trans(w_hi);
             }
-            // P^T B fragments: head g8, tokens 2*t4 (+1) and 8 + 2*t4 (+1).
-            const uint32_t pb0 = movmatrix_trans(w_lo), pb1 = movmatrix_trans(w_hi);
             // The same for the second column half of a wide shared unit.
             uint32_t pc0 = 0u, pc1 = 0u;
             if constexpr (SHARED) {
                 if (two) {
+                    const bool v_lo = g8 < valid, v_hi = g8 + 8 < valid;
                     const float y0 = v_lo ? fmaf(u[0] + u2[0], uq, kd0) : -INFINITY;
                     const float y1 = v_lo ? fmaf(u[1] + u2[1], uq, kd1) : -INFINITY;
                     const float y2 = v_hi ? fmaf(u[2] + u2[2], uq, kd0) : -INFINITY;
@@ -893,11 +945,14 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
             }
 
             // ---------------- O^T += V^T . P^T ----------------------------------
-            if (valid < 16) {
-                // Stale or never-written slots past the context must not reach
-                // the product (their weight is 0 but 0 * NaN is NaN): zero them.
+            if (valid < TR) {
+                // Stale or never-written slots past the context in a loaded
+                // sub-tile must not reach the product (their weight is 0 but
+                // 0 * NaN is NaN): zero them. A sub-tile that was not loaded is
+                // not multiplied at all.
+                const int end = (valid + 15) & ~15;
                 uint8_t *vt = ring + stage * Gm::STAGE_BYTES + Gm::HALF_BYTES;
-                for (int idx = lane; idx < (16 - valid) * Gm::CHUNKS; idx += 32) {
+                for (int idx = lane; idx < (end - valid) * Gm::CHUNKS; idx += 32) {
                     const int r = valid + idx / Gm::CHUNKS;
                     const int c = idx % Gm::CHUNKS;
                     *reinterpret_cast<uint4 *>(vt + Gm::addr(r, c)) = make_uint4(0, 0, 0, 0);
@@ -913,27 +968,31 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                 const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
                 const int csel = lane >> 4;
 #pragma unroll
-                for (int i = 0; i < Gm::KS; i += 2) {
-                    uint32_t r[4];
-                    ldsm_x4_trans(r, vs_s + Gm::addr(row, i + csel));
+                for (int j = 0; j < NT; ++j) {
+                    if (j > 0 && valid <= 16 * j) break;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t a[4];
-                        if constexpr (I8) {
-                            // Bytes 0 / 2 are element 2*g8 of the two tokens, 1 / 3 element 2*g8+1.
-                            a[0] = i8_unbias(__byte_perm(r[2 * h], 0x64646464u, 0x4240));
-                            a[1] = i8_unbias(__byte_perm(r[2 * h], 0x64646464u, 0x4341));
-                            a[2] = i8_unbias(__byte_perm(r[2 * h + 1], 0x64646464u, 0x4240));
-                            a[3] = i8_unbias(__byte_perm(r[2 * h + 1], 0x64646464u, 0x4341));
-                        } else {
-                            const uint32_t x = __byte_perm(r[2 * h], 0, 0x3120);      // tokens 0-7
-                            const uint32_t y = __byte_perm(r[2 * h + 1], 0, 0x3120);  // tokens 8-15
-                            a[0] = e4m3x2_to_f16x2(x); a[1] = e4m3x2_hi_to_f16x2(x);
-                            a[2] = e4m3x2_to_f16x2(y); a[3] = e4m3x2_hi_to_f16x2(y);
-                        }
-                        MmaType<__half>::mma(o[i + h], a, pb0, pb1);
-                        if constexpr (SHARED) {
-                            if (two) MmaType<__half>::mma(o2[i + h], a, pc0, pc1);
+                    for (int i = 0; i < Gm::KS; i += 2) {
+                        uint32_t r[4];
+                        ldsm_x4_trans(r, vs_s + Gm::addr(16 * j + row, i + csel));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t a[4];
+                            if constexpr (I8) {
+                                // Bytes 0 / 2 are element 2*g8 of the two tokens, 1 / 3 element 2*g8+1.
+                                a[0] = i8_unbias(__byte_perm(r[2 * h], 0x64646464u, 0x4240));
+                                a[1] = i8_unbias(__byte_perm(r[2 * h], 0x64646464u, 0x4341));
+                                a[2] = i8_unbias(__byte_perm(r[2 * h + 1], 0x64646464u, 0x4240));
+                                a[3] = i8_unbias(__byte_perm(r[2 * h + 1], 0x64646464u, 0x4341));
+                            } else {
+                                const uint32_t x8 = __byte_perm(r[2 * h], 0, 0x3120);      // tokens 0-7
+                                const uint32_t y8 = __byte_perm(r[2 * h + 1], 0, 0x3120);  // tokens 8-15
+                                a[0] = e4m3x2_to_f16x2(x8); a[1] = e4m3x2_hi_to_f16x2(x8);
+                                a[2] = e4m3x2_to_f16x2(y8); a[3] = e4m3x2_hi_to_f16x2(y8);
+                            }
+                            MmaType<__half>::mma(o[i + h], a, pb[j][0], pb[j][1]);
+                            if constexpr (SHARED) {
+                                if (two) MmaType<__half>::mma(o2[i + h], a, pc0, pc1);
+                            }
                         }
                     }
                 }
@@ -944,7 +1003,7 @@ __global__ void __launch_bounds__(mma_max_warps<G, KV8, SHARED>() * 32, 1)
                 for (int i = 0; i < Gm::KS; ++i) {
                     uint32_t a[4];
                     ldsm_x4_trans(a, vs_s + Gm::addr(row, 2 * i + csel));
-                    MmaType<T>::mma(o[i], a, pb0, pb1);
+                    MmaType<T>::mma(o[i], a, pb[0][0], pb[0][1]);
                     if constexpr (SHARED) {
                         if (two) MmaType<T>::mma(o2[i], a, pc0, pc1);
                     }

@@ -221,7 +221,7 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     const CUtensorMapDataType type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : pa::MmaType<T>::tma_type;
     if ((st = encode_pool_map(&tmk, p.k_pool, rows, D, KV8 ? 1 : 2, type, info.dev)) != PA_OK) return st;
     if ((st = encode_pool_map(&tmv, p.v_pool, rows, D, KV8 ? 1 : 2, type, info.dev)) != PA_OK) return st;
-    constexpr int max_warps = pa::mma_max_warps<G, KV8, SHARED>();
+    constexpr int max_warps = pa::mma_max_warps<D, G, KV8, SHARED>();
     int warps = (info.smem_optin - 1024) / pa::mma_warp_bytes<D, G, NS, KV8, SHARED>();
     if (warps > max_warps) warps = max_warps;
     if (warps < 1) return fail(PA_ERR_UNSUPPORTED, "not enough shared memory for one warp");
