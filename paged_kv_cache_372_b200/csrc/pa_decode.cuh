@@ -71,7 +71,7 @@ struct DecodeParams {
     int *member_nparts;  // partitions of members[i] to merge (0: none, or written directly)
     int append_guard;    // 1: a sequence's last position never lies in a shared block
     int early;           // 1: the attention kernel starts without waiting for the one-warp plan
-    int reduce_launch;   // 1: split partitions merge in pa_reduce_kernel, a launch of their own
+    int reduce_launch;   // 1: a merge launch follows (long sequences; every sequence with shared units)
 };
 
 // Split merges: a (sequence, KV head) with more than MERGE_FANIN partitions

@@ -60,12 +60,13 @@ struct MmaGeo {
     static __device__ __forceinline__ uint32_t addr(int row, int chunk);
 };
 
-// Tokens per item (stage): 32 for the 8-bit kernels without shared units (two
+// Tokens per item (stage): 32 where a 16-token tile of K and V is at most
+// 4 KB (an 8-bit cache, or head_dim 64) and the units are not shared: two
 // 16-token MMA sub-tiles behind one wait, one softmax update and one issue,
-// which halves the per-token share of that fixed work), 16 otherwise.
-template <bool KV8, bool SHARED>
+// which halves the per-token share of that fixed work. 16 otherwise.
+template <int D, bool KV8, bool SHARED>
 __host__ __device__ constexpr int mma_tile_rows() {
-    return KV8 && !SHARED ? 32 : 16;
+    return !SHARED && (KV8 || D == 64) ? 32 : 16;
 }
 
 // Query rows of a unit shared by several sequences: two n8 column halves of
@@ -87,7 +88,7 @@ __host__ __device__ constexpr int mma_q_slots() {
 
 template <int D, int G, int NS, bool KV8 = false, bool SHARED = false>
 __host__ __device__ constexpr int mma_warp_bytes() {
-    return NS * MmaGeo<D, G, KV8, mma_tile_rows<KV8, SHARED>()>::STAGE_BYTES +
+    return NS * MmaGeo<D, G, KV8, mma_tile_rows<D, KV8, SHARED>()>::STAGE_BYTES +
            mma_q_slots<SHARED>() * mma_q_slot_bytes<D, G, SHARED>() + NS * 8;
 }
 
@@ -382,6 +383,16 @@ __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, s
 // out = sum_j 2^(m_j - M) acc_j / sum_j 2^(m_j - M) l_j.
 constexpr int REDUCE_GROUPS = 4;
 
+// Partitions above which a sequence's split merge runs in the merge launch
+// (pa_reduce_kernel, one CTA per (sequence, KV head), its partitions shared
+// by four thread groups) instead of in the attention kernel's last-arriving
+// warps; the launch happens when some sequence has more, and the others still
+// merge in the attention kernel. Measured: long32k with 64 partitions per
+// sequence 189.3 -> 178.1 us (fp8 cache 119.3 -> 107.9 us); llama3_8b, where
+// the few long sequences have up to 11, 146.2 -> 149.5 us with every merge
+// moved (the launch costs more than the merges it moves).
+constexpr int REDUCE_LAUNCH_MIN_PARTS = 16;
+
 // The merge launch of shared-prefix decode: a member has few partitions (its
 // shared ones and its own), so one warp merges one (grouping position, KV
 // head) with mma_merge, 8 per CTA; the sequence and its partition count come
@@ -417,7 +428,7 @@ __global__ void pa_reduce_kernel(const DecodeParams p) {
     } else {
         s = pos;
         nparts = (clamped_context(p, s, false) + p.partition - 1) / p.partition;
-        if (nparts <= 1) return;  // written by the attention kernel
+        if (nparts <= REDUCE_LAUNCH_MIN_PARTS) return;  // merged or written by the attention kernel
     }
     const size_t group = (size_t)s * p.num_kv_heads + kvh;
     const float2 *ml = p.ml + group * p.max_parts * G;
@@ -469,10 +480,13 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                          const __grid_constant__ CUtensorMap tm_v) {
     static_assert(!I8 || KV8, "INT8 codes are an 8-bit cache");
     static_assert(!HS || KV8, "per-head scales are an 8-bit cache's");
-    using Gm = MmaGeo<D, G, KV8, mma_tile_rows<KV8, SHARED>()>;
+    using Gm = MmaGeo<D, G, KV8, mma_tile_rows<D, KV8, SHARED>()>;
     constexpr int TR = Gm::TR;   // tokens of an item
     constexpr int NT = TR / 16;  // its 16-token MMA sub-tiles
     static_assert(!SHARED || NT == 1, "shared units keep 16-token items");
+    // The merge's two-pass form (no partials requested up front) where
+    // registers are scarce: the 8-bit kernels, and 8 query heads at head_dim 128.
+    constexpr bool LEAN_MERGE = KV8 || (G == 8 && D == 128);
     constexpr int QB = mma_q_slot_bytes<D, G, SHARED>();  // bytes of one query slot
     constexpr int QS = mma_q_slots<SHARED>();              // query slots per warp
     constexpr int QG = G * D * 2;                          // query rows of one sequence
@@ -846,12 +860,16 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                 const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
                 const int csel = lane >> 4;
 #pragma unroll
-                for (int i = 0; i < Gm::KS; ++i) {
-                    uint32_t a[4];
-                    ldsm_x4(a, ks_s + Gm::addr(row, 2 * i + csel));
-                    MmaType<T>::mma((i & 1) ? s2[0] : s[0], a, qb[i][0], qb[i][1]);
-                    if constexpr (SHARED) {
-                        if (two) MmaType<T>::mma((i & 1) ? u2 : u, a, qc[i][0], qc[i][1]);
+                for (int j = 0; j < NT; ++j) {
+                    if (j > 0 && valid <= 16 * j) break;
+#pragma unroll
+                    for (int i = 0; i < Gm::KS; ++i) {
+                        uint32_t a[4];
+                        ldsm_x4(a, ks_s + Gm::addr(16 * j + row, 2 * i + csel));
+                        MmaType<T>::mma((i & 1) ? s2[j] : s[j], a, qb[i][0], qb[i][1]);
+                        if constexpr (SHARED) {
+                            if (two) MmaType<T>::mma((i & 1) ? u2 : u, a, qc[i][0], qc[i][1]);
+                        }
                     }
                 }
             }
@@ -1000,12 +1018,16 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                 const int row = (lane & 7) + 8 * (lane >> 4);
                 const int csel = (lane >> 3) & 1;
 #pragma unroll
-                for (int i = 0; i < Gm::KS; ++i) {
-                    uint32_t a[4];
-                    ldsm_x4_trans(a, vs_s + Gm::addr(row, 2 * i + csel));
-                    MmaType<T>::mma(o[i], a, pb[0][0], pb[0][1]);
-                    if constexpr (SHARED) {
-                        if (two) MmaType<T>::mma(o2[i], a, pc0, pc1);
+                for (int j = 0; j < NT; ++j) {
+                    if (j > 0 && valid <= 16 * j) break;
+#pragma unroll
+                    for (int i = 0; i < Gm::KS; ++i) {
+                        uint32_t a[4];
+                        ldsm_x4_trans(a, vs_s + Gm::addr(16 * j + row, 2 * i + csel));
+                        MmaType<T>::mma(o[i], a, pb[j][0], pb[j][1]);
+                        if constexpr (SHARED) {
+                            if (two) MmaType<T>::mma(o2[i], a, pc0, pc1);
+                        }
                     }
                 }
             }
@@ -1080,7 +1102,7 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                 lm &= lm - 1;
                 const int sj = __shfl_sync(FULL_MASK, cur.mseq, j);
                 const int nj = __shfl_sync(FULL_MASK, cur.mnp, j);
-                mma_merge<D, G, T, KV8>(p, (size_t)sj * Hkv + cur.kvh, (size_t)sj * H + (size_t)cur.kvh * G, 0, nj,
+                mma_merge<D, G, T, LEAN_MERGE>(p, (size_t)sj * Hkv + cur.kvh, (size_t)sj * H + (size_t)cur.kvh * G, 0, nj,
                                         lane);
             }
         } else if (KV8 && cur.nparts == 1) {
@@ -1130,7 +1152,9 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
             }
             if (g8 == 0 && hv0) p.ml[row * G + h0] = make_float2(M0, l0);
             if (g8 == 0 && hv1) p.ml[row * G + h1] = make_float2(M1, l1);
-            if (p.reduce_launch) goto next_unit;  // merged by pa_reduce_kernel
+            // Merged by the merge launch: shared mode's every sequence, else
+            // the sequences with more than REDUCE_LAUNCH_MIN_PARTS partitions.
+            if (p.reduce_launch && (SHARED || cur.nparts > REDUCE_LAUNCH_MIN_PARTS)) goto next_unit;
             src.wait_plan();  // the merge counters are zeroed by the plan kernel
             // One level (at most MERGE_FANIN partitions, or shared-prefix units'
             // workspace), or two: this partition's chunk into its chunk
@@ -1153,7 +1177,7 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
             }
 #pragma unroll 1
             while (__shfl_sync(FULL_MASK, go, 0)) {
-                mma_merge<D, G, T, KV8>(p, group, head0, first, n, lane, dst);
+                mma_merge<D, G, T, LEAN_MERGE>(p, group, head0, first, n, lane, dst);
                 if (dst < 0) break;
                 go = count_partition(&p.merge_count[group], nch, lane == 0);
                 first = p.l1_base;

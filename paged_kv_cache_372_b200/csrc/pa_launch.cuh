@@ -24,13 +24,14 @@ enum class PartMode { plain, shared, fp8 };
 
 // With shared-prefix units (which always merge) 16 blocks for grouped heads:
 // the shared tiles are streamed once per group, so the remaining work is
-// spread better over the warps in smaller units. The fp8 kernel is
-// issue-bound rather than memory-bound and was measured best at 512 tokens
-// for one query head per KV head and at max(256 tokens, 8 blocks) otherwise.
+// spread better over the warps in smaller units. The 8-bit kernels: 512
+// tokens at every group size (measured on the Llama-3-8B-shaped batch: 84.8 us
+// against 93.8 at 256, whose longest sequences needed the merge launch; at
+// head_dim 64, 64.6 against 70.5 us on the LLaMA-7B-shaped batch).
 int auto_partition(int group, int block_size, PartMode mode = PartMode::plain) {
     switch (mode) {
         case PartMode::shared: return group >= 2 ? 16 * block_size : 256;
-        case PartMode::fp8: return group >= 2 ? (8 * block_size > 256 ? 8 * block_size : 256) : 512;
+        case PartMode::fp8: return 512;
         default: return group >= 2 ? 32 * block_size : 256;
     }
 }
@@ -192,14 +193,9 @@ pa_status encode_pool_map(CUtensorMap *map, const void *pool, long long rows, in
 // plan (each warp passes over the context lengths once or twice at start).
 constexpr int EARLY_MAX_SEQS = 512;
 
-// Partitions a sequence can have above which the split merge runs as its own
-// launch (pa_reduce_kernel, one CTA per (sequence, KV head), its partitions
-// shared by four thread groups) instead of in the attention kernel's
-// last-arriving warps. Measured: long32k with 64 partitions per sequence
-// 189.3 -> 178.1 us (fp8 cache 119.3 -> 107.9 us); llama3_8b, where the few
-// long sequences have up to 11, 146.2 -> 149.5 us (the launch costs more than
-// the merges it moves), so only above this many.
-constexpr int REDUCE_LAUNCH_MIN_PARTS = 16;
+// pa::REDUCE_LAUNCH_MIN_PARTS (the kernel header) decides which sequences'
+// split merges run in the merge launch.
+using pa::REDUCE_LAUNCH_MIN_PARTS;
 constexpr int REDUCE_SMEM_MAX = 200 * 1024;
 
 // Dynamic shared memory of pa_reduce_kernel<D, G>: the thread groups' sums and
@@ -238,8 +234,9 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
         ++g_launches;
     } else {
         p.early = p.num_seqs <= EARLY_MAX_SEQS;
-        // Many partitions per sequence: merge them in a launch of their own
-        // (while its (max, sum) pairs fit the reduce kernel's shared memory).
+        // Sequences with many partitions merge in a launch of their own (while
+        // its (max, sum) pairs fit the reduce kernel's shared memory), the
+        // others in the attention kernel.
         p.reduce_launch = p.l1_base > REDUCE_LAUNCH_MIN_PARTS && reduce_smem_bytes<D, G>(p.l1_base) <= REDUCE_SMEM_MAX;
         pa::pa_plan_kernel<<<1, pa::PLAN_WARP_THREADS, 0, stream>>>(p);
         ++g_launches;

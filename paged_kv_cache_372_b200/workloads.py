@@ -167,9 +167,11 @@ def tiny(seed: int = 0) -> Workload:
     return wl
 
 
-def _shape_name(base: str, block_size: int, head_dim: int) -> str:
-    """Name of a workload run at a block size / head size other than its own."""
-    return base if (block_size, head_dim) == (16, 128) else f"{base}_bs{block_size}_d{head_dim}"
+def _shape_name(base: str, block_size: int, head_dim: int, kv_heads: int | None = None) -> str:
+    """Name of a workload run at a block size / head size (/ KV head count)
+    other than its own."""
+    name = base if (block_size, head_dim) == (16, 128) else f"{base}_bs{block_size}_d{head_dim}"
+    return name if kv_heads is None else f"{name}_kv{kv_heads}"
 
 
 def llama7b(seed: int = 0, num_seqs: int = 64, block_size: int = 16, head_dim: int = 128) -> Workload:
@@ -180,11 +182,13 @@ def llama7b(seed: int = 0, num_seqs: int = 64, block_size: int = 16, head_dim: i
     return wl
 
 
-def llama3_8b(seed: int = 0, num_seqs: int = 256, block_size: int = 16, head_dim: int = 128) -> Workload:
+def llama3_8b(seed: int = 0, num_seqs: int = 256, block_size: int = 16, head_dim: int = 128,
+              kv_heads: int = 8) -> Workload:
     gen = inputs.generator(seed + 3000)
     ctx = inputs.lognormal_int(512.0, 1.0, 16, 8192, num_seqs, gen)
-    wl, _ = _decode_batch(_shape_name("llama3_8b", block_size, head_dim), ctx, heads=32, kv_heads=8,
-                          head_dim=head_dim, block_size=block_size, dtype="bf16", seed=seed + 3001)
+    wl, _ = _decode_batch(_shape_name("llama3_8b", block_size, head_dim, None if kv_heads == 8 else kv_heads), ctx,
+                          heads=32, kv_heads=kv_heads, head_dim=head_dim, block_size=block_size, dtype="bf16",
+                          seed=seed + 3001)
     return wl
 
 

@@ -52,14 +52,18 @@ def test_shared_decode_host_checks_without_a_device():
     parts = 2048 // 512
     assert shared >= plain + 64 * 32 * (8 + 128 * 4) + 64 * (parts + 1) * 16 + 2 * 64 * 4
     assert lib.pa_decode_shared_workspace_size(4, 2, 2, 96, 16, 33, 0) == 0
-    # fp8 cache: 512 tokens for one query head per KV head, max(256, 8 blocks) otherwise, head_dim 64 or 128
+    # 8-bit cache: 512 tokens at every group size, head_dim 64 or 128
     assert pa.pa_decode_fp8_partition_size(64, 32, 32, 128, 16, 2048, 0) == 512
-    assert pa.pa_decode_fp8_partition_size(256, 32, 8, 128, 16, 8192, 0) == 256
+    assert pa.pa_decode_fp8_partition_size(256, 32, 8, 128, 16, 8192, 0) == 512
     assert pa.pa_decode_fp8_partition_size(8, 32, 8, 128, 64, 32768, 0) == 512
-    assert pa.pa_decode_fp8_partition_size(8, 32, 8, 64, 16, 4096, 0) == 256
+    assert pa.pa_decode_fp8_partition_size(8, 32, 8, 64, 16, 4096, 0) == 512
+    assert pa.pa_decode_fp8_partition_size(8, 32, 8, 64, 32, 300, 0) == 320  # one partition
     assert pa.pa_decode_fp8_partition_size(8, 32, 8, 96, 16, 4096, 0) == 0
-    assert pa.pa_decode_fp8_workspace_size(256, 32, 8, 128, 16, 8192, 0) > pa.pa_decode_workspace_size(
+    # same partitions as pa_decode here (512 tokens), so the same workspace
+    assert pa.pa_decode_fp8_workspace_size(256, 32, 8, 128, 16, 8192, 0) == pa.pa_decode_workspace_size(
         256, 32, 8, 128, 16, 8192, 0)
+    assert 0 < pa.pa_decode_fp8_workspace_size(64, 32, 32, 128, 16, 2048, 0) < pa.pa_decode_workspace_size(
+        64, 32, 32, 128, 16, 2048, 0)  # 512 against 256 tokens at one head per KV head: fewer slots
     # shared-prefix units: 16 blocks for grouped heads, as pa_decode otherwise
     assert pa.pa_decode_shared_partition_size(4, 32, 8, 128, 16, 8192, 0) == 256
     assert pa.pa_decode_shared_partition_size(4, 32, 32, 128, 16, 8192, 0) == 256

@@ -38,11 +38,16 @@ def test_committed_traffic_matches_the_current_kernels():
 
 
 def test_shape_options_only_for_the_decode_batches():
-    args = types.SimpleNamespace(block_size=32, head_dim=None, workload="llama7b")
+    args = types.SimpleNamespace(block_size=32, head_dim=None, kv_heads=None, workload="llama7b")
     assert bench.shape_args(args) == {"block_size": 32}
-    args = types.SimpleNamespace(block_size=None, head_dim=64, workload="llama3_8b")
+    args = types.SimpleNamespace(block_size=None, head_dim=64, kv_heads=None, workload="llama3_8b")
     assert bench.shape_args(args) == {"head_dim": 64}
-    args = types.SimpleNamespace(block_size=32, head_dim=None, workload="beam")
+    args = types.SimpleNamespace(block_size=None, head_dim=None, kv_heads=4, workload="llama3_8b")
+    assert bench.shape_args(args) == {"kv_heads": 4}
+    from paged_kv_cache_372_b200 import workloads
+    wl = workloads.llama3_8b(0, num_seqs=4, kv_heads=4)
+    assert (wl.num_heads, wl.num_kv_heads, wl.name) == (32, 4, "llama3_8b_kv4")
+    args = types.SimpleNamespace(block_size=32, head_dim=None, kv_heads=None, workload="beam")
     try:
         bench.shape_args(args)
     except SystemExit:

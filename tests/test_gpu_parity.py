@@ -162,3 +162,17 @@ def test_launch_count(partition, launches):
     assert pa.pa_launch_count() - n0 == launches
     torch.cuda.synchronize()
     assert pa.pa_device_errors() == 0
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_merge_launch_beside_in_kernel_merges(dtype):
+    """One sequence with more than 16 partitions (merged in the merge launch)
+    next to sequences of 1, 2, 8, 9 and 16 partitions (written directly, merged
+    in one level and in two levels inside the attention kernel) in one call."""
+    P = 64
+    ctx = [40 * P + 5, 1, P, 2 * P - 3, 8 * P, 9 * P - 1, 16 * P, 17 * P, 3]
+    wl, _ = workloads._decode_batch("mixed_merges", ctx, heads=8, kv_heads=2, head_dim=128, block_size=16,
+                                    dtype=dtype, seed=77)
+    n0 = pa.pa_launch_count()
+    run_and_compare(wl, partition_size=P)
+    assert pa.pa_launch_count() - n0 == 4  # cache write, plan, attention, merge launch

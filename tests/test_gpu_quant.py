@@ -210,3 +210,19 @@ def test_quant_every_head_group(fmt, group, dtype, head_dim):
         err = float(np.abs(out.float().cpu().double().numpy() - ref).max())
         assert err <= TOL[dtype], (partition, err)
         margins.record(f"{fmt} per-head G={group} D={head_dim} {dtype} P={partition or 'auto'}", err, TOL[dtype])
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_quant_merge_launch_beside_in_kernel_merges(fmt):
+    """8-bit cache: one sequence past 16 partitions (merge launch) next to
+    sequences merged in the attention kernel or written directly."""
+    P = 64
+    ctx = [40 * P + 5, 1, P, 2 * P - 3, 8 * P, 9 * P - 1, 16 * P, 17 * P, 3]
+    wl, _ = workloads._decode_batch("mixed_merges", ctx, heads=8, kv_heads=2, head_dim=128, block_size=16,
+                                    dtype="bf16", seed=78)
+    k8, v8, ks, vs = quant_pools(wl, fmt)
+    out = run_decode(wl, fmt, k8, v8, ks, vs, P)
+    ref = oracle_decode(wl, fmt, k8, v8, ks, vs)
+    assert not torch.isnan(out).any()
+    err = float(np.abs(out.float().cpu().double().numpy() - ref).max())
+    assert err <= TOL[wl.dtype], err
