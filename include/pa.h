@@ -190,11 +190,14 @@ PA_API pa_status pa_decode_append(void *out, const void *q, const void *k_new, c
  * units balance better once the shared tiles are streamed once per group),
  * otherwise as pa_decode.
  *
- * Requirements beyond pa_decode's: num_seqs <= 1024, fp16/bf16 cache
- * (the tensor-core kernel). workspace: at least
- * pa_decode_shared_workspace_size(...) bytes (one more partition per
- * sequence than pa_decode, plus the grouping). Errors: PA_ERR_UNSUPPORTED
- * for num_seqs > 1024 or a build without the tensor-core kernel for this
+ * The grouping runs in one CTA of 1024 threads: a batch of more than 1024
+ * sequences runs as consecutive chunks of 1024 (in stream order, on the same
+ * workspace), and sequences share work only with others of their chunk.
+ *
+ * Requirements beyond pa_decode's: fp16/bf16 cache (the tensor-core kernel).
+ * workspace: at least pa_decode_shared_workspace_size(...) bytes (one more
+ * partition per sequence than pa_decode, plus the grouping). Errors:
+ * PA_ERR_UNSUPPORTED for a build without the tensor-core kernel for this
  * head group; otherwise as pa_decode / pa_decode_append.
  */
 PA_API pa_status pa_decode_shared(void *out, const void *q, const void *k_new, const void *v_new,

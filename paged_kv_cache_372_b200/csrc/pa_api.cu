@@ -174,9 +174,6 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     g_last_error.clear();
     if ((k_scales == nullptr) != (v_scales == nullptr) || (k_scales && (!aligned(k_scales, 4) || !aligned(v_scales, 4))))
         return fail(PA_ERR_INVALID, "k_scales and v_scales: both null or both 4-byte aligned device arrays");
-    if (shared && num_seqs > pa::SHARE_MAX_SEQS)
-        return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode takes at most %d sequences, got %d", pa::SHARE_MAX_SEQS,
-                    num_seqs);
     if (kv8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || k_scale == INFINITY || v_scale == INFINITY))
         return fail(PA_ERR_INVALID, "k_scale and v_scale must be positive and finite");
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 || partition_size < 0)
@@ -192,6 +189,25 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
         return fail(PA_ERR_INVALID, "misaligned pointer (16 B tensors, 4 B int arrays, 256 B workspace)");
+    if (shared && num_seqs > pa::SHARE_MAX_SEQS) {
+        // The grouping plan is one CTA: a larger batch runs as consecutive
+        // chunks of SHARE_MAX_SEQS sequences, in stream order on the same
+        // workspace; sequences share blocks' work only within their chunk.
+        const size_t es = 2;  // bytes of a q / out / k_new / v_new element
+        const size_t qrow = (size_t)num_heads * head_dim * es, kvrow = (size_t)num_kv_heads * head_dim * es;
+        for (int c0 = 0; c0 < num_seqs; c0 += pa::SHARE_MAX_SEQS) {
+            const int n = num_seqs - c0 < pa::SHARE_MAX_SEQS ? num_seqs - c0 : pa::SHARE_MAX_SEQS;
+            const pa_status st = decode_impl(
+                static_cast<uint8_t *>(out) + c0 * qrow, static_cast<const uint8_t *>(q) + c0 * qrow,
+                k_new ? static_cast<const uint8_t *>(k_new) + c0 * kvrow : nullptr,
+                v_new ? static_cast<const uint8_t *>(v_new) + c0 * kvrow : nullptr, k_pool, v_pool,
+                block_tables + (size_t)c0 * max_blocks_per_seq, context_lens + c0, n, num_heads, num_kv_heads,
+                head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale, dtype, partition_size,
+                workspace, workspace_bytes, stream, kv8, k_scale, v_scale, shared, int8, k_scales, v_scales);
+            if (st != PA_OK) return st;
+        }
+        return PA_OK;
+    }
     const int P = resolve_partition(num_heads / num_kv_heads, block_size, max_context_len, partition_size,
                                     shared ? PartMode::shared : kv8 ? PartMode::fp8 : PartMode::plain);
     if (P == 0)

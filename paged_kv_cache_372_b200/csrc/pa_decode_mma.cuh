@@ -108,10 +108,17 @@ __host__ __device__ constexpr int mma_smem_bytes(int warps) {
 // Shared-prefix units keep a second half of query columns (accumulators and
 // query fragments): 8 warps per CTA, so each thread has up to 255 registers.
 constexpr int SHARE_MAX_WARPS = 8;
+// 8 query heads per KV head at head_dim 128: a full 8-column MMA tile of
+// accumulators per slice; 8 warps per CTA give each thread 255 registers.
+#ifndef PA_G8_MAX_WARPS
+#define PA_G8_MAX_WARPS 8
+#endif
+constexpr int G8_MAX_WARPS = PA_G8_MAX_WARPS;
 template <int D, int G, bool KV8, bool SHARED = false>
 __host__ __device__ constexpr int mma_max_warps() {
     return SHARED ? SHARE_MAX_WARPS
-                  : KV8 && D == 64 && G <= PA_FP8_WIDE_MAX_GROUP ? DECODE_MAX_WARPS_FP8 : DECODE_MAX_WARPS;
+                  : KV8 && D == 64 && G <= PA_FP8_WIDE_MAX_GROUP ? DECODE_MAX_WARPS_FP8
+                  : G == 8 && D == 128 ? G8_MAX_WARPS : DECODE_MAX_WARPS;
 }
 
 // E4M3 -> f16 widening: every E4M3 value is exactly an f16. One cvt converts

@@ -74,17 +74,18 @@ def test_shared_decode_host_checks_without_a_device():
     rest = [32, 8, 128, 16, 64, 4096, 1024, ctypes.c_float(0.1), 0, 0, dummy, 1 << 30, None]
     # k_new without v_new
     assert lib.pa_decode_shared(dummy, dummy, dummy, None, *args[4:], 8, *rest) == pa.PA_ERR_INVALID
-    # more sequences than the grouping takes
-    assert lib.pa_decode_shared(*args, 1025, *rest) == pa.PA_ERR_UNSUPPORTED
-    assert b"1024" in lib.pa_last_error()
+    # more sequences than one grouping takes are chunked, after the argument checks
+    bad_dtype = rest[:8] + [7] + rest[9:]
+    assert lib.pa_decode_shared(*args, 1025, *bad_dtype) == pa.PA_ERR_INVALID
     # 8-bit cache: format, scale arrays, then the same limits
     qargs = [dummy, dummy, dummy, dummy, dummy, dummy]
     qrest = [32, 8, 128, 16, 64, 4096, 1024, ctypes.c_float(0.1), 0]
     tail = [0, dummy, 1 << 30, None]
     assert lib.pa_decode_shared_quant(*qargs, 8, *qrest, 7, dummy, dummy, *tail) == pa.PA_ERR_INVALID
     assert lib.pa_decode_shared_quant(*qargs, 8, *qrest, pa.PA_KV_INT8, None, dummy, *tail) == pa.PA_ERR_INVALID
-    assert lib.pa_decode_shared_quant(*qargs, 1025, *qrest, pa.PA_KV_E4M3, dummy, dummy, *tail) == \
-        pa.PA_ERR_UNSUPPORTED
+    qbad_dtype = qrest[:8] + [7]
+    assert lib.pa_decode_shared_quant(*qargs, 1025, *qbad_dtype, pa.PA_KV_E4M3, dummy, dummy, *tail) == \
+        pa.PA_ERR_INVALID
 
 
 def _header_declarations():

@@ -275,17 +275,37 @@ def test_without_sharing_equals_plain_decode():
         assert float((a.float() - b.float()).abs().max()) <= H.TOL[wl.dtype]
 
 
-def test_too_many_sequences_rejected():
-    dev = torch.device("cuda")
-    B = 1025
-    q = torch.zeros((B, 8, 64), dtype=torch.float16, device=dev)
-    kp = torch.zeros((4, 8, 16, 64), dtype=torch.float16, device=dev)
-    tab = torch.zeros((B, 1), dtype=torch.int32, device=dev)
-    ctx = torch.ones((B,), dtype=torch.int32, device=dev)
-    ws = torch.empty(1 << 20, dtype=torch.uint8, device=dev)
-    with pytest.raises(pa.PagedAttentionError) as e:
-        pa.pa_decode_shared(torch.empty_like(q), q, kp, kp.clone(), tab, ctx, 0.125, 1, 0, ws)
-    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+def test_more_sequences_than_one_grouping():
+    """1100 sequences (more than the grouping plan's 1024): the call runs as two
+    chunks, sharing within each, and matches the oracle and pa_decode."""
+    from paged_kv_cache_372_b200 import inputs
+    gen = inputs.generator(404)
+    B, heads, kvh, D, bs, NB = 1100, 8, 2, 64, 16, 2400
+    rng = np.random.default_rng(404)
+    perm = inputs.permutation(NB, gen)
+    tables = np.full((B, 3), -1, dtype=np.int32)
+    ctx = np.zeros(B, dtype=np.int32)
+    nxt = 0
+    for i in range(0, B, 2):  # pairs with one shared full block and a private second one
+        shared = perm[nxt]
+        nxt += 1
+        for j in (i, i + 1):
+            tables[j, 0] = shared
+            tables[j, 1] = perm[nxt]
+            nxt += 1
+            ctx[j] = bs + int(rng.integers(1, bs + 1))
+    case = dict(kp=inputs.normal((NB, kvh, bs, D), "f16", gen), vp=inputs.normal((NB, kvh, bs, D), "f16", gen),
+                q=inputs.normal((B, heads, D), "f16", gen), tables=tables, ctx=ctx, scale=D ** -0.5, dtype="f16",
+                bs=bs, heads=heads, kv_heads=kvh)
+    ref, _, _ = run_oracle(case, False)
+    n0 = pa.pa_launch_count()
+    out = run_shared(case, 0, False)[0]
+    assert pa.pa_launch_count() - n0 == 6  # per chunk: grouping plan, attention, merge launch
+    assert not torch.isnan(out).any()
+    err = H.max_err(out, ref)
+    assert err <= H.TOL["f16"], err
+    plain = run_plain(case, 0, False)[0]
+    assert float((plain.float() - out.float()).abs().max()) <= H.TOL["f16"]
 
 
 def whole_unit_case(group):
