@@ -112,6 +112,31 @@ def head_scales(n: int, base: float) -> torch.Tensor:
     return torch.tensor(s[order], dtype=torch.float32)
 
 
+def non_kv_bytes(wl, P: int, fused: bool, shared: bool) -> dict:
+    """Bytes a decode call moves besides the K/V rows of valid tokens, from the
+    workload's shapes (the mean over its steps): the query rows read and the
+    output rows written, the block-table entries and context lengths, the fp32
+    partials of split sequences (written by the attention kernel and read by
+    the merge: per partition and query head D floats and a (max, sum) pair;
+    with shared-prefix units one more partition per sequence, an upper bound),
+    and the new K/V rows the fused append reads and writes."""
+    H, Hkv, D, bs = wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
+    e = 2
+    acc = {"q_and_out": 0.0, "tables_and_contexts": 0.0, "partials": 0.0, "appended_rows": 0.0}
+    for st in wl.steps:
+        B = len(st.context_lens)
+        ctx = st.context_lens.astype(np.int64)
+        acc["q_and_out"] += 2 * B * H * D * e
+        acc["tables_and_contexts"] += 4 * int((-(-ctx // bs)).sum()) + 4 * B
+        nparts = -(-ctx // P) + (1 if shared else 0)
+        split = nparts[nparts > 1]
+        acc["partials"] += 2 * int(split.sum()) * H * (D * 4 + 8)
+        if fused:
+            acc["appended_rows"] += 2 * 2 * B * Hkv * D * e
+    n = len(wl.steps)
+    return {k: int(v / n) for k, v in acc.items()}
+
+
 def needs_flush(wl) -> bool:
     return wl.kv_bytes_unique() < 4 * L2_BYTES
 
@@ -473,6 +498,12 @@ def run_ours(args, world, rank, local, extras=True):
         "clocks": clk,
     }
     result["shared_prefix_units"] = bool(share)
+    B0, mx = wl.num_seqs, int(max(int(st.context_lens.max()) for st in wl.steps))
+    part_fn = (pa.pa_decode_shared_partition_size if share else pa.pa_decode_fp8_partition_size if kv8
+               else pa.pa_decode_partition_size)
+    P_used = part_fn(B0, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, mx, P)
+    result["non_kv_bytes_per_call"] = non_kv_bytes(wl, P_used, fused, share) if P_used > 0 else None
+    result["partition_size"] = P_used
     if unflushed is not None:
         unflushed["decode_kv_gbs"] = kv_unique / (unflushed["decode_ms"] * 1e-3) / 1e9
         unflushed["decode_kv_gbs_logical"] = kv_bytes / (unflushed["decode_ms"] * 1e-3) / 1e9

@@ -255,8 +255,7 @@ PA_API size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int n
  * query element above 65504 in magnitude has no fp16 value: the kernel sets
  * PA_DEVERR_QRANGE and that head's output is undefined). The
  * workspace is sized by pa_decode_fp8_workspace_size: partition_size 0 picks
- * 512 tokens for one query head per KV head and max(256 tokens, 8 blocks)
- * otherwise (pa_decode_fp8_partition_size).
+ * 512 tokens (pa_decode_fp8_partition_size).
  *
  * Defined by: "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
  * section 3.2 (内存压缩技术) — keep the KV cache in fewer bits to cut its

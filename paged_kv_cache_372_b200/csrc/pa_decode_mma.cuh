@@ -17,7 +17,7 @@
 // same rounded values.
 //
 // Variants (template flags): KV8 reads an 8-bit cache (byte tiles widened to
-// f16 in registers, 16 warps per CTA for head groups up to 4), I8 with INT8
+// f16 in registers, items of 32 tokens), I8 with INT8
 // codes, HS with one scale per KV head; SHARED lets a unit serve up to 16 / G
 // sequences that share the unit's blocks, their G query rows each filling
 // columns of two 8-column MMA tiles (pa_decode_shared, 8 warps per CTA).
@@ -256,7 +256,8 @@ __device__ __forceinline__ uint32_t MmaGeo<D, G, KV8, TR_>::addr(int row, int ch
 // dst_slot < 0 the result is normalised into the output rows; otherwise it is
 // written, unnormalised with its (max, sum), to partial slot dst_slot (a chunk
 // merge, see MERGE_FANIN).
-// LEAN (kernels under a 128-register cap) keeps fewer values live: the
+// LEAN (where registers are scarce: the 8-bit kernels, and 8 query heads at
+// head_dim 128) keeps fewer values live: the
 // (max, sum) pairs are read twice and no partials are loaded ahead.
 template <int D, int G, typename T, bool LEAN = false>
 __device__ __forceinline__ void mma_merge(const DecodeParams &p, size_t group, size_t head0, int first, int nparts,
@@ -1166,9 +1167,9 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
             // One level (at most MERGE_FANIN partitions, or shared-prefix units'
             // workspace), or two: this partition's chunk into its chunk
             // partial, then the chunk partials. One merge call site in a loop
-            // keeps the merge inlined once. The 8-bit kernels, under a
-            // 128-register cap, keep one level (beyond REDUCE_LAUNCH_MIN_PARTS
-            // partitions their merges run in the separate launch anyway).
+            // keeps the merge inlined once. The 8-bit kernels keep one level,
+            // for registers (beyond REDUCE_LAUNCH_MIN_PARTS partitions their
+            // merges run in the separate launch anyway).
             const bool chunked = !KV8 && cur.nparts > MERGE_FANIN && p.max_chunks > 0;
             const int nch = (cur.nparts + MERGE_FANIN - 1) / MERGE_FANIN;
             int first = 0, n = cur.nparts, dst = -1;

@@ -70,3 +70,21 @@ def test_cpu_baseline_and_reference_arm_time_the_same_sample():
     assert ref["impl"] == "reference" and ref["config"] == bench.describe(wl)
     n = min(wl.num_seqs, bench.ORACLE_SAMPLE_SEQS)
     assert cb["sample"].startswith(f"{n} of ") and ref["cpu_baseline"]["sample"].startswith(f"{n} of ")
+
+
+def test_non_kv_bytes_counts_each_part():
+    """q/out rows, table entries, split partials and appended rows, against a
+    count written out for the tiny workload (contexts 1, 7, 16, 33; H = Hkv = 2,
+    D = 64, bs = 16)."""
+    from paged_kv_cache_372_b200 import workloads
+    wl = workloads.tiny(0)
+    ctx = [int(c) for c in wl.steps[0].context_lens]
+    assert sorted(ctx) == [1, 7, 16, 33]
+    H, Hkv, D = 2, 2, 64
+    nb = bench.non_kv_bytes(wl, 16, fused=True, shared=False)
+    assert nb["q_and_out"] == 2 * 4 * H * D * 2
+    assert nb["tables_and_contexts"] == 4 * (1 + 1 + 1 + 3) + 4 * 4
+    assert nb["partials"] == 2 * 3 * H * (D * 4 + 8)  # only the 33-token sequence splits, into 3
+    assert nb["appended_rows"] == 2 * 2 * 4 * Hkv * D * 2
+    assert bench.non_kv_bytes(wl, 64, fused=False, shared=False)["partials"] == 0
+    assert bench.non_kv_bytes(wl, 64, fused=False, shared=False)["appended_rows"] == 0
