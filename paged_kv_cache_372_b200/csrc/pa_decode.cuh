@@ -1,24 +1,32 @@
-// Paged decode attention for sm_100a: two launches per call.
+// Paged decode attention for sm_100a: two launches per call (three when a
+// sequence has more partitions than the attention kernel merges itself).
 //
-//  1. pa_plan_kernel   (1 CTA) cuts every sequence into partitions of P tokens
-//     and writes the work list, longest partitions first, so that the
+//  1. pa_plan_kernel (one warp) cuts every sequence into partitions of P
+//     tokens and writes the work list: every sequence's full partitions in
+//     sequence order, then the partial last ones, longest first, so that the
 //     persistent attention kernel finishes with the short ones. It also
-//     zeroes the per-(sequence, KV head) merge counters.
-//     pa_plan_shared_kernel does the same for pa_decode_shared, after
-//     grouping sequences whose tables begin with the same blocks.
+//     zeroes the per-(sequence, KV head) merge counters. The attention warps
+//     take their first units without waiting for it (they derive them from
+//     the contexts). pa_plan_shared_kernel (one CTA) does the same for
+//     pa_decode_shared, after grouping sequences whose tables begin with the
+//     same blocks.
 //  2. The attention kernel (one persistent CTA per SM, launched with
-//     programmatic dependent launch so its set-up overlaps the plan) — every
+//     programmatic dependent launch so that it overlaps the plan) — every
 //     warp is an independent worker. It takes (sequence, KV head, partition)
 //     units from the work list with an atomic counter and streams the unit's
-//     16-token K and V tiles through a private ring of shared-memory stages
-//     filled by TMA copies that complete on mbarriers. The block-table
-//     entries of a unit are loaded once into lane registers and handed to
-//     the copy-issuing lane by a shuffle. Per tile: scores of the G query
-//     heads of the KV head, online softmax, weighted sum of the values. A
-//     unit that is a whole sequence writes the normalised output; otherwise
-//     it writes (max, sum, unnormalised output) partials, and the last warp
-//     to finish a (sequence, KV head) merges its partitions by the
-//     log-sum-exp identity.
+//     K and V tiles (16 tokens, or 32 where a 16-token tile is at most 4 KB)
+//     through a private ring of shared-memory stages filled by TMA copies
+//     that complete on mbarriers. The block-table entries of a unit are
+//     loaded once into lane registers and handed to the copy-issuing lane by
+//     a shuffle. Per tile: scores of the G query heads of the KV head, online
+//     softmax, weighted sum of the values. A unit that is a whole sequence
+//     writes the normalised output; otherwise it writes (max, sum,
+//     unnormalised output) partials, and the last warp to finish a (sequence,
+//     KV head) merges its partitions by the log-sum-exp identity, in one
+//     level or two (chunks of MERGE_FANIN).
+//  3. The merge launch (pa_reduce_kernel, or pa_reduce_members_kernel for
+//     shared-prefix decode) merges the sequences of many partitions (every
+//     sequence in shared-prefix decode) after the attention kernel.
 //     The default attention kernel is the tensor-core one in
 //     pa_decode_mma.cuh. This file holds the CUDA-core kernel
 //     (pa_decode_kernel: 1-D bulk copies of each tile, FFMA2 dot products),

@@ -16,11 +16,14 @@
 // input type for the second product and the softmax denominator sums the
 // same rounded values.
 //
+// An item (one ring stage) is one such tile, or two (32 tokens) where a
+// 16-token tile is at most 4 KB (mma_tile_rows).
+//
 // Variants (template flags): KV8 reads an 8-bit cache (byte tiles widened to
-// f16 in registers, items of 32 tokens), I8 with INT8
-// codes, HS with one scale per KV head; SHARED lets a unit serve up to 16 / G
-// sequences that share the unit's blocks, their G query rows each filling
-// columns of two 8-column MMA tiles (pa_decode_shared, 8 warps per CTA).
+// f16 in registers), I8 with INT8 codes, HS with one scale per KV head;
+// SHARED lets a unit serve up to 16 / G sequences that share the unit's
+// blocks, their G query rows each filling columns of two 8-column MMA tiles
+// (pa_decode_shared and pa_decode_shared_quant, 8 warps per CTA).
 #pragma once
 
 #include <cuda.h>
@@ -32,9 +35,9 @@
 
 namespace pa {
 
-// KV8: the pools hold E4M3 (fp8) codes, one byte per element, dequantised
-// with per-tensor scales (k_scale folded into the score scale, v_scale into
-// the output scale).
+// KV8: the pools hold 8-bit codes (E4M3, or INT8 with I8), one byte per
+// element, dequantised with per-tensor or (HS) per-KV-head scales: the key
+// scale folded into the score scale, the value scale into the output scale.
 //
 // A tile row is D * EB bytes: 256 or 128 (loaded in 128-byte boxes with the
 // 128-byte swizzle) or 64 (an 8-bit cache at head_dim 64: one 64-byte box
