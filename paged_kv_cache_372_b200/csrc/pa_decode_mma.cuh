@@ -421,26 +421,16 @@ __global__ void __launch_bounds__(256) pa_reduce_members_kernel(const DecodePara
                        lane);
 }
 
-// SM (shared-prefix decode): CTA = (grouping position, KV head); the
-// sequence and its partition count come from the grouping plan's members /
-// member_nparts.
-template <int D, int G, typename T, bool SM = false>
+// CTA = (sequence, KV head).
+template <int D, int G, typename T>
 __global__ void pa_reduce_kernel(const DecodeParams p) {
     constexpr int V4 = D * G / 4;
     extern __shared__ float4 s_red[];  // [REDUCE_GROUPS][V4] sums, [REDUCE_GROUPS][V4] weight sums, (max, sum)s
     float2 *s_ml = reinterpret_cast<float2 *>(s_red + 2 * REDUCE_GROUPS * V4);  // [nparts][G]
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int pos = blockIdx.x / p.num_kv_heads, kvh = blockIdx.x - pos * p.num_kv_heads;
-    int s, nparts;
-    if constexpr (SM) {
-        s = p.members[pos];
-        nparts = p.member_nparts[pos];
-        if (nparts < 1) return;  // empty, or written by the attention kernel (member_nparts 0)
-    } else {
-        s = pos;
-        nparts = (clamped_context(p, s, false) + p.partition - 1) / p.partition;
-        if (nparts <= REDUCE_LAUNCH_MIN_PARTS) return;  // merged or written by the attention kernel
-    }
+    const int s = blockIdx.x / p.num_kv_heads, kvh = blockIdx.x - s * p.num_kv_heads;
+    const int nparts = (clamped_context(p, s, false) + p.partition - 1) / p.partition;
+    if (nparts <= REDUCE_LAUNCH_MIN_PARTS) return;  // merged or written by the attention kernel
     const size_t group = (size_t)s * p.num_kv_heads + kvh;
     const float2 *ml = p.ml + group * p.max_parts * G;
     for (int i = threadIdx.x; i < nparts * G; i += blockDim.x) s_ml[i] = __ldcg(ml + i);
