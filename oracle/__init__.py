@@ -95,6 +95,10 @@ class Oracle:
                                                  ctypes.c_double, _I, _I, _P, _P, _I]
         L.oracle_reshape_and_cache_kv8.restype = None
         L.oracle_reshape_and_cache_kv8.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
+        L.oracle_paged_attention_kv8_blocks.restype = None
+        L.oracle_paged_attention_kv8_blocks.argtypes = L.oracle_paged_attention_kv8.argtypes
+        L.oracle_reshape_and_cache_kv8_blocks.restype = None
+        L.oracle_reshape_and_cache_kv8_blocks.argtypes = L.oracle_reshape_and_cache_kv8.argtypes
         L.oracle_slot_mapping.restype = None
         L.oracle_slot_mapping.argtypes = [_P, _P, _I, _P, _P, _I, _I]
 
@@ -167,7 +171,8 @@ class Oracle:
     def paged_attention_kv8(self, q, k_pool, v_pool, block_tables, context_lens, scale, q_dtype, kv_format,
                             k_scales, v_scales, num_threads: int = 0) -> np.ndarray:
         """out[s][h][:] in fp64 over an 8-bit cache (uint8 codes; kv_format "e4m3" or
-        "int8") with one scale per KV head (k_scales, v_scales: [num_kv_heads])."""
+        "int8") with one scale per KV head (k_scales, v_scales: [num_kv_heads]) or
+        one per (physical block, KV head) ([num_blocks][num_kv_heads])."""
         q = np.ascontiguousarray(q, dtype=np.uint16)
         k_pool = np.ascontiguousarray(k_pool, dtype=np.uint8)
         v_pool = np.ascontiguousarray(v_pool, dtype=np.uint8)
@@ -178,7 +183,8 @@ class Oracle:
         assert D2 == D and v_pool.shape == k_pool.shape and H % Hkv == 0
         ks = np.ascontiguousarray(k_scales, dtype=np.float64)
         vs = np.ascontiguousarray(v_scales, dtype=np.float64)
-        assert ks.shape == (Hkv,) and vs.shape == (Hkv,)
+        per_block = ks.ndim == 2
+        assert ks.shape == vs.shape and ks.shape in ((Hkv,), (NB, Hkv))
         for s in range(B):
             n = int(context_lens[s])
             pages = -(-n // bs)
@@ -187,7 +193,8 @@ class Oracle:
                 used = block_tables[s, :pages]
                 assert used.min() >= 0 and used.max() < NB
         out = np.zeros((B, H, D), dtype=np.float64)
-        self.lib.oracle_paged_attention_kv8(
+        fn = self.lib.oracle_paged_attention_kv8_blocks if per_block else self.lib.oracle_paged_attention_kv8
+        fn(
             _ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), _ptr(context_lens),
             B, H, Hkv, D, bs, block_tables.shape[1], float(scale), dtype_code(q_dtype), KV_FORMATS[kv_format],
             _ptr(ks), _ptr(vs), int(num_threads))
@@ -195,7 +202,9 @@ class Oracle:
 
     def reshape_and_cache_kv8(self, k, v, k_pool, v_pool, slot_mapping, dtype, kv_format, k_scales,
                               v_scales) -> None:
-        """In place on uint8 pools: code = encode(x / scale[h]) in fp32, per KV head h."""
+        """In place on uint8 pools: code = encode(x / scale) in fp32, the scale of
+        KV head h ([num_kv_heads] arrays) or of (the slot's block, h)
+        ([num_blocks][num_kv_heads])."""
         for a in (k_pool, v_pool):
             assert a.dtype == np.uint8 and a.flags.c_contiguous
         k = np.ascontiguousarray(k, dtype=np.uint16)
@@ -207,10 +216,11 @@ class Oracle:
         assert slot_mapping.max(initial=-1) < NB * bs
         ks = np.ascontiguousarray(k_scales, dtype=np.float32)
         vs = np.ascontiguousarray(v_scales, dtype=np.float32)
-        assert ks.shape == (Hkv,) and vs.shape == (Hkv,)
-        self.lib.oracle_reshape_and_cache_kv8(_ptr(k), _ptr(v), _ptr(k_pool), _ptr(v_pool), _ptr(slot_mapping),
-                                              T, Hkv, D, bs, dtype_code(dtype), KV_FORMATS[kv_format], _ptr(ks),
-                                              _ptr(vs))
+        per_block = ks.ndim == 2
+        assert ks.shape == vs.shape and ks.shape in ((Hkv,), (NB, Hkv))
+        fn = self.lib.oracle_reshape_and_cache_kv8_blocks if per_block else self.lib.oracle_reshape_and_cache_kv8
+        fn(_ptr(k), _ptr(v), _ptr(k_pool), _ptr(v_pool), _ptr(slot_mapping), T, Hkv, D, bs, dtype_code(dtype),
+           KV_FORMATS[kv_format], _ptr(ks), _ptr(vs))
 
     def max_threads(self) -> int:
         return int(self.lib.oracle_max_threads())

@@ -30,6 +30,9 @@
  *  - The scale is an argument (the configurations pass 1/sqrt(head_dim)).
  *  - Grouped-query attention: query head h reads KV head h / (H / H_kv).
  *  - context_len == 0 gives a zero output row.
+ *  - 8-bit caches (section 3.2 of the first page, 内存压缩技术): one scale per
+ *    tensor, per KV head, or per (physical block, KV head); a block's scale
+ *    applies to every token written into that block.
  *
  * Element formats: fp16 is IEEE 754 binary16; bf16 is the upper half of an
  * IEEE 754 binary32. Both are decoded here from their bit fields.
@@ -376,6 +379,24 @@ static double kv8_to_double(uint8_t code, int format)
 }
 
 /*
+ * The scale of KV head kvh of physical block `page`: one per (block, KV head)
+ * ([num_blocks][num_kv_heads] arrays) when per_block, else one per KV head.
+ */
+static double kv8_scale(const double *scales, int per_block, size_t page, int kvh, int num_kv_heads)
+{
+    return per_block ? scales[page * (size_t)num_kv_heads + kvh] : scales[kvh];
+}
+
+static void paged_attention_kv8(double *out, const uint16_t *q,
+                                const uint8_t *k_pool, const uint8_t *v_pool,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int num_heads, int num_kv_heads,
+                                int head_dim, int block_size, int max_blocks_per_seq,
+                                double scale, int q_dtype, int format,
+                                const double *k_scales, const double *v_scales, int per_block,
+                                int num_threads);
+
+/*
  * Paged decode attention over an 8-bit KV cache (E4M3 or INT8 codes) with one
  * scale per KV head: key element of KV head j = k_scales[j] * decode(code),
  * value element = v_scales[j] * decode(code). Otherwise the computation of
@@ -389,6 +410,38 @@ void oracle_paged_attention_kv8(double *out, const uint16_t *q,
                                 double scale, int q_dtype, int format,
                                 const double *k_scales, const double *v_scales, int num_threads)
 {
+    paged_attention_kv8(out, q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads, num_kv_heads,
+                        head_dim, block_size, max_blocks_per_seq, scale, q_dtype, format, k_scales, v_scales, 0,
+                        num_threads);
+}
+
+/*
+ * The same with one scale per (physical block, KV head): the key element of KV
+ * head j in block b = k_scales[b * num_kv_heads + j] * decode(code), the value
+ * element likewise with v_scales.
+ */
+void oracle_paged_attention_kv8_blocks(double *out, const uint16_t *q,
+                                       const uint8_t *k_pool, const uint8_t *v_pool,
+                                       const int32_t *block_tables, const int32_t *context_lens,
+                                       int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_dim, int block_size, int max_blocks_per_seq,
+                                       double scale, int q_dtype, int format,
+                                       const double *k_scales, const double *v_scales, int num_threads)
+{
+    paged_attention_kv8(out, q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads, num_kv_heads,
+                        head_dim, block_size, max_blocks_per_seq, scale, q_dtype, format, k_scales, v_scales, 1,
+                        num_threads);
+}
+
+static void paged_attention_kv8(double *out, const uint16_t *q,
+                                const uint8_t *k_pool, const uint8_t *v_pool,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int num_heads, int num_kv_heads,
+                                int head_dim, int block_size, int max_blocks_per_seq,
+                                double scale, int q_dtype, int format,
+                                const double *k_scales, const double *v_scales, int per_block,
+                                int num_threads)
+{
     const int group = num_heads / num_kv_heads;
     const long pairs = (long)num_seqs * num_heads;
 #ifdef _OPENMP
@@ -401,7 +454,6 @@ void oracle_paged_attention_kv8(double *out, const uint16_t *q,
         const int h = (int)(sh % num_heads);
         const int kvh = h / group;
         const int n = context_lens[s];
-        const double ks = k_scales[kvh], vs = v_scales[kvh];
         double *o = out + (size_t)sh * head_dim;
         for (int d = 0; d < head_dim; d++)
             o[d] = 0.0;
@@ -415,6 +467,7 @@ void oracle_paged_attention_kv8(double *out, const uint16_t *q,
         const int32_t *table = block_tables + (size_t)s * max_blocks_per_seq;
         for (int i = 0; i < pages; i++) {
             const size_t page = (size_t)table[i];
+            const double ks = kv8_scale(k_scales, per_block, page, kvh, num_kv_heads);
             for (int r = 0; r < block_size; r++) {
                 const int t = i * block_size + r;
                 if (t >= n)
@@ -439,6 +492,7 @@ void oracle_paged_attention_kv8(double *out, const uint16_t *q,
             scores[t] /= total;
         for (int i = 0; i < pages; i++) {
             const size_t page = (size_t)table[i];
+            const double vs = kv8_scale(v_scales, per_block, page, kvh, num_kv_heads);
             for (int r = 0; r < block_size; r++) {
                 const int t = i * block_size + r;
                 if (t >= n)
@@ -453,6 +507,11 @@ void oracle_paged_attention_kv8(double *out, const uint16_t *q,
     }
 }
 
+static void reshape_and_cache_kv8(const uint16_t *k, const uint16_t *v, uint8_t *k_pool, uint8_t *v_pool,
+                                  const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                  int block_size, int dtype, int format, const float *k_scales,
+                                  const float *v_scales, int per_block);
+
 /*
  * Quantising cache write with one scale per KV head: element x of head h is
  * stored as encode(x / k_scales[h]) (keys) or encode(x / v_scales[h])
@@ -464,6 +523,29 @@ void oracle_reshape_and_cache_kv8(const uint16_t *k, const uint16_t *v,
                                   int num_kv_heads, int head_dim, int block_size,
                                   int dtype, int format, const float *k_scales, const float *v_scales)
 {
+    reshape_and_cache_kv8(k, v, k_pool, v_pool, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size, dtype,
+                          format, k_scales, v_scales, 0);
+}
+
+/*
+ * The same with one scale per (physical block, KV head): a token written into
+ * block b divides by k_scales[b * num_kv_heads + h] (v_scales for values).
+ */
+void oracle_reshape_and_cache_kv8_blocks(const uint16_t *k, const uint16_t *v,
+                                         uint8_t *k_pool, uint8_t *v_pool,
+                                         const int64_t *slot_mapping, int num_tokens,
+                                         int num_kv_heads, int head_dim, int block_size,
+                                         int dtype, int format, const float *k_scales, const float *v_scales)
+{
+    reshape_and_cache_kv8(k, v, k_pool, v_pool, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size, dtype,
+                          format, k_scales, v_scales, 1);
+}
+
+static void reshape_and_cache_kv8(const uint16_t *k, const uint16_t *v, uint8_t *k_pool, uint8_t *v_pool,
+                                  const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                  int block_size, int dtype, int format, const float *k_scales,
+                                  const float *v_scales, int per_block)
+{
     for (int t = 0; t < num_tokens; t++) {
         const int64_t slot = slot_mapping[t];
         if (slot < 0)
@@ -473,9 +555,10 @@ void oracle_reshape_and_cache_kv8(const uint16_t *k, const uint16_t *v,
         for (int h = 0; h < num_kv_heads; h++) {
             const size_t src = ((size_t)t * num_kv_heads + h) * head_dim;
             const size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) * head_dim;
+            const size_t si = per_block ? (size_t)block * num_kv_heads + h : (size_t)h;
             for (int d = 0; d < head_dim; d++) {
-                const float kx = (float)oracle_to_double(k[src + d], dtype) / k_scales[h];
-                const float vx = (float)oracle_to_double(v[src + d], dtype) / v_scales[h];
+                const float kx = (float)oracle_to_double(k[src + d], dtype) / k_scales[si];
+                const float vx = (float)oracle_to_double(v[src + d], dtype) / v_scales[si];
                 k_pool[dst + d] = format == ORACLE_KV_INT8 ? oracle_int8_encode(kx) : oracle_e4m3_encode(kx);
                 v_pool[dst + d] = format == ORACLE_KV_INT8 ? oracle_int8_encode(vx) : oracle_e4m3_encode(vx);
             }

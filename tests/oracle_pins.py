@@ -461,6 +461,59 @@ def pin_kv8_cache_write(orc, seed=18):
             assert np.array_equal(kp, ek) and np.array_equal(vp, ev), (fmt, dt)
 
 
+def _block_scales(rng, NB, Hkv, base):
+    """[NB][Hkv] scales spanning up to 100x around `base`."""
+    return base * 10.0 ** rng.uniform(-1.0, 1.0, (NB, Hkv))
+
+
+def pin_kv8_blocks_attention_bruteforce(orc, seed=19):
+    """Attention over an 8-bit cache with one scale per (physical block, KV
+    head) = the brute force over the cache dequantised by numpy, block by
+    block (each element times the scale of its own block and head)."""
+    rng = np.random.default_rng(seed)
+    for fmt in ("e4m3", "int8"):
+        for B, H, Hkv, D, bs, ctx, dt in SHAPES:
+            q, k8, v8, tab, cl = _fp8_case(rng, B, H, Hkv, D, bs, ctx, dt)
+            NB = k8.shape[0]
+            ks, vs = _block_scales(rng, NB, Hkv, 0.05), _block_scales(rng, NB, Hkv, 0.05)
+            got = orc.paged_attention_kv8(q, k8, v8, tab, cl, 1.0 / math.sqrt(D), dt, fmt, ks, vs)
+            kd = _dequant_kv8(k8, fmt, np.ones(Hkv)) * ks[:, :, None, None]
+            vd = _dequant_kv8(v8, fmt, np.ones(Hkv)) * vs[:, :, None, None]
+            ref = contiguous_attention(decode(q, dt), kd, vd, tab, cl, 1.0 / math.sqrt(D))
+            assert np.abs(got - ref).max() <= ATOL * max(1.0, np.abs(ref).max()), (fmt, B, H, Hkv)
+
+
+def pin_kv8_blocks_cache_write(orc, seed=20):
+    """Quantising write with one scale per (block, KV head): code =
+    encode(x / scale[block of the slot][h]) with the division in float32."""
+    rng = np.random.default_rng(seed)
+    NB, Hkv, bs, D, T = 6, 3, 16, 32, 40
+    for fmt in ("e4m3", "int8"):
+        for dt in ("f16", "bf16"):
+            k = _rand_bits(rng, (T, Hkv, D), dt)
+            v = _rand_bits(rng, (T, Hkv, D), dt)
+            kp = rng.integers(0, 256, (NB, Hkv, bs, D), dtype=np.uint8)
+            vp = rng.integers(0, 256, (NB, Hkv, bs, D), dtype=np.uint8)
+            slots = rng.choice(NB * bs, T, replace=False).astype(np.int64)
+            slots[5] = -1
+            ks = _block_scales(rng, NB, Hkv, 0.02).astype(np.float32)
+            vs = _block_scales(rng, NB, Hkv, 0.02).astype(np.float32)
+            ek, ev = kp.copy(), vp.copy()
+            for t in range(T):
+                if slots[t] < 0:
+                    continue
+                b, o = int(slots[t]) // bs, int(slots[t]) % bs
+                for pool, x, sc in ((ek, k, ks), (ev, v, vs)):
+                    y = (decode(x[t], dt).astype(np.float32) / sc[b][:, None]).astype(np.float32)
+                    if fmt == "e4m3":
+                        codes = _torch_e4m3_codes(np.clip(y, -448, 448))
+                    else:
+                        codes = (np.clip(np.rint(y), -127, 127).astype(np.int64) + 128).astype(np.uint8)
+                    pool[b, :, o, :] = codes
+            orc.reshape_and_cache_kv8(k, v, kp, vp, slots, dt, fmt, ks, vs)
+            assert np.array_equal(kp, ek) and np.array_equal(vp, ev), (fmt, dt)
+
+
 def pin_slot_mapping(orc, seed=10):
     rng = np.random.default_rng(seed)
     bs, B, W = 16, 5, 6
@@ -481,4 +534,5 @@ ALL_PINS = [pin_decode_f16, pin_decode_bf16, pin_bruteforce, pin_sdpa, pin_rando
             pin_shared_equals_duplicated, pin_tail_slots_ignored, pin_gqa_mapping,
             pin_empty_context, pin_reshape_and_cache, pin_copy_blocks, pin_swap_blocks, pin_slot_mapping,
             pin_e4m3_decode, pin_e4m3_encode, pin_fp8_attention_bruteforce, pin_fp8_cache_write,
-            pin_int8_codes, pin_kv8_attention_bruteforce, pin_kv8_cache_write]
+            pin_int8_codes, pin_kv8_attention_bruteforce, pin_kv8_cache_write,
+            pin_kv8_blocks_attention_bruteforce, pin_kv8_blocks_cache_write]

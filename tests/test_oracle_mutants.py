@@ -56,11 +56,17 @@ MUTATIONS = {
     "int8_excess_127": ("return (double)code - 128.0;", "return (double)code - 127.0;"),
     "int8_ties_away": ("if (f > 0.5 || (f == 0.5 && fmod(r, 2.0) != 0.0))", "if (f >= 0.5)"),
     "int8_clamps_at_minus_128": ("if (y <= -127.0f)\n        return 1;", "if (y <= -127.0f)\n        return 0;"),
-    "kv8_scale_of_query_head": ("const double ks = k_scales[kvh], vs = v_scales[kvh];",
-                                "const double ks = k_scales[h % num_kv_heads], vs = v_scales[h % num_kv_heads];"),
-    "kv8_scales_swapped": ("const double ks = k_scales[kvh], vs = v_scales[kvh];",
-                           "const double ks = v_scales[kvh], vs = k_scales[kvh];"),
-    "kv8_write_scale_of_head_0": ("/ k_scales[h];", "/ k_scales[0];"),
+    "kv8_scale_of_query_head": ("const double ks = kv8_scale(k_scales, per_block, page, kvh, num_kv_heads);",
+                                "const double ks = kv8_scale(k_scales, per_block, page, h % num_kv_heads, "
+                                "num_kv_heads);"),
+    "kv8_scales_swapped": ("const double ks = kv8_scale(k_scales, per_block, page, kvh, num_kv_heads);",
+                           "const double ks = kv8_scale(v_scales, per_block, page, kvh, num_kv_heads);"),
+    "kv8_write_scale_of_head_0": ("/ k_scales[si];", "/ k_scales[0];"),
+    "kv8_block_scale_of_head": ("return per_block ? scales[page * (size_t)num_kv_heads + kvh] : scales[kvh];",
+                                "return per_block ? scales[kvh] : scales[kvh];"),
+    "kv8_write_block_scale_of_head": (
+        "const size_t si = per_block ? (size_t)block * num_kv_heads + h : (size_t)h;",
+        "const size_t si = (size_t)h;"),
     "kv8_format_ignored": (
         "return format == ORACLE_KV_INT8 ? oracle_int8_to_double(code) : oracle_e4m3_to_double(code);",
         "return oracle_e4m3_to_double(code);"),
