@@ -328,6 +328,38 @@ PA_API pa_status pa_decode_quant(void *out, const void *q, const void *k_pool, c
                                  int kv_format, const float *k_scales, const float *v_scales, int partition_size,
                                  void *workspace, size_t workspace_bytes, pa_stream_t stream);
 
+/*
+ * The 8-bit cache with one scale per (physical block, KV head): k_scales and
+ * v_scales are fp32 device arrays [num_blocks][num_kv_heads], 4-byte aligned;
+ * a token written into block b of KV head h is stored as
+ * encode(x / k_scales[b * num_kv_heads + h]) (v_scales for values), and
+ * decoding multiplies by the same scale. Otherwise exactly
+ * pa_reshape_and_cache_quant / pa_decode_quant (same codes, layouts,
+ * partition, workspace and errors). A block's scale applies to every token
+ * written into it, so it has to be chosen before its first token is written
+ * (a serving loop sets it when it allocates the block, e.g. from prefill
+ * statistics). The decode reads each unit's block scales beside its
+ * block-table entries; the value product weighs each token by its block's
+ * value scale relative to the unit's largest, and the denominator sums the
+ * unweighted fp32 probabilities.
+ *
+ * Defined by: "别再让GPU内存拖后腿了：vLLM的PagedAttention如何像操作系统一样管理KV Cache",
+ * section 3.2 (内存压缩技术), keep the cache in fewer bits, with the scales at the
+ * granularity of the cache's own unit, the physical block of section 2.1.
+ */
+PA_API pa_status pa_reshape_and_cache_quant_blocks(const void *k, const void *v, void *k_pool, void *v_pool,
+                                                   const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                                                   int head_dim, int block_size, int num_blocks, int dtype,
+                                                   int kv_format, const float *k_scales, const float *v_scales,
+                                                   pa_stream_t stream);
+PA_API pa_status pa_decode_quant_blocks(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                        const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                        int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                        int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                                        int dtype, int kv_format, const float *k_scales, const float *v_scales,
+                                        int partition_size, void *workspace, size_t workspace_bytes,
+                                        pa_stream_t stream);
+
 /* Workspace bytes pa_decode needs for these sizes (0 if the shape is invalid). */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
                                 int head_dim, int block_size, int max_context_len,

@@ -89,9 +89,13 @@ def lib() -> ctypes.CDLL:
         L.pa_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _P]
         L.pa_reshape_and_cache_quant.restype = _I
         L.pa_reshape_and_cache_quant.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.pa_reshape_and_cache_quant_blocks.restype = _I
+        L.pa_reshape_and_cache_quant_blocks.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.pa_decode_quant_blocks.restype = _I
         L.pa_decode_quant.restype = _I
         L.pa_decode_quant.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P,
                                       _I, _P, _SZ, _P]
+        L.pa_decode_quant_blocks.argtypes = L.pa_decode_quant.argtypes
         L.pa_decode_shared_quant.restype = _I
         L.pa_decode_shared_quant.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                                              _P, _P, _I, _P, _SZ, _P]
@@ -309,9 +313,11 @@ def pa_reshape_and_cache_fp8(k, v, k_pool, v_pool, slot_mapping, k_scale, v_scal
 KV_FORMATS = {"e4m3": PA_KV_E4M3, "int8": PA_KV_INT8}
 
 
-def _scales(t, name, n):
-    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != (n,):
-        raise ValueError(f"{name} must be a float32 CUDA tensor of shape [num_kv_heads]")
+def _scales(t, name, n, blocks=None):
+    shape = (n,) if blocks is None else (blocks, n)
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != shape:
+        what = "[num_kv_heads]" if blocks is None else "[num_blocks][num_kv_heads]"
+        raise ValueError(f"{name} must be a float32 CUDA tensor of shape {what}")
     return _cuda(t, name)
 
 
@@ -351,6 +357,47 @@ def pa_decode_quant(out, q, k_pool, v_pool, block_tables, context_lens, scale, m
         _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
         B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
         KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv), _scales(v_scales, "v_scales", Hkv),
+        int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return out
+
+
+def pa_reshape_and_cache_quant_blocks(k, v, k_pool, v_pool, slot_mapping, kv_format, k_scales, v_scales,
+                                      stream=None) -> None:
+    """pa_reshape_and_cache_quant with one scale per (physical block, KV head):
+    k_scales, v_scales float32 CUDA tensors [NB][Hkv]."""
+    T, Hkv, D = k.shape
+    NB, Hkv2, bs, D2 = k_pool.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(v.shape) != tuple(k.shape) or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("shape mismatch between k, v and the pools")
+    if k.dtype not in _DTYPES or v.dtype != k.dtype or k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("k, v fp16/bf16; pools uint8")
+    _check(lib().pa_reshape_and_cache_quant_blocks(
+        _cuda(k, "k"), _cuda(v, "v"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, bs, NB, _DTYPES[k.dtype],
+        KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv, NB), _scales(v_scales, "v_scales", Hkv, NB),
+        _stream(stream)))
+
+
+def pa_decode_quant_blocks(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len, kv_format,
+                           k_scales, v_scales, partition_size=0, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode_quant with one scale per (physical block, KV head): k_scales,
+    v_scales float32 CUDA tensors [NB][Hkv]."""
+    B, H, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch between q, out and the pools")
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("8-bit pools must be uint8 tensors of codes")
+    if q.dtype not in _DTYPES or out.dtype != q.dtype:
+        raise ValueError("q and out must share one dtype, fp16 or bf16")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device, fp8=True)
+    _check(lib().pa_decode_quant_blocks(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
+        B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
+        KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv, NB), _scales(v_scales, "v_scales", Hkv, NB),
         int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream)))
     return out

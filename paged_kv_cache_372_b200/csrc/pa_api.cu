@@ -164,13 +164,23 @@ size_t pa_decode_shared_workspace_size(int num_seqs, int num_heads, int num_kv_h
 
 namespace {
 
+// 8-bit cache kernels by code format and scale granularity.
+template <int D, typename T>
+pa_status dispatch_kv8(pa::DecodeParams &p, int group, cudaStream_t s, bool int8, int hs) {
+    if (int8)
+        return hs == 2 ? dispatch_group_fp8<D, T, true, 2>(p, group, s) : dispatch_group_fp8<D, T, true, 1>(p, group, s);
+    return hs == 2   ? dispatch_group_fp8<D, T, false, 2>(p, group, s)
+           : hs == 1 ? dispatch_group_fp8<D, T, false, 1>(p, group, s)
+                     : dispatch_group_fp8<D, T, false, 0>(p, group, s);
+}
+
 pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v_new, const void *k_pool,
                       const void *v_pool, const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                       int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
                       int num_blocks, int max_context_len, float scale, int dtype, int partition_size,
                       void *workspace, size_t workspace_bytes, pa_stream_t stream, bool kv8 = false,
                       float k_scale = 1.f, float v_scale = 1.f, bool shared = false, bool int8 = false,
-                      const float *k_scales = nullptr, const float *v_scales = nullptr) {
+                      const float *k_scales = nullptr, const float *v_scales = nullptr, bool block_scales = false) {
     g_last_error.clear();
     if ((k_scales == nullptr) != (v_scales == nullptr) || (k_scales && (!aligned(k_scales, 4) || !aligned(v_scales, 4))))
         return fail(PA_ERR_INVALID, "k_scales and v_scales: both null or both 4-byte aligned device arrays");
@@ -203,7 +213,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
                 v_new ? static_cast<const uint8_t *>(v_new) + c0 * kvrow : nullptr, k_pool, v_pool,
                 block_tables + (size_t)c0 * max_blocks_per_seq, context_lens + c0, n, num_heads, num_kv_heads,
                 head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale, dtype, partition_size,
-                workspace, workspace_bytes, stream, kv8, k_scale, v_scale, shared, int8, k_scales, v_scales);
+                workspace, workspace_bytes, stream, kv8, k_scale, v_scale, shared, int8, k_scales, v_scales,
+                block_scales);
             if (st != PA_OK) return st;
         }
         return PA_OK;
@@ -282,21 +293,13 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
                            : dispatch_group_shared_kv8<64, __nv_bfloat16, false>(p, group, s));
     }
     if (kv8) {
-        const bool d128 = head_dim == 128, f16 = dtype == PA_F16;
-        if (int8)
-            return d128 ? (f16 ? dispatch_group_fp8<128, __half, true, true>(p, group, s)
-                               : dispatch_group_fp8<128, __nv_bfloat16, true, true>(p, group, s))
-                        : (f16 ? dispatch_group_fp8<64, __half, true, true>(p, group, s)
-                               : dispatch_group_fp8<64, __nv_bfloat16, true, true>(p, group, s));
-        if (k_scales)
-            return d128 ? (f16 ? dispatch_group_fp8<128, __half, false, true>(p, group, s)
-                               : dispatch_group_fp8<128, __nv_bfloat16, false, true>(p, group, s))
-                        : (f16 ? dispatch_group_fp8<64, __half, false, true>(p, group, s)
-                               : dispatch_group_fp8<64, __nv_bfloat16, false, true>(p, group, s));
-        return d128 ? (f16 ? dispatch_group_fp8<128, __half>(p, group, s)
-                           : dispatch_group_fp8<128, __nv_bfloat16>(p, group, s))
-                    : (f16 ? dispatch_group_fp8<64, __half>(p, group, s)
-                           : dispatch_group_fp8<64, __nv_bfloat16>(p, group, s));
+        // Scales: per (block, KV head) 2, per KV head 1, per tensor 0 (E4M3 only).
+        const int hs = block_scales ? 2 : k_scales ? 1 : 0;
+        if (head_dim == 128)
+            return dtype == PA_F16 ? dispatch_kv8<128, __half>(p, group, s, int8, hs)
+                                   : dispatch_kv8<128, __nv_bfloat16>(p, group, s, int8, hs);
+        return dtype == PA_F16 ? dispatch_kv8<64, __half>(p, group, s, int8, hs)
+                               : dispatch_kv8<64, __nv_bfloat16>(p, group, s, int8, hs);
     }
     if (shared) {
         if (head_dim == 128)
@@ -418,7 +421,7 @@ namespace {
 pa_status reshape_kv8_impl(const void *k, const void *v, void *k_pool, void *v_pool, const int64_t *slot_mapping,
                            int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                            bool int8, float k_scale, float v_scale, const float *k_scales, const float *v_scales,
-                           pa_stream_t stream) {
+                           pa_stream_t stream, bool scales_per_block = false) {
     DeviceInfo info;
     pa_status st = device_info(&info);
     if (st != PA_OK) return st;
@@ -433,7 +436,7 @@ pa_status reshape_kv8_impl(const void *k, const void *v, void *k_pool, void *v_p
                                                  static_cast<uint2 *>(k_pool), static_cast<uint2 *>(v_pool),
                                                  slot_mapping, total, vec_per_row, num_kv_heads, block_size,
                                                  (long long)num_blocks * block_size, k_scale, v_scale, k_scales,
-                                                 v_scales);
+                                                 v_scales, scales_per_block ? 1 : 0);
     };
     if (dtype == PA_F16)
         int8 ? launch(pa::pa_reshape_kv8_kernel<__half, true>) : launch(pa::pa_reshape_kv8_kernel<__half, false>);
@@ -469,10 +472,33 @@ pa_status pa_reshape_and_cache_fp8(const void *k, const void *v, void *k_pool, v
                             num_blocks, dtype, false, k_scale, v_scale, nullptr, nullptr, stream);
 }
 
+static pa_status reshape_quant_checked(const void *k, const void *v, void *k_pool, void *v_pool,
+                                       const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                       int block_size, int num_blocks, int dtype, int kv_format,
+                                       const float *k_scales, const float *v_scales, pa_stream_t stream,
+                                       bool scales_per_block);
+
 pa_status pa_reshape_and_cache_quant(const void *k, const void *v, void *k_pool, void *v_pool,
                                      const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
                                      int block_size, int num_blocks, int dtype, int kv_format, const float *k_scales,
                                      const float *v_scales, pa_stream_t stream) {
+    return reshape_quant_checked(k, v, k_pool, v_pool, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                                 num_blocks, dtype, kv_format, k_scales, v_scales, stream, false);
+}
+
+pa_status pa_reshape_and_cache_quant_blocks(const void *k, const void *v, void *k_pool, void *v_pool,
+                                            const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                                            int head_dim, int block_size, int num_blocks, int dtype, int kv_format,
+                                            const float *k_scales, const float *v_scales, pa_stream_t stream) {
+    return reshape_quant_checked(k, v, k_pool, v_pool, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                                 num_blocks, dtype, kv_format, k_scales, v_scales, stream, true);
+}
+
+static pa_status reshape_quant_checked(const void *k, const void *v, void *k_pool, void *v_pool,
+                                       const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                       int block_size, int num_blocks, int dtype, int kv_format,
+                                       const float *k_scales, const float *v_scales, pa_stream_t stream,
+                                       bool scales_per_block) {
     g_last_error.clear();
     if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return fail(PA_ERR_INVALID, "size argument");
     if (dtype != PA_F16 && dtype != PA_BF16) return fail(PA_ERR_INVALID, "dtype %d", dtype);
@@ -487,7 +513,8 @@ pa_status pa_reshape_and_cache_quant(const void *k, const void *v, void *k_pool,
         !aligned(slot_mapping, 8) || !aligned(k_scales, 4) || !aligned(v_scales, 4))
         return fail(PA_ERR_INVALID, "misaligned pointer");
     return reshape_kv8_impl(k, v, k_pool, v_pool, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
-                            num_blocks, dtype, kv_format == PA_KV_INT8, 1.f, 1.f, k_scales, v_scales, stream);
+                            num_blocks, dtype, kv_format == PA_KV_INT8, 1.f, 1.f, k_scales, v_scales, stream,
+                            scales_per_block);
 }
 
 pa_status pa_decode_quant(void *out, const void *q, const void *k_pool, const void *v_pool,
@@ -503,6 +530,21 @@ pa_status pa_decode_quant(void *out, const void *q, const void *k_pool, const vo
                        num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
                        dtype, partition_size, workspace, workspace_bytes, stream, true, 1.f, 1.f, false,
                        kv_format == PA_KV_INT8, k_scales, v_scales);
+}
+
+pa_status pa_decode_quant_blocks(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                 const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                 int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, int dtype,
+                                 int kv_format, const float *k_scales, const float *v_scales, int partition_size,
+                                 void *workspace, size_t workspace_bytes, pa_stream_t stream) {
+    g_last_error.clear();
+    if (kv_format != PA_KV_E4M3 && kv_format != PA_KV_INT8) return fail(PA_ERR_INVALID, "kv_format %d", kv_format);
+    if (num_seqs > 0 && (!k_scales || !v_scales)) return fail(PA_ERR_INVALID, "null scale array");
+    return decode_impl(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream, true, 1.f, 1.f, false,
+                       kv_format == PA_KV_INT8, k_scales, v_scales, true);
 }
 
 pa_status pa_copy_blocks(void *const *pools, int num_pools, const int64_t *src_dst_pairs, int num_pairs,

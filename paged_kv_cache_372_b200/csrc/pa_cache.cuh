@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(256) pa_reshape_kv8_kernel(const uint4 *__rest
                                                              int num_kv_heads, int block_size, long long num_slots,
                                                              float k_scale, float v_scale,
                                                              const float *__restrict__ k_scales,
-                                                             const float *__restrict__ v_scales) {
+                                                             const float *__restrict__ v_scales,
+                                                             int scales_per_block) {
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vectors; i += stride) {
         const long long row = i / vec_per_row;
@@ -85,7 +86,9 @@ __global__ void __launch_bounds__(256) pa_reshape_kv8_kernel(const uint4 *__rest
         const int64_t off = slot - blk * block_size;
         const size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * vec_per_row + vec;
         const uint4 src[2] = {k[i], v[i]};
-        const float sc[2] = {k_scales ? k_scales[h] : k_scale, v_scales ? v_scales[h] : v_scale};
+        // One scale per KV head, or per (block, KV head) with scales_per_block.
+        const size_t si = scales_per_block ? (size_t)blk * num_kv_heads + h : (size_t)h;
+        const float sc[2] = {k_scales ? k_scales[si] : k_scale, v_scales ? v_scales[si] : v_scale};
         uint2 codes[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {

@@ -20,7 +20,8 @@
 // 16-token tile is at most 4 KB (mma_tile_rows).
 //
 // Variants (template flags): KV8 reads an 8-bit cache (byte tiles widened to
-// f16 in registers), I8 with INT8 codes, HS with one scale per KV head;
+// f16 in registers), I8 with INT8 codes, HS the scales' granularity (0: one
+// per tensor, 1: one per KV head, 2: one per (physical block, KV head));
 // SHARED lets a unit serve up to 16 / G sequences that share the unit's
 // blocks, their G query rows each filling columns of two 8-column MMA tiles
 // (pa_decode_shared and pa_decode_shared_quant, 8 warps per CTA).
@@ -475,12 +476,13 @@ __global__ void pa_reduce_kernel(const DecodeParams p) {
     }
 }
 
-template <int D, int G, typename T, int NS, bool KV8 = false, bool SHARED = false, bool I8 = false, bool HS = false>
+template <int D, int G, typename T, int NS, bool KV8 = false, bool SHARED = false, bool I8 = false, int HS = 0>
 __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
     pa_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
     static_assert(!I8 || KV8, "INT8 codes are an 8-bit cache");
-    static_assert(!HS || KV8, "per-head scales are an 8-bit cache's");
+    static_assert(!HS || KV8, "per-head and per-block scales are an 8-bit cache's");
+    static_assert(HS != 2 || !SHARED, "per-block scales: units of one sequence");
     using Gm = MmaGeo<D, G, KV8, mma_tile_rows<D, KV8, SHARED>()>;
     constexpr int TR = Gm::TR;   // tokens of an item
     constexpr int NT = TR / 16;  // its 16-token MMA sub-tiles
@@ -709,12 +711,29 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
         const bool app_unit = append && cur.part == cur.nparts - 1;
         // Dequantisation of an 8-bit cache: the key scale folds into the
         // score scale uq, the value scale uv applies at the store (per unit
-        // with per-head scales, HS; kernel parameters otherwise). kc0 / kc1
-        // take the INT8 offset off the scores of query rows h0 / h1.
+        // with per-head scales, HS == 1; kernel parameters otherwise). kc0 /
+        // kc1 take the INT8 offset off the scores of query rows h0 / h1.
+        // Per-block scales (HS == 2): lane j holds the scales of the unit's
+        // block j (the table slice it holds); a sub-tile's key scale joins uq
+        // and the INT8 offsets, its value scale, relative to the unit's
+        // largest (uv), weights the probabilities of the value product.
         float uq = p.qscale, uv = p.v_scale, kc0 = 0.f, kc1 = 0.f, kd0 = 0.f, kd1 = 0.f;
-        if constexpr (HS) {
+        float kbl = 1.f, vbl = 1.f, ivmax = 1.f;
+        if constexpr (HS == 1) {
             uq = p.qscale * __ldg(p.k_scales + cur.kvh);
             uv = __ldg(p.v_scales + cur.kvh);
+        } else if constexpr (HS == 2) {
+            float vmax = 0.f;
+            if (lane < (cur.ntok + bs - 1) / bs && (unsigned)cur.tbl < (unsigned)p.num_blocks) {
+                const size_t si = (size_t)cur.tbl * Hkv + cur.kvh;
+                kbl = __ldg(p.k_scales + si);
+                vbl = __ldg(p.v_scales + si);
+                vmax = vbl;
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(FULL_MASK, vmax, off));
+            uv = vmax;
+            ivmax = vmax > 0.f ? 1.f / vmax : 0.f;
         }
         uint4 newrow = make_uint4(0, 0, 0, 0);
         if (app_unit && lane < 2 * NVR) {
@@ -875,15 +894,25 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                 }
             }
             // s[j][0], s[j][1]: token 16j + g8, heads h0, h1; s[j][2], s[j][3]: token 16j + g8 + 8.
-            float x[NT][4];
+            float x[NT][4], vr[NT];
             float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
+                float uqj = uq, kcj0 = kc0, kcj1 = kc1;
+                vr[j] = 1.f;
+                if constexpr (HS == 2) {  // the scales of the sub-tile's block
+                    const int bj = (TR * k + 16 * j) / bs;
+                    const float ksc = __shfl_sync(FULL_MASK, kbl, bj & 31);
+                    vr[j] = __shfl_sync(FULL_MASK, vbl, bj & 31) * ivmax;
+                    uqj = uq * ksc;
+                    kcj0 = kc0 * ksc;
+                    kcj1 = kc1 * ksc;
+                }
                 const bool lo_in = 16 * j + g8 < valid, hi_in = 16 * j + g8 + 8 < valid;
-                x[j][0] = lo_in ? fmaf(s[j][0] + s2[j][0], uq, kc0) : -INFINITY;
-                x[j][1] = lo_in ? fmaf(s[j][1] + s2[j][1], uq, kc1) : -INFINITY;
-                x[j][2] = hi_in ? fmaf(s[j][2] + s2[j][2], uq, kc0) : -INFINITY;
-                x[j][3] = hi_in ? fmaf(s[j][3] + s2[j][3], uq, kc1) : -INFINITY;
+                x[j][0] = lo_in ? fmaf(s[j][0] + s2[j][0], uqj, kcj0) : -INFINITY;
+                x[j][1] = lo_in ? fmaf(s[j][1] + s2[j][1], uqj, kcj1) : -INFINITY;
+                x[j][2] = hi_in ? fmaf(s[j][2] + s2[j][2], uqj, kcj0) : -INFINITY;
+                x[j][3] = hi_in ? fmaf(s[j][3] + s2[j][3], uqj, kcj1) : -INFINITY;
                 mx0 = fmaxf(mx0, fmaxf(x[j][0], x[j][2]));
                 mx1 = fmaxf(mx1, fmaxf(x[j][1], x[j][3]));
             }
@@ -914,10 +943,21 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
             for (int j = 0; j < NT; ++j) {
                 const float p0 = hv0 ? exp2f(x[j][0] - M0) : 0.f, p1 = hv1 ? exp2f(x[j][1] - M1) : 0.f;
                 const float p2 = hv0 ? exp2f(x[j][2] - M0) : 0.f, p3 = hv1 ? exp2f(x[j][3] - M1) : 0.f;
-                const uint32_t w_lo = Elem<MT>::pack(p0, p1), w_hi = Elem<MT>::pack(p2, p3);
-                const float2 r_lo = Elem<MT>::pair(w_lo), r_hi = Elem<MT>::pair(w_hi);
-                l0 += r_lo.x + r_hi.x;
-                l1 += r_lo.y + r_hi.y;
+                uint32_t w_lo, w_hi;
+                if constexpr (HS == 2) {
+                    // The value product weighs each token by its block's value
+                    // scale (relative to uv); the denominator sums the weights.
+                    w_lo = Elem<MT>::pack(p0 * vr[j], p1 * vr[j]);
+                    w_hi = Elem<MT>::pack(p2 * vr[j], p3 * vr[j]);
+                    l0 += p0 + p2;
+                    l1 += p1 + p3;
+                } else {
+                    w_lo = Elem<MT>::pack(p0, p1);
+                    w_hi = Elem<MT>::pack(p2, p3);
+                    const float2 r_lo = Elem<MT>::pair(w_lo), r_hi = Elem<MT>::pair(w_hi);
+                    l0 += r_lo.x + r_hi.x;
+                    l1 += r_lo.y + r_hi.y;
+                }
                 pb[j][0] = movmatrix_trans(w_lo);
                 pb[j][1] = movmatrix_trans(w_hi);
             }

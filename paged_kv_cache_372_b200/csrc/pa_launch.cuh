@@ -205,7 +205,7 @@ size_t reduce_smem_bytes(int parts) {
     return 2 * pa::REDUCE_GROUPS * (D * G / 4) * 16 + (size_t)parts * G * 8;
 }
 
-template <int D, int G, typename T, bool KV8 = false, bool SHARED = false, bool I8 = false, bool HS = false>
+template <int D, int G, typename T, bool KV8 = false, bool SHARED = false, bool I8 = false, int HS = 0>
 pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     constexpr int NS = KV8 ? pa::DECODE_MMA_STAGES_FP8 : pa::DECODE_MMA_STAGES;
     DeviceInfo info;
@@ -282,9 +282,10 @@ pa_status launch_decode_mma(pa::DecodeParams &p, cudaStream_t stream) {
     return PA_OK;
 }
 
-// 8-bit cache (E4M3, or INT8 with I8; per-head scales with HS): tensor-core
+// 8-bit cache (E4M3, or INT8 with I8; HS: scales per tensor 0, per KV head 1,
+// per (block, KV head) 2): tensor-core
 // kernel, head_dim 64 or 128.
-template <int D, typename T, bool I8 = false, bool HS = false>
+template <int D, typename T, bool I8 = false, int HS = 0>
 pa_status dispatch_group_fp8(pa::DecodeParams &p, int group, cudaStream_t stream) {
     switch (group) {
         case 1: return launch_decode_mma<D, 1, T, true, false, I8, HS>(p, stream);
@@ -313,10 +314,10 @@ pa_status dispatch_group_shared(pa::DecodeParams &p, int group, cudaStream_t str
 template <int D, typename T, bool I8>
 pa_status dispatch_group_shared_kv8(pa::DecodeParams &p, int group, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_decode_mma<D, 1, T, true, true, I8, true>(p, stream);
-        case 2: return launch_decode_mma<D, 2, T, true, true, I8, true>(p, stream);
-        case 4: return launch_decode_mma<D, 4, T, true, true, I8, true>(p, stream);
-        case 8: return launch_decode_mma<D, 8, T, true, true, I8, true>(p, stream);
+        case 1: return launch_decode_mma<D, 1, T, true, true, I8, 1>(p, stream);
+        case 2: return launch_decode_mma<D, 2, T, true, true, I8, 1>(p, stream);
+        case 4: return launch_decode_mma<D, 4, T, true, true, I8, 1>(p, stream);
+        case 8: return launch_decode_mma<D, 8, T, true, true, I8, 1>(p, stream);
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }
