@@ -48,10 +48,12 @@ def parse():
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition", type=int, default=None)
-    ap.add_argument("--kv", default="auto", choices=["auto", "fp8", "e4m3h", "int8"],
+    ap.add_argument("--kv", default="auto", choices=["auto", "fp8", "e4m3h", "int8", "e4m3b", "int8b"],
                     help="fp8: E4M3 KV cache, one scale per tensor (pa_reshape_and_cache_fp8 + pa_decode_fp8); "
                          "e4m3h / int8: E4M3 / INT8 codes with one scale per KV head, spanning 100x "
-                         "(pa_reshape_and_cache_quant + pa_decode_quant)")
+                         "(pa_reshape_and_cache_quant + pa_decode_quant); e4m3b / int8b: one scale per "
+                         "(block, KV head), spanning 100x (pa_reshape_and_cache_quant_blocks + "
+                         "pa_decode_quant_blocks)")
     ap.add_argument("--unfused", action="store_true",
                     help="separate cache-write launch instead of pa_decode_append")
     ap.add_argument("--share", default="auto", choices=["auto", "on", "off"],
@@ -103,6 +105,12 @@ def describe(wl) -> dict:
 L2_BYTES = 126 * 1024 * 1024
 FP8_SCALE = 0.0375  # N(0,1) values / 0.0375 stay well inside E4M3's +-448
 INT8_SCALE = 0.035  # about max |N(0,1)| / 127 over a pool
+
+
+def block_scales(nb: int, n: int, base: float, seed: int) -> torch.Tensor:
+    """Per-(block, KV head) scales from base / 10 to base * 10, seeded."""
+    g = torch.Generator().manual_seed(seed)
+    return (base * 10.0 ** (2.0 * torch.rand((nb, n), generator=g, dtype=torch.float64) - 1.0)).float()
 
 
 def head_scales(n: int, base: float) -> torch.Tensor:
@@ -323,18 +331,24 @@ def run_ours(args, world, rank, local, extras=True):
         flush_w.fill_(i & 0xff)
         flush_r.sum()
 
-    kv8 = args.kv in ("fp8", "e4m3h", "int8")
-    quant = args.kv in ("e4m3h", "int8")
-    qfmt = {"e4m3h": "e4m3", "int8": "int8"}.get(args.kv)
+    kv8 = args.kv in ("fp8", "e4m3h", "int8", "e4m3b", "int8b")
+    quant = args.kv in ("e4m3h", "int8", "e4m3b", "int8b")
+    per_block = args.kv in ("e4m3b", "int8b")
+    qfmt = {"e4m3h": "e4m3", "int8": "int8", "e4m3b": "e4m3", "int8b": "int8"}.get(args.kv)
     if quant:
         base = INT8_SCALE if qfmt == "int8" else FP8_SCALE
-        ksc = head_scales(wl.num_kv_heads, base).to(dev)
-        vsc = head_scales(wl.num_kv_heads, base).flip(0).contiguous().to(dev)
+        if per_block:
+            ksc = block_scales(kp.shape[0], wl.num_kv_heads, base, args.seed + 61).to(dev)
+            vsc = block_scales(kp.shape[0], wl.num_kv_heads, base, args.seed + 62).to(dev)
+        else:
+            ksc = head_scales(wl.num_kv_heads, base).to(dev)
+            vsc = head_scales(wl.num_kv_heads, base).flip(0).contiguous().to(dev)
+    write_quant = pa.pa_reshape_and_cache_quant_blocks if per_block else pa.pa_reshape_and_cache_quant
     if kv8:
         ws = pa.alloc_workspace(B, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, max_ctx, P, dev,
                                 fp8=True)
     fused = not args.unfused and not kv8 and appends_at_last_positions(wl)
-    share = (quant or not kv8) and (args.share == "on" or
+    share = ((quant and not per_block) or not kv8) and (args.share == "on" or
                                      (args.share == "auto" and wl.kv_bytes_unique() < wl.kv_bytes()))
     if share:
         ws = pa.alloc_workspace(B, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, max_ctx, P, dev,
@@ -348,7 +362,7 @@ def run_ours(args, world, rank, local, extras=True):
         krows = kp.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
         vrows = vp.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
         if quant:
-            pa.pa_reshape_and_cache_quant(krows, vrows, k8, v8, all_slots, qfmt, ksc, vsc)
+            write_quant(krows, vrows, k8, v8, all_slots, qfmt, ksc, vsc)
         else:
             pa.pa_reshape_and_cache_fp8(krows, vrows, k8, v8, all_slots, FP8_SCALE, FP8_SCALE)
         del krows, vrows
@@ -363,7 +377,7 @@ def run_ours(args, world, rank, local, extras=True):
         if d["pairs"].shape[0]:
             pa.pa_copy_blocks([kp, vp], d["pairs"])
         if quant:
-            pa.pa_reshape_and_cache_quant(d["k"], d["v"], kp, vp, d["slots"], qfmt, ksc, vsc)
+            write_quant(d["k"], d["v"], kp, vp, d["slots"], qfmt, ksc, vsc)
         elif kv8:
             pa.pa_reshape_and_cache_fp8(d["k"], d["v"], kp, vp, d["slots"], FP8_SCALE, FP8_SCALE)
         elif fused:
@@ -376,6 +390,9 @@ def run_ours(args, world, rank, local, extras=True):
         if quant and share:
             pa.pa_decode_shared_quant(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, qfmt,
                                       ksc, vsc, P, ws)
+        elif quant and per_block:
+            pa.pa_decode_quant_blocks(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, qfmt, ksc,
+                                      vsc, P, ws)
         elif quant:
             pa.pa_decode_quant(d["out"], d["q"], kp, vp, d["tables"], d["ctx"], wl.scale, max_ctx, qfmt, ksc, vsc,
                                P, ws)
@@ -458,7 +475,8 @@ def run_ours(args, world, rank, local, extras=True):
     result = {
         "metric": METRIC, "value": value, "unit": "seqs/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": (f"{qfmt} KV cache (per-head scales), {wl.dtype} q/out" if quant else
+        "vs_baseline": None, "dtype": (f"{qfmt} KV cache (per-block scales), {wl.dtype} q/out" if per_block else
+                                       f"{qfmt} KV cache (per-head scales), {wl.dtype} q/out" if quant else
                                        f"e4m3 KV cache, {wl.dtype} q/out" if kv8 else wl.dtype),
         "data": "synthetic (seeded N(0,1) K/V/Q, shuffled block pool)",
         "config": describe(wl),
@@ -473,7 +491,10 @@ def run_ours(args, world, rank, local, extras=True):
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "kernel": ("pa_decode_shared_quant call (grouping plan + attention launches; split merge "
                                 "in a launch of its own)" if quant and share else
-                                "pa_decode_quant call (plan + attention launches; split merge fused)" if quant else
+                                "pa_decode_quant_blocks call (plan + attention launches; split merge fused up to 16 "
+                                "partitions)" if per_block else
+                                "pa_decode_quant call (plan + attention launches; split merge fused up to 16 "
+                                "partitions)" if quant else
                                 "pa_decode_fp8 call (plan + attention launches; split merge fused)" if kv8 else
                                 "pa_decode_shared call (grouping plan + attention launches; cache write fused, "
                                 "split merge in a launch of its own)" if share and fused else
@@ -488,7 +509,8 @@ def run_ours(args, world, rank, local, extras=True):
                                                  + ("" if args.partition is None else f"@P{args.partition}"))},
         "gpu_launches": launches,
         "step": ("pa_copy_blocks (if any), pa_reshape_and_cache_quant, pa_decode_shared_quant" if quant and share
-                 else "pa_copy_blocks (if any), pa_reshape_and_cache_quant, pa_decode_quant" if quant else
+                 else "pa_copy_blocks (if any), pa_reshape_and_cache_quant_blocks, pa_decode_quant_blocks"
+                 if per_block else "pa_copy_blocks (if any), pa_reshape_and_cache_quant, pa_decode_quant" if quant else
                  "pa_copy_blocks (if any), pa_reshape_and_cache_fp8, pa_decode_fp8" if kv8 else
                  "pa_copy_blocks (if any), pa_reshape_and_cache of extra tokens (if any), pa_decode_shared with "
                  "the new tokens" if share and fused else
@@ -508,7 +530,11 @@ def run_ours(args, world, rank, local, extras=True):
         unflushed["decode_kv_gbs"] = kv_unique / (unflushed["decode_ms"] * 1e-3) / 1e9
         unflushed["decode_kv_gbs_logical"] = kv_bytes / (unflushed["decode_ms"] * 1e-3) / 1e9
         result["unflushed"] = unflushed
-    if quant:
+    if per_block:
+        result["config"]["kv_cache"] = (f"{qfmt} codes, one scale per (block, KV head): {base / 10:g} to "
+                                        f"{base * 10:g} (100x), drawn per block and head")
+        result["config"]["kv_bytes_per_step"] = int(kv_bytes)
+    elif quant:
         result["config"]["kv_cache"] = (f"{qfmt} codes, one scale per KV head: {base / 10:g} to {base * 10:g} "
                                         "(100x), keys and values in opposite head order")
         result["config"]["kv_bytes_per_step"] = int(kv_bytes)
