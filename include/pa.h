@@ -352,6 +352,16 @@ PA_API pa_status pa_reshape_and_cache_quant_blocks(const void *k, const void *v,
                                                    int head_dim, int block_size, int num_blocks, int dtype,
                                                    int kv_format, const float *k_scales, const float *v_scales,
                                                    pa_stream_t stream);
+/* pa_decode_shared_quant with one scale per (physical block, KV head), as
+ * above: the shared units stream a block once for the whole group with that
+ * block's scales (the blocks are the same physical blocks for every member). */
+PA_API pa_status pa_decode_shared_quant_blocks(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                               const int32_t *block_tables, const int32_t *context_lens,
+                                               int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                               int block_size, int max_blocks_per_seq, int num_blocks,
+                                               int max_context_len, float scale, int dtype, int kv_format,
+                                               const float *k_scales, const float *v_scales, int partition_size,
+                                               void *workspace, size_t workspace_bytes, pa_stream_t stream);
 PA_API pa_status pa_decode_quant_blocks(void *out, const void *q, const void *k_pool, const void *v_pool,
                                         const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                                         int num_heads, int num_kv_heads, int head_dim, int block_size,

@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_quant.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P,
                                       _I, _P, _SZ, _P]
         L.pa_decode_quant_blocks.argtypes = L.pa_decode_quant.argtypes
+        L.pa_decode_shared_quant_blocks.restype = _I
+        L.pa_decode_shared_quant_blocks.argtypes = L.pa_decode_quant.argtypes
         L.pa_decode_shared_quant.restype = _I
         L.pa_decode_shared_quant.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                                              _P, _P, _I, _P, _SZ, _P]
@@ -422,6 +424,31 @@ def pa_decode_shared_quant(out, q, k_pool, v_pool, block_tables, context_lens, s
         _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
         B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
         KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv), _scales(v_scales, "v_scales", Hkv),
+        int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return out
+
+
+def pa_decode_shared_quant_blocks(out, q, k_pool, v_pool, block_tables, context_lens, scale, max_context_len,
+                                  kv_format, k_scales, v_scales, partition_size=0, workspace=None,
+                                  stream=None) -> torch.Tensor:
+    """pa_decode_shared_quant with one scale per (physical block, KV head):
+    k_scales, v_scales float32 CUDA tensors [NB][Hkv]."""
+    B, H, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch between q, out and the pools")
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("8-bit pools must be uint8 tensors of codes")
+    if q.dtype not in _DTYPES or out.dtype != q.dtype:
+        raise ValueError("q and out must share one dtype, fp16 or bf16")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, Hkv, D, bs, max_context_len, partition_size, q.device, shared=True)
+    _check(lib().pa_decode_shared_quant_blocks(
+        _cuda(out, "out"), _cuda(q, "q"), _cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"),
+        _cuda(block_tables, "block_tables", torch.int32), _cuda(context_lens, "context_lens", torch.int32),
+        B, H, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(scale), _DTYPES[q.dtype],
+        KV_FORMATS[kv_format], _scales(k_scales, "k_scales", Hkv, NB), _scales(v_scales, "v_scales", Hkv, NB),
         int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream)))
     return out

@@ -174,6 +174,16 @@ pa_status dispatch_kv8(pa::DecodeParams &p, int group, cudaStream_t s, bool int8
                      : dispatch_group_fp8<D, T, false, 0>(p, group, s);
 }
 
+// Shared-prefix units over an 8-bit cache, by code format and scale granularity.
+template <int D, typename T>
+pa_status dispatch_shared_kv8(pa::DecodeParams &p, int group, cudaStream_t s, bool int8, bool block_scales) {
+    if (int8)
+        return block_scales ? dispatch_group_shared_kv8<D, T, true, 2>(p, group, s)
+                            : dispatch_group_shared_kv8<D, T, true, 1>(p, group, s);
+    return block_scales ? dispatch_group_shared_kv8<D, T, false, 2>(p, group, s)
+                        : dispatch_group_shared_kv8<D, T, false, 1>(p, group, s);
+}
+
 pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v_new, const void *k_pool,
                       const void *v_pool, const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                       int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
@@ -281,16 +291,11 @@ pa_status decode_impl(void *out, const void *q, const void *k_new, const void *v
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int group = num_heads / num_kv_heads;
     if (kv8 && shared) {
-        const bool d128 = head_dim == 128, f16 = dtype == PA_F16;
-        if (int8)
-            return d128 ? (f16 ? dispatch_group_shared_kv8<128, __half, true>(p, group, s)
-                               : dispatch_group_shared_kv8<128, __nv_bfloat16, true>(p, group, s))
-                        : (f16 ? dispatch_group_shared_kv8<64, __half, true>(p, group, s)
-                               : dispatch_group_shared_kv8<64, __nv_bfloat16, true>(p, group, s));
-        return d128 ? (f16 ? dispatch_group_shared_kv8<128, __half, false>(p, group, s)
-                           : dispatch_group_shared_kv8<128, __nv_bfloat16, false>(p, group, s))
-                    : (f16 ? dispatch_group_shared_kv8<64, __half, false>(p, group, s)
-                           : dispatch_group_shared_kv8<64, __nv_bfloat16, false>(p, group, s));
+        if (head_dim == 128)
+            return dtype == PA_F16 ? dispatch_shared_kv8<128, __half>(p, group, s, int8, block_scales)
+                                   : dispatch_shared_kv8<128, __nv_bfloat16>(p, group, s, int8, block_scales);
+        return dtype == PA_F16 ? dispatch_shared_kv8<64, __half>(p, group, s, int8, block_scales)
+                               : dispatch_shared_kv8<64, __nv_bfloat16>(p, group, s, int8, block_scales);
     }
     if (kv8) {
         // Scales: per (block, KV head) 2, per KV head 1, per tensor 0 (E4M3 only).
@@ -378,6 +383,22 @@ pa_status pa_decode_shared_quant(void *out, const void *q, const void *k_pool, c
                        num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
                        dtype, partition_size, workspace, workspace_bytes, stream, true, 1.f, 1.f, true,
                        kv_format == PA_KV_INT8, k_scales, v_scales);
+}
+
+pa_status pa_decode_shared_quant_blocks(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                        const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                        int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                        int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                                        int dtype, int kv_format, const float *k_scales, const float *v_scales,
+                                        int partition_size, void *workspace, size_t workspace_bytes,
+                                        pa_stream_t stream) {
+    g_last_error.clear();
+    if (kv_format != PA_KV_E4M3 && kv_format != PA_KV_INT8) return fail(PA_ERR_INVALID, "kv_format %d", kv_format);
+    if (num_seqs > 0 && (!k_scales || !v_scales)) return fail(PA_ERR_INVALID, "null scale array");
+    return decode_impl(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale,
+                       dtype, partition_size, workspace, workspace_bytes, stream, true, 1.f, 1.f, true,
+                       kv_format == PA_KV_INT8, k_scales, v_scales, true);
 }
 
 pa_status pa_reshape_and_cache(const void *k, const void *v, void *k_pool, void *v_pool, const int64_t *slot_mapping,

@@ -482,7 +482,6 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                          const __grid_constant__ CUtensorMap tm_v) {
     static_assert(!I8 || KV8, "INT8 codes are an 8-bit cache");
     static_assert(!HS || KV8, "per-head and per-block scales are an 8-bit cache's");
-    static_assert(HS != 2 || !SHARED, "per-block scales: units of one sequence");
     using Gm = MmaGeo<D, G, KV8, mma_tile_rows<D, KV8, SHARED>()>;
     constexpr int TR = Gm::TR;   // tokens of an item
     constexpr int NT = TR / 16;  // its 16-token MMA sub-tiles
@@ -894,19 +893,20 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                 }
             }
             // s[j][0], s[j][1]: token 16j + g8, heads h0, h1; s[j][2], s[j][3]: token 16j + g8 + 8.
-            float x[NT][4], vr[NT];
+            float x[NT][4], vr[NT], ksc[NT];
             float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
                 float uqj = uq, kcj0 = kc0, kcj1 = kc1;
                 vr[j] = 1.f;
+                ksc[j] = 1.f;
                 if constexpr (HS == 2) {  // the scales of the sub-tile's block
                     const int bj = (TR * k + 16 * j) / bs;
-                    const float ksc = __shfl_sync(FULL_MASK, kbl, bj & 31);
+                    ksc[j] = __shfl_sync(FULL_MASK, kbl, bj & 31);
                     vr[j] = __shfl_sync(FULL_MASK, vbl, bj & 31) * ivmax;
-                    uqj = uq * ksc;
-                    kcj0 = kc0 * ksc;
-                    kcj1 = kc1 * ksc;
+                    uqj = uq * ksc[j];
+                    kcj0 = kc0 * ksc[j];
+                    kcj1 = kc1 * ksc[j];
                 }
                 const bool lo_in = 16 * j + g8 < valid, hi_in = 16 * j + g8 + 8 < valid;
                 x[j][0] = lo_in ? fmaf(s[j][0] + s2[j][0], uqj, kcj0) : -INFINITY;
@@ -966,10 +966,12 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
             if constexpr (SHARED) {
                 if (two) {
                     const bool v_lo = g8 < valid, v_hi = g8 + 8 < valid;
-                    const float y0 = v_lo ? fmaf(u[0] + u2[0], uq, kd0) : -INFINITY;
-                    const float y1 = v_lo ? fmaf(u[1] + u2[1], uq, kd1) : -INFINITY;
-                    const float y2 = v_hi ? fmaf(u[2] + u2[2], uq, kd0) : -INFINITY;
-                    const float y3 = v_hi ? fmaf(u[3] + u2[3], uq, kd1) : -INFINITY;
+                    // (per-block scales: the tile's key scale, as for the first half)
+                    const float uqb = uq * ksc[0], kdb0 = kd0 * ksc[0], kdb1 = kd1 * ksc[0];
+                    const float y0 = v_lo ? fmaf(u[0] + u2[0], uqb, kdb0) : -INFINITY;
+                    const float y1 = v_lo ? fmaf(u[1] + u2[1], uqb, kdb1) : -INFINITY;
+                    const float y2 = v_hi ? fmaf(u[2] + u2[2], uqb, kdb0) : -INFINITY;
+                    const float y3 = v_hi ? fmaf(u[3] + u2[3], uqb, kdb1) : -INFINITY;
                     const bool raise2 = (hw0 && !(fmaxf(y0, y2) <= N0 + LAZY_MAX_LOG2)) ||
                                         (hw1 && !(fmaxf(y1, y3) <= N1 + LAZY_MAX_LOG2));
                     if (__any_sync(FULL_MASK, raise2)) {
@@ -994,10 +996,19 @@ __global__ void __launch_bounds__(mma_max_warps<D, G, KV8, SHARED>() * 32, 1)
                     }
                     const float q0 = hw0 ? exp2f(y0 - N0) : 0.f, q1 = hw1 ? exp2f(y1 - N1) : 0.f;
                     const float q2 = hw0 ? exp2f(y2 - N0) : 0.f, q3 = hw1 ? exp2f(y3 - N1) : 0.f;
-                    const uint32_t z_lo = Elem<MT>::pack(q0, q1), z_hi = Elem<MT>::pack(q2, q3);
-                    const float2 r_lo = Elem<MT>::pair(z_lo), r_hi = Elem<MT>::pair(z_hi);
-                    m0s += r_lo.x + r_hi.x;
-                    m1s += r_lo.y + r_hi.y;
+                    uint32_t z_lo, z_hi;
+                    if constexpr (HS == 2) {  // weighted by the tile's value scale, as for the first half
+                        z_lo = Elem<MT>::pack(q0 * vr[0], q1 * vr[0]);
+                        z_hi = Elem<MT>::pack(q2 * vr[0], q3 * vr[0]);
+                        m0s += q0 + q2;
+                        m1s += q1 + q3;
+                    } else {
+                        z_lo = Elem<MT>::pack(q0, q1);
+                        z_hi = Elem<MT>::pack(q2, q3);
+                        const float2 r_lo = Elem<MT>::pair(z_lo), r_hi = Elem<MT>::pair(z_hi);
+                        m0s += r_lo.x + r_hi.x;
+                        m1s += r_lo.y + r_hi.y;
+                    }
                     pc0 = movmatrix_trans(z_lo);
                     pc1 = movmatrix_trans(z_hi);
                 }

@@ -310,14 +310,15 @@ pa_status dispatch_group_shared(pa::DecodeParams &p, int group, cudaStream_t str
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }
 
-// Shared-prefix units over an 8-bit cache (one scale per KV head).
-template <int D, typename T, bool I8>
+// Shared-prefix units over an 8-bit cache (one scale per KV head, HS 1, or
+// per (block, KV head), HS 2).
+template <int D, typename T, bool I8, int HS = 1>
 pa_status dispatch_group_shared_kv8(pa::DecodeParams &p, int group, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_decode_mma<D, 1, T, true, true, I8, 1>(p, stream);
-        case 2: return launch_decode_mma<D, 2, T, true, true, I8, 1>(p, stream);
-        case 4: return launch_decode_mma<D, 4, T, true, true, I8, 1>(p, stream);
-        case 8: return launch_decode_mma<D, 8, T, true, true, I8, 1>(p, stream);
+        case 1: return launch_decode_mma<D, 1, T, true, true, I8, HS>(p, stream);
+        case 2: return launch_decode_mma<D, 2, T, true, true, I8, HS>(p, stream);
+        case 4: return launch_decode_mma<D, 4, T, true, true, I8, HS>(p, stream);
+        case 8: return launch_decode_mma<D, 8, T, true, true, I8, HS>(p, stream);
     }
     return fail(PA_ERR_UNSUPPORTED, "group size %d", group);
 }

@@ -4,7 +4,9 @@ Each case draws the batch size, query heads per KV head, KV heads, head size,
 block size, dtype, context lengths (empty, one token, block edges, several
 partitions), the partition size and the entry point: pa_decode,
 pa_decode_append, pa_decode_shared (with and without the fused append),
-pa_decode_fp8, pa_decode_quant in both formats and pa_decode_shared_quant.
+pa_decode_fp8, pa_decode_quant in both formats, pa_decode_shared_quant, and
+the per-(block, KV head) scale entry points pa_decode_quant_blocks and
+pa_decode_shared_quant_blocks.
 Sequences of the shared-prefix cases come in groups whose tables begin with
 the same blocks. Every output row starts as NaN, so a row no kernel writes
 fails; cache writes are compared bit for bit.
@@ -23,11 +25,12 @@ from paged_kv_cache_372_b200 import inputs
 from tests import gpu_harness as H
 from tests.bruteforce import bits_of
 from tests.test_gpu_quant import head_scales, quantise
+from tests.test_gpu_quant_blocks import block_scales, quantise_blocks
 
 pytestmark = pytest.mark.gpu
 
 PATHS = ("plain", "append", "shared", "shared_append", "fp8", "quant_int8", "quant_e4m3", "shared_quant_int8",
-         "shared_quant_e4m3")
+         "shared_quant_e4m3", "blocks_int8", "blocks_e4m3", "shared_blocks_int8")
 CASES = 8 * len(PATHS)
 
 
@@ -131,15 +134,26 @@ def test_random_shape(seed):
             assert H.pools_equal(kpd, vpd, okp, ovp), label
     else:
         fmt = "int8" if path.endswith("int8") else "e4m3"
+        blocks = "blocks" in path
+        base = 0.01 if fmt == "int8" else 0.0375
         if path == "fp8":
             ks = vs = torch.full((Hkv,), 0.0375, dtype=torch.float32)
+        elif blocks:
+            ks, vs = block_scales(NB, Hkv, base, 9300 + seed), block_scales(NB, Hkv, base, 9400 + seed)
         else:
-            base = 0.01 if fmt == "int8" else 0.0375
             ks, vs = head_scales(Hkv, base), head_scales(Hkv, base).flip(0).contiguous()
-        k8, v8 = quantise(kp, ks, fmt), quantise(vp, vs, fmt)
+        if blocks:
+            k8, v8 = quantise_blocks(kp, ks, fmt), quantise_blocks(vp, vs, fmt)
+        else:
+            k8, v8 = quantise(kp, ks, fmt), quantise(vp, vs, fmt)
         k8d, v8d = k8.to(dev), v8.to(dev)
         if path == "fp8":
             pa.pa_decode_fp8(out, qd, k8d, v8d, tab, ctx_d, scale, mx, 0.0375, 0.0375, c["P"])
+        elif path == "shared_blocks_int8":
+            pa.pa_decode_shared_quant_blocks(out, qd, k8d, v8d, tab, ctx_d, scale, mx, fmt, ks.to(dev), vs.to(dev),
+                                             c["P"])
+        elif blocks:
+            pa.pa_decode_quant_blocks(out, qd, k8d, v8d, tab, ctx_d, scale, mx, fmt, ks.to(dev), vs.to(dev), c["P"])
         elif path.startswith("shared"):
             pa.pa_decode_shared_quant(out, qd, k8d, v8d, tab, ctx_d, scale, mx, fmt, ks.to(dev), vs.to(dev), c["P"])
         else:

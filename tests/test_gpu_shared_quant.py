@@ -161,3 +161,67 @@ def test_shared_quant_rejects():
         pa.pa_decode_shared_quant(torch.empty_like(q), q, k8.half(), k8.half(), tab, ctx, 0.1, 1, "e4m3", s, s)
     with pytest.raises(ValueError):
         pa.pa_decode_shared_quant(torch.empty_like(q), q, k8, k8.clone(), tab, ctx, 0.1, 1, "int8", s[:4], s)
+
+
+def quant_case_blocks(case, fmt, seed):
+    """As quant_case with one scale per (block, KV head), spanning 100x."""
+    from tests.test_gpu_quant_blocks import block_scales, quantise_blocks
+    kp, vp = case["kp"], case["vp"]
+    bad = torch.isnan(kp)
+    NB, Hkv = kp.shape[0], kp.shape[1]
+    base = 0.01 if fmt == "int8" else 0.0375
+    ks, vs = block_scales(NB, Hkv, base, seed), block_scales(NB, Hkv, base, seed + 1)
+    k8 = quantise_blocks(torch.nan_to_num(kp), ks, fmt)
+    v8 = quantise_blocks(torch.nan_to_num(vp), vs, fmt)
+    if fmt == "e4m3":
+        k8[bad] = 0x7F
+        v8[bad] = 0x7F
+    return k8, v8, ks, vs
+
+
+def run_shared_quant_blocks(case, fmt, k8, v8, ks, vs, P):
+    dev = torch.device("cuda")
+    q = case["q"].to(dev)
+    out = torch.full_like(q, float("nan"))
+    mx = int(case["ctx"].max())
+    pa.pa_decode_shared_quant_blocks(out, q, k8.to(dev), v8.to(dev), torch.from_numpy(case["tables"]).to(dev),
+                                     torch.from_numpy(case["ctx"]).to(dev), case["scale"], mx, fmt, ks.to(dev),
+                                     vs.to(dev), P)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    return out
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("shape", SHAPES)
+def test_shared_quant_block_scales_match_oracle(shape, fmt):
+    """Shared units over an 8-bit cache with one scale per (block, KV head):
+    the group's shared blocks carry their own scales, for every member."""
+    heads, kv_heads, D, bs, dtype = shape
+    case = sharing_case(31 + bs + D, heads, kv_heads, D, bs, dtype, False)
+    k8, v8, ks, vs = quant_case_blocks(case, fmt, 8)
+    ref = oracle_quant(case, fmt, k8, v8, ks, vs)
+    for P in (0, 2 * bs):
+        out = run_shared_quant_blocks(case, fmt, k8, v8, ks, vs, P)
+        assert not torch.isnan(out).any()
+        err = H.max_err(out, ref)
+        assert err <= H.TOL[dtype], (shape, fmt, P, err)
+        margins.record(f"shared {fmt} per-block {heads}/{kv_heads} D={D} bs={bs} {dtype} P={P or 'auto'}", err,
+                       H.TOL[dtype])
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_shared_quant_block_scales_beam(fmt):
+    from tests.test_gpu_quant_blocks import block_scales, quantise_blocks
+    wl = workloads.build("beam", 0, steps=1)
+    st = wl.steps[0]
+    NB = wl.k_pool.shape[0]
+    ks, vs = block_scales(NB, wl.num_kv_heads, 0.0375, 21), block_scales(NB, wl.num_kv_heads, 0.05, 22)
+    k8, v8 = quantise_blocks(wl.k_pool, ks, fmt), quantise_blocks(wl.v_pool, vs, fmt)
+    case = dict(q=st.q, tables=st.block_tables, ctx=st.context_lens, scale=wl.scale, dtype=wl.dtype,
+                kv_heads=wl.num_kv_heads, bs=wl.block_size)
+    out = run_shared_quant_blocks(case, fmt, k8, v8, ks, vs, 0)
+    ref = oracle_quant(case, fmt, k8, v8, ks, vs)
+    err = H.max_err(out, ref)
+    assert err <= H.TOL[wl.dtype]
+    margins.record(f"shared {fmt} per-block beam {wl.dtype}", err, H.TOL[wl.dtype])
