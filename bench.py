@@ -554,17 +554,20 @@ def run_ours(args, world, rank, local, extras=True):
 # After the default (LLaMA-7B-shaped) line, the Llama-3-8B-shaped GQA batch is
 # timed the same way on the same GPU and reported under its own key, so that
 # one run covers both decode batches the throughput target names.
-SECONDARY = {"llama7b": "llama3_8b"}
+# Workloads timed after the default line, in the same run: the Llama-3-8B GQA
+# batch, the long-context batch at its own 512-token partitions, and the
+# shared-prefix beam batch (each with its own L2 rule).
+SECONDARY = {"llama7b": ("llama3_8b", "long32k", "beam")}
 SECONDARY_STEPS = 300
 
 
-def run_secondary(args, world, rank, local):
-    name = SECONDARY[args.workload]
+def run_secondary(args, world, rank, local, name):
     sub = argparse.Namespace(**vars(args))
     sub.workload, sub.steps = name, min(args.steps, SECONDARY_STEPS)
     r = run_ours(sub, world, rank, local, extras=False)
     keep = ("value", "unit", "steps", "warmup", "ms_per_step", "dtype", "config", "decode_ms",
-            "decode_ms_p10_p50_p90", "decode_kv_gbs", "roofline", "gpu_launches", "clocks", "step")
+            "decode_ms_p10_p50_p90", "decode_kv_gbs", "decode_kv_gbs_logical", "roofline", "gpu_launches",
+            "clocks", "step", "shared_prefix_units", "unflushed", "non_kv_bytes_per_call", "partition_size")
     return {k: r[k] for k in keep if k in r}
 
 
@@ -842,7 +845,8 @@ def main():
         res = run_swap(args, world, rank, local) if args.workload == "swap" else run_ours(args, world, rank, local)
         if (args.workload in SECONDARY and world == 1 and args.kv == "auto" and args.partition is None
                 and not shape_args(args)):
-            res["secondary_workloads"] = {SECONDARY[args.workload]: run_secondary(args, world, rank, local)}
+            res["secondary_workloads"] = {name: run_secondary(args, world, rank, local, name)
+                                          for name in SECONDARY[args.workload]}
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
