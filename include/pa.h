@@ -330,7 +330,8 @@ PA_API pa_status pa_decode_quant(void *out, const void *q, const void *k_pool, c
 
 /*
  * The 8-bit cache with one scale per (physical block, KV head): k_scales and
- * v_scales are fp32 device arrays [num_blocks][num_kv_heads], 4-byte aligned;
+ * v_scales are fp32 device arrays [num_blocks][num_kv_heads] of positive
+ * finite floats (not checked on the device), 4-byte aligned;
  * a token written into block b of KV head h is stored as
  * encode(x / k_scales[b * num_kv_heads + h]) (v_scales for values), and
  * decoding multiplies by the same scale. Otherwise exactly
