@@ -104,7 +104,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
-// ---- bulk copy global -> shared (TMA, no tensor map, no multicast) ----------
+// ---- bulk copy global -> this CTA's shared memory (TMA, no tensor map) -------
 // dst and src 16-byte aligned, bytes a multiple of 16. Completion is counted
 // on the mbarrier as transaction bytes.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,

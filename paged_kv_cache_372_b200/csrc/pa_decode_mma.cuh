@@ -219,7 +219,7 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
     return d;
 }
 
-// Tiled 2-D TMA load of one box {x = column, y = row} (no multicast).
+// Tiled 2-D TMA load of one box {x = column, y = row} into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar,
                                             uint64_t policy) {
     asm volatile(
